@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""DSA decode benchmark on B200: query-tokens/s and the HBM roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full DSA decode step (indexer -> top-k -> sparse MLA [-> LSE
+combine], every layer of the workload) over one batch of synthetic inputs
+resident in HBM.  Rank 0 prints one JSON line.  Under torchrun each rank runs
+its own replica of the workload (independent sequences, no data-path
+collective: weak scaling); the timed region is bracketed by barriers and the
+slowest rank's device time is reported.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA decode query-tokens/s on 1 B200 at 128K ctx; % of HBM roofline"
+UNIT = "query-tokens/s"
+DEFAULT_WORKLOAD = "decode_b32_ctx128k"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(inp):
+    """Roofline bytes of one step: indexer FP8 keys read (once per sequence and
+    indexer layer) + bf16 latent rows gathered (576 x 2 B per selected token,
+    per layer; position-0 reuse gathers one set per sequence)."""
+    import numpy as np
+    vis = inp.q_vis.cpu().numpy().astype(np.int64)
+    qo = inp.q_offsets.cpu().numpy()
+    T = inp.T
+    keys = 0
+    for b in range(inp.B):
+        qv = vis[qo[b]:qo[b + 1]]
+        keys += int((qv[:1] if inp.mtp_index_share else qv).max()) * 128
+    n_groups = (inp.n_layers + inp.index_share - 1) // inp.index_share
+    key_bytes = keys * n_groups
+    sel = np.minimum(vis, inp.topk)
+    if inp.mtp_index_share:
+        sel = sel.reshape(inp.B, T)[:, 0]
+    gather_bytes = int(sel.sum()) * 576 * 2 * inp.n_layers
+    return key_bytes, gather_bytes
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        loaded = [s for s, p in zip(sm, pw) if p is not None and p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def host_subproblem(inp, b):
+    """Host numpy inputs of sequence b alone (for the oracle baseline sample):
+    its keys, its queries and a compact pool of its pages."""
+    import numpy as np
+    from tests._helpers import np_bits
+    T = inp.T
+    so = inp.seq_offsets.cpu().numpy()
+    k0, k1 = int(so[b]), int(so[b + 1])
+    pt = inp.page_table[b].cpu().numpy()
+    pages = pt[pt >= 0]
+    qs = slice(b * T, (b + 1) * T)
+    return {
+        "B": 1, "T": T, "topk": inp.topk, "scale": inp.scale, "num_splits": inp.num_splits,
+        "index_share": inp.index_share, "mtp_index_share": inp.mtp_index_share,
+        "n_layers": inp.n_layers, "seq_offsets": np.array([0, k1 - k0]),
+        "q_vis": np_bits(inp.q_vis[qs]), "page_table": np.arange(len(pages), dtype=np.int32)[None],
+        "indexer": [{"q_idx": np_bits(d["q_idx"][qs]), "w": np_bits(d["w"][qs]),
+                     "k_idx": np_bits(d["k_idx"][k0:k1])} for d in inp.indexer],
+        "layers": [{"q": np_bits(L["q"][qs]),
+                    "pool": np_bits(L["pool"][__import__("torch").from_numpy(pages).long().to(L["pool"].device)])}
+                   for L in inp.layers],
+    }
+
+
+def oracle_sample(inp, seconds):
+    """Time the oracle as it stands on whole sequences of the workload until
+    about `seconds` of CPU work is done; returns (queries/s, sample text, cores)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    done_q, spent, seqs = 0, 0.0, 0
+    for b in range(inp.B):
+        sub = host_subproblem(inp, b)
+        t0 = time.perf_counter()
+        O.decode_step(sub)
+        spent += time.perf_counter() - t0
+        done_q += inp.T
+        seqs += 1
+        if spent >= seconds:
+            break
+    return done_q / spent, f"{seqs} of {inp.B} sequences ({done_q} query tokens, all layers), {spent:.1f} s", cores
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import sparse_attention_decode_lightning_b200 as dsa
+    from sparse_attention_decode_lightning_b200.build import build
+    from synth import get_workload, make_inputs
+
+    build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    wl = get_workload(args.workload)
+    inp = make_inputs(wl, seed=args.seed + rank, device=dev)
+    Q, G, n = inp.Q, inp.index_share, inp.n_layers
+    S = inp.num_splits
+    stream = torch.cuda.current_stream(dev)
+    ws = dsa.workspace(Q, inp.max_len, inp.topk, S, device=dev)
+    outs = [torch.empty(Q, 128, 512, device=dev) for _ in range(n)]
+    lses = [torch.empty(Q, 128, device=dev) for _ in range(n)]
+    ng = (n + G - 1) // G
+    idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=dev)
+    qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
+    wl_ = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
+    kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
+    qs = [L["q"] for L in inp.layers]
+    pools = [L["pool"] for L in inp.layers]
+    pts = [inp.page_table] * n
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(q_layers=qs, out_layers=outs, lse_layers=lses):
+        dsa.dsa_decode_step(qi, wl_, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B,
+                            inp.max_len, inp.topk, q_layers, pools, pts, inp.scale, out_layers,
+                            lse_layers, idx, ws, index_share=G, mtp_index_share=inp.mtp_index_share,
+                            num_splits=S, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    dsa.dsa_check_error(ws, stream)
+
+    # ---- timed region: K steps, L2 flushed between steps (outside the events)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with Clocks(local_rank) as clk:
+        barrier()
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        barrier()
+        t_wall = time.perf_counter() - t_wall
+    clocks = clk.summary()
+    dsa.dsa_check_error(ws, stream)
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- per-kernel breakdown of the same step, live (decomposed calls, same kernels)
+    scores = torch.empty(Q, ((inp.max_len + 63) // 64) * 64, device=dev)
+    first = inp.mtp_index_share
+    stage = {"indexer": [], "topk": [], "mla": []}
+    for i in range(args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        dsa.dsa_indexer_scores(qi[0], wl_[0], kl[0], inp.seq_offsets, inp.q_offsets, inp.q_vis,
+                               inp.B, inp.max_len, scores, ws, first_only=first, stream=stream)
+        e[1].record(stream)
+        dsa.dsa_topk_select(scores, inp.q_offsets, inp.q_vis, inp.B, inp.max_len, inp.topk,
+                            idx[0], ws, first_only=first, stream=stream)
+        e[2].record(stream)
+        dsa.dsa_sparse_mla_decode(qs[0], pools[0], pts[0], inp.q_offsets, inp.q_vis, idx[0], inp.B,
+                                  inp.scale, outs[0], lses[0], ws, num_splits=S, stream=stream)
+        e[3].record(stream)
+        stage["_ev"] = stage.get("_ev", []) + [e]
+    torch.cuda.synchronize(dev)
+    for e in stage.pop("_ev"):
+        stage["indexer"].append(e[0].elapsed_time(e[1]))
+        stage["topk"].append(e[1].elapsed_time(e[2]))
+        stage["mla"].append(e[2].elapsed_time(e[3]))
+    dsa.dsa_check_error(ws, stream)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_qi = [t.cpu().pin_memory() if t is not None else None for t in qi]
+        h_w = [t.cpu().pin_memory() if t is not None else None for t in wl_]
+        h_q = [t.cpu().pin_memory() for t in qs]
+        h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        h_lse = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lses]
+        d_qi = [torch.empty_like(t) if t is not None else None for t in qi]
+        d_w = [torch.empty_like(t) if t is not None else None for t in wl_]
+        d_q = [torch.empty_like(t) for t in qs]
+        h2d = sum(t.numel() * t.element_size() for t in h_qi + h_w + h_q if t is not None)
+        d2h = sum(t.numel() * t.element_size() for t in h_out + h_lse)
+
+        def e2e_step():
+            for d, h in zip(d_qi + d_w + d_q, h_qi + h_w + h_q):
+                if h is not None:
+                    d.copy_(h, non_blocking=True)
+            dsa.dsa_decode_step(d_qi, d_w, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B,
+                                inp.max_len, inp.topk, d_q, pools, pts, inp.scale, outs, lses, idx,
+                                ws, index_share=G, mtp_index_share=inp.mtp_index_share,
+                                num_splits=S, stream=stream)
+            for h, d in zip(h_out + h_lse, outs + lses):
+                h.copy_(d, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            e2e_step()
+            ev[i][1].record(stream)
+        barrier()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ev)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": Q * world * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        dsa.dsa_check_error(ws, stream)
+
+    key_b, gat_b = algorithmic_bytes(inp)
+    hbm, hbm_kind = peaks()
+    idx_ms = statistics.mean(stage["indexer"])
+    idx_bytes = key_b // ((n + G - 1) // G)
+    achieved = idx_bytes / (idx_ms / 1e3) / 1e9
+    step_mean_ms = total_ms / args.steps
+    launches_per_step = ng * (1 + 3 + (1 if inp.mtp_index_share else 0)) + n * (1 + (1 if S > 1 else 0))
+    res = {
+        "metric": METRIC, "value": Q * world * args.steps / (total_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_mean_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 indexer, bf16 attention, f32 accumulate", "data": "synthetic",
+        "config": {"workload": wl.name, "B": inp.B, "T": inp.T, "L": wl.L,
+                   "L_range": list(wl.L_range) if wl.L_range else None, "layers": n,
+                   "index_share": G, "mtp_index_share": inp.mtp_index_share, "topk": inp.topk,
+                   "num_splits": S, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (FP8 keys) and a 256 MiB L2 flush before every step"},
+        "roofline": {"bound": "hbm", "kernel": "indexer_kernel", "achieved": achieved, "peak": hbm,
+                     "peak_source": hbm_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None},
+        "step_roofline": {"bytes_per_step": key_b + gat_b, "key_bytes": key_b, "gather_bytes": gat_b,
+                          "achieved_gbs": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9,
+                          "frac_of_measured": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9 / hbm,
+                          "frac_of_8tbs": (key_b + gat_b) / (step_mean_ms / 1e3) / 8e12},
+        "stages_ms": {k: statistics.mean(v) for k, v in stage.items()},
+        "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, cores = oracle_sample(inp, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    return res
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The fp64 CPU oracle as it stands, on whole sequences of the workload
+    drawn on the host (one sequence per step)."""
+    import oracle as O
+    from synth import get_workload, make_inputs
+    wl = get_workload(args.workload)
+    one = get_workload(args.workload, B=1)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    inp = make_inputs(one, seed=args.seed, device="cpu")
+    from tests._helpers import oracle_inputs
+    host = oracle_inputs(inp)
+    for _ in range(args.warmup):
+        O.decode_step(host)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.decode_step(host)
+    dt = time.perf_counter() - t0
+    v = inp.Q * args.steps / dt
+    return {
+        "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": wl.name, "sample": "one sequence of the workload per step"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps x 1 sequence ({inp.Q} query tokens, all layers)"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+/*
+ * dsa.h -- C ABI of libdsa: DeepSeek Sparse Attention (DSA) decode on B200.
+ *
+ * What the library computes (pages cited by title and section):
+ *   "大语言模型结构总览" (LLM structure overview), section 2.2 DeepSeek-V3.2:
+ *     DSA is a two-stage select-then-attend pipeline.  A lightning indexer
+ *     (64 heads, head dim 128, FP8) scores every prior token of a query; a
+ *     token selector keeps the k = 2048 best tokens; MLA attention in MQA mode
+ *     then runs over those tokens only.  Paged and non-paged forms exist.
+ *   Same page, section 2.1 DeepSeek-V3: one cached latent per token, kv rank
+ *     512 plus a 64-d RoPE part (576 values), 128 attention heads.
+ *   Same page, section 7.2 GLM-5.2 / Figure 7-2: IndexShare -- one indexer per
+ *     group of sparse layers; the following layers reuse its top-k indices.
+ *   "GLM-5.2 推理部署" (inference deployment), MTP draft + verify flow: top-K
+ *     = 2048 indices computed once and reused across the MTP positions.
+ *
+ * Definitions used throughout (readings where the pages give no formula):
+ *   indexer score   I[q,s] = sum_{h<64} w[q,h] * max(0, sum_{d<128} qi[q,h,d]*K[s,d])
+ *                   qi and K are FP8 e4m3 bytes at scale 1, w is fp32;
+ *   selector        the topk positions s < vis[q] with the largest I[q,s],
+ *                   ties to the lower s; if vis[q] < topk every visible s is
+ *                   kept and the remaining slots hold -1;
+ *   sparse MLA      per head h:  z_j = scale * <q[h,0:576], C[idx_j,0:576]>,
+ *                   O[h] = sum_j softmax_j(z) * C[idx_j,0:512],
+ *                   LSE[h] = ln sum_j exp(z_j)  (empty set: O = 0, LSE = -inf);
+ *   split-K         the selected set is partitioned into num_splits parts, each
+ *                   attended separately, then merged exactly by LSE.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or torch-owned)
+ *     unless a parameter says "host".  The caller allocates and owns every
+ *     buffer, including the workspace; the library allocates nothing and
+ *     keeps no per-call state (it caches TMA descriptors and the SM count).
+ *   - Calls are asynchronous: work is enqueued on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream) and the caller synchronises.
+ *   - Argument checks run on the host before anything is enqueued; a failed
+ *     check returns DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED and enqueues
+ *     nothing.  Nothing traps and nothing throws across the ABI.
+ *   - Values the host cannot check (indices, page ids, lengths living in
+ *     device memory) are checked by the kernels: an out-of-range entry is
+ *     treated as masked and raises a flag in the workspace that
+ *     dsa_check_error() reports as DSA_ERR_DEVICE_BOUNDS.  Device-side waits
+ *     are bounded; an expired wait raises DSA_ERR_TIMEOUT the same way.
+ *   - Layouts are dense row-major with the shapes given; `e4m3` is one byte
+ *     per value (OCP FP8 E4M3), `bf16` two bytes.  Pointers must be 16-byte
+ *     aligned.
+ *   - Query/sequence bookkeeping: the queries of sequence b are the
+ *     contiguous rows q_offsets[b] .. q_offsets[b+1]-1 (at most
+ *     DSA_MAX_Q_PER_SEQ of them); the indexer keys of sequence b are rows
+ *     seq_offsets[b] .. seq_offsets[b+1]-1 of the packed key array, token
+ *     position s of b at row seq_offsets[b] + s.  vis[q] = number of keys
+ *     query q may see (positions 0 .. vis[q]-1, causal).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_PAGE_SIZE 64        /* latent-cache page (tokens) */
+#define DSA_HEADS 128           /* MLA query heads */
+#define DSA_DIM 576             /* latent row: 512 kv-rank + 64 RoPE */
+#define DSA_DIM_V 512           /* value dims (first 512 of the row) */
+#define DSA_IDX_HEADS 64        /* indexer heads */
+#define DSA_IDX_DIM 128         /* indexer head dim */
+#define DSA_MAX_TOPK 2048
+#define DSA_MAX_Q_PER_SEQ 8     /* 1 decode token + up to 7 MTP drafts */
+#define DSA_MAX_BATCH 2048      /* sequences per call */
+#define DSA_MAX_SPLITS 32
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+  DSA_ERR_UNSUPPORTED = 2,   /* shape outside the fixed constants above */
+  DSA_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+  DSA_ERR_DEVICE_BOUNDS = 4, /* a kernel met an out-of-range index/page/length */
+  DSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired */
+  DSA_ERR_WORKSPACE = 6      /* workspace smaller than dsa_workspace_bytes() */
+} dsa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* dsa_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int dsa_version(void);
+
+/*
+ * Bytes of device workspace the calls below need for Q queries, contexts of at
+ * most max_len keys, `topk` selected tokens and `num_splits` split-K parts
+ * (0 = let the library choose).  The workspace holds the fp32 score rows
+ * [Q, max_len], the selector's histograms and candidate lists, the split-K
+ * partial outputs and the device error flag.  The same workspace may be
+ * reused by consecutive calls on one stream; it must be zeroed once
+ * (cudaMemset) before its first use so the error flag starts clear.
+ * Returns 0 for invalid sizes.
+ */
+size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits);
+
+/*
+ * Lightning indexer, scores only  (section 2.2: the indexer stage).
+ *   q_idx  e4m3 [Q,64,128]     w [Q,64] fp32      k_idx e4m3 [total_keys,128]
+ *   seq_offsets int64 [B+1], q_offsets int32 [B+1], q_vis int32 [Q] (device)
+ *   scores fp32 [Q, ld_scores]: row q gets I[q,s] for s < q_vis[q]; other
+ *          entries are left untouched.  ld_scores >= max_len, multiple of 4.
+ *   first_only != 0: only the first query of each sequence is scored.
+ * The FP8 products accumulate in fp32 on the tensor cores.
+ */
+dsa_status dsa_indexer_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                              int64_t total_keys, const int64_t* seq_offsets,
+                              const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                              int max_len, int first_only, float* scores, int ld_scores,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Token selector on given scores  (section 2.2: the token selector stage).
+ *   scores fp32 [Q, ld_scores] (row q, entries s < q_vis[q] are read)
+ *   out_idx int32 [Q, topk]: the selected positions of each query in
+ *           unspecified order, then -1 padding when q_vis[q] < topk.
+ *   out_scores fp32 [Q, topk] or NULL: the score of each selected position
+ *           (-inf in padding slots).
+ *   first_only != 0: only the first query of each sequence (rows
+ *           q_offsets[b]) is selected; other rows are untouched.
+ * Exact: the set equals a full sort by (score desc, position asc); -0 == +0.
+ * Scores must not be NaN.  ws: dsa_workspace_bytes(Q, ld_scores, topk, 1) bytes.
+ */
+dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_offsets,
+                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           int first_only, int32_t* out_idx, float* out_scores,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Indexer + selector in one call  (section 2.2, both stages).  Arguments as
+ * above; scores live in the workspace (dsa_workspace_bytes(Q, max_len, topk, 1)
+ * bytes at least).  With first_only != 0 (IndexShare on
+ * MTP) the first query of each sequence is scored and selected and its index
+ * row is copied to every other query of the sequence.
+ */
+dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                            int64_t total_keys, const int64_t* seq_offsets,
+                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                            int max_len, int topk, int first_only, int32_t* out_idx,
+                            float* out_scores, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse MLA decode in absorbed-MQA form over the selected tokens
+ * (section 2.2: MLA in MQA mode; section 2.1: 576-d latent, 128 heads).
+ *   q          bf16 [Q,128,576]  absorbed queries (512 latent + 64 RoPE)
+ *   kv_pool    bf16 [num_pages,64,576]  paged latent cache shared by all heads
+ *   page_table int32 [B,max_pages]: page of token s of sequence b is
+ *              page_table[b*max_pages + s/64], row s%64 in that page.  A
+ *              non-paged cache is the identity table.
+ *   idx        int32 [Q,topk]: token positions (any order), -1 = skip.
+ *   scale      softmax scale applied to the 576-d dot product.
+ *   num_splits split-K parts (1..DSA_MAX_SPLITS, 0 = library's choice); the
+ *              idx row is cut into equal-count parts merged exactly by LSE.
+ *   out        fp32 [Q,128,512]      lse fp32 [Q,128] (natural log)
+ * Entries with idx >= q_vis[q], a page id outside [0,num_pages) or a page
+ * slot beyond max_pages are skipped and flagged (DSA_ERR_DEVICE_BOUNDS).
+ * ws: at least dsa_workspace_bytes(Q, 1, topk, num_splits) bytes.
+ */
+dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
+                                 const int32_t* page_table, int max_pages,
+                                 const int32_t* q_offsets, const int32_t* q_vis,
+                                 const int32_t* idx, int B, int Q, int topk, float scale,
+                                 int num_splits, float* out, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Merge of split-K partial attentions (exact LSE combine).
+ *   o_parts fp32 [Q,S,128,512], lse_parts fp32 [Q,S,128] (-inf = empty part)
+ *   out fp32 [Q,128,512], lse fp32 [Q,128].
+ */
+dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S,
+                           float* out, float* lse, void* stream);
+
+/*
+ * One DSA decode step over n_layers sparse layers  (section 2.2 pipeline;
+ * section 7.2 IndexShare; MTP flow of the inference page for IndexShare on
+ * MTP).  Every pointer array below is a HOST array of n_layers device
+ * pointers.
+ *   index_share      layers per indexer group G >= 1: layer l uses the top-k
+ *                    of the indexer of layer G*(l/G); only those layers' entries
+ *                    of q_idx_layers / w_layers / k_idx_layers are read.
+ *                    G = 4 is GLM-5.2's IndexShare; G = 1 runs every indexer.
+ *   mtp_index_share  != 0: the first query of each sequence supplies the
+ *                    top-k of all its queries (draft positions reuse step 1).
+ *   idx_out          int32 [ceil(n_layers/G), Q, topk]: the index rows used.
+ *   out_layers / lse_layers: per layer fp32 [Q,128,512] / [Q,128].
+ * Other arguments as in dsa_indexer_topk and dsa_sparse_mla_decode.
+ */
+dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
+                           const uint8_t* const* q_idx_layers, const float* const* w_layers,
+                           const uint8_t* const* k_idx_layers, int64_t total_keys,
+                           const int64_t* seq_offsets, const int32_t* q_offsets,
+                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           const void* const* q_layers, const void* const* pool_layers,
+                           int num_pages, const int32_t* const* page_table_layers,
+                           int max_pages, float scale, int num_splits,
+                           float* const* out_layers, float* const* lse_layers,
+                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, reads and clears the workspace's device error flag.
+ * Returns DSA_OK, DSA_ERR_DEVICE_BOUNDS, DSA_ERR_TIMEOUT or DSA_ERR_CUDA.
+ */
+dsa_status dsa_check_error(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */

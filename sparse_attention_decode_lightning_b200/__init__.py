@@ -1,0 +1,176 @@
+"""Thin Python binding of libdsa (DSA decode on B200, sm_100a).
+
+Argument marshalling only: every function below forwards torch tensors'
+device pointers to the C ABI declared in include/dsa.h, under the same name,
+and raises DSAError on a non-zero status.  No step of the computation runs in
+Python, and there is no fallback: if libdsa.so is missing, loading fails.
+"""
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+PAGE_SIZE = 64
+HEADS = 128
+DIM = 576
+DIM_V = 512
+IDX_HEADS = 64
+IDX_DIM = 128
+MAX_TOPK = 2048
+MAX_Q_PER_SEQ = 8
+
+STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_CUDA",
+          4: "DSA_ERR_DEVICE_BOUNDS", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_WORKSPACE"}
+
+# name -> (restype, argtypes) of every exported entry point
+_P, _I, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_PP = ctypes.POINTER(ctypes.c_void_p)
+SIGNATURES = {
+    "dsa_status_string": (ctypes.c_char_p, [_I]),
+    "dsa_version": (_I, []),
+    "dsa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "dsa_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _SZ, _P]),
+    "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P,
+                                   _SZ, _P]),
+    "dsa_lse_combine": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _PP, _PP,
+                             _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
+    "dsa_check_error": (_I, [_P, _P]),
+}
+
+_lib = None
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa.so (built in-tree by build.py); fails loudly if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_attention_decode_lightning_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libdsa takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libdsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise DSAError(status, where)
+
+
+def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = None if t is None else _ptr(t).value
+    return arr
+
+
+def dsa_version() -> int:
+    return lib().dsa_version()
+
+
+def dsa_status_string(s: int) -> str:
+    return lib().dsa_status_string(s).decode()
+
+
+def dsa_workspace_bytes(Q: int, max_len: int, topk: int, num_splits: int = 0) -> int:
+    return lib().dsa_workspace_bytes(Q, max_len, topk, num_splits)
+
+
+def workspace(Q: int, max_len: int, topk: int, num_splits: int = 0, device="cuda") -> torch.Tensor:
+    """A zeroed device workspace of dsa_workspace_bytes(...) bytes."""
+    n = dsa_workspace_bytes(Q, max_len, topk, num_splits)
+    if n == 0:
+        raise DSAError(1, "dsa_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def dsa_indexer_scores(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len, scores, ws,
+                       first_only=False, stream=None):
+    _check(lib().dsa_indexer_scores(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
+        _ptr(q_vis), B, q_idx.shape[0], max_len, int(first_only), _ptr(scores), scores.shape[1],
+        _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_scores")
+
+
+def dsa_topk_select(scores, q_offsets, q_vis, B, max_len, topk, out_idx, ws, out_scores=None,
+                    first_only=False, stream=None):
+    _check(lib().dsa_topk_select(
+        _ptr(scores), scores.shape[1], _ptr(q_offsets), _ptr(q_vis), B, scores.shape[0], max_len,
+        topk, int(first_only), _ptr(out_idx), _ptr(out_scores), _ptr(ws), ws.numel(),
+        _stream(stream)), "dsa_topk_select")
+
+
+def dsa_indexer_topk(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len, topk, out_idx,
+                     ws, out_scores=None, first_only=False, stream=None):
+    _check(lib().dsa_indexer_topk(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
+        _ptr(q_vis), B, q_idx.shape[0], max_len, topk, int(first_only), _ptr(out_idx),
+        _ptr(out_scores), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
+
+
+def dsa_sparse_mla_decode(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scale, out, lse, ws,
+                          num_splits=0, stream=None):
+    _check(lib().dsa_sparse_mla_decode(
+        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
+        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], idx.shape[1], float(scale),
+        num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+        "dsa_sparse_mla_decode")
+
+
+def dsa_lse_combine(o_parts, lse_parts, out, lse, stream=None):
+    Q, S = lse_parts.shape[0], lse_parts.shape[1]
+    _check(lib().dsa_lse_combine(_ptr(o_parts), _ptr(lse_parts), Q, S, _ptr(out), _ptr(lse),
+                                 _stream(stream)), "dsa_lse_combine")
+
+
+def dsa_decode_step(q_idx_layers, w_layers, k_idx_layers, seq_offsets, q_offsets, q_vis, B,
+                    max_len, topk, q_layers, pool_layers, page_table_layers, scale, out_layers,
+                    lse_layers, idx_out, ws, index_share=1, mtp_index_share=False, num_splits=0,
+                    stream=None):
+    """Per-layer lists; entries of the indexer lists for non-indexer layers may be None."""
+    n = len(q_layers)
+    lead = next(t for t in k_idx_layers if t is not None)
+    _check(lib().dsa_decode_step(
+        n, index_share, int(mtp_index_share), _ptr_array(q_idx_layers), _ptr_array(w_layers),
+        _ptr_array(k_idx_layers), lead.shape[0], _ptr(seq_offsets), _ptr(q_offsets), _ptr(q_vis),
+        B, q_layers[0].shape[0], max_len, topk, _ptr_array(q_layers), _ptr_array(pool_layers),
+        pool_layers[0].shape[0], _ptr_array(page_table_layers), page_table_layers[0].shape[1],
+        float(scale), num_splits, _ptr_array(out_layers), _ptr_array(lse_layers), _ptr(idx_out),
+        _ptr(ws), ws.numel(), _stream(stream)), "dsa_decode_step")
+
+
+def dsa_check_error(ws, stream=None):
+    _check(lib().dsa_check_error(_ptr(ws), _stream(stream)), "dsa_check_error")

@@ -1,0 +1,338 @@
+// Host side of the libdsa C ABI: argument checks, workspace carve-up and the
+// launch sequence of each entry point.  Nothing here computes attention; every
+// step of the path runs in the kernels of the sibling files.
+#include "common.cuh"
+#include "internal.h"
+
+#include <mutex>
+
+namespace dsa {
+
+cudaError_t launch_sparse_mla_simt(const __nv_bfloat16* q, const __nv_bfloat16* pool,
+                                   int num_pages, const int32_t* page_table, int max_pages,
+                                   const int32_t* q_offsets, const int32_t* q_vis,
+                                   const int32_t* idx, int B, int Q, int topk, float scale,
+                                   int S, float* out, float* lse, float* o_part, float* l_part,
+                                   uint32_t* err, cudaStream_t st);
+
+namespace {
+
+constexpr int B200_SMS = 148;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int choose_splits(int Q, int topk, int requested) {
+  int S = requested;
+  if (S <= 0) {
+    // enough (query, split) work units to cover the SMs twice, each with at
+    // least 128 selected rows
+    S = (2 * B200_SMS + Q - 1) / (Q > 0 ? Q : 1);
+    const int cap = topk / 128 > 0 ? topk / 128 : 1;
+    if (S > cap) S = cap;
+    if (S > 16) S = 16;
+  }
+  if (S < 1) S = 1;
+  if (S > DSA_MAX_SPLITS) S = DSA_MAX_SPLITS;
+  if (S > topk) S = topk;
+  return S;
+}
+
+bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* L) {
+  if (Q <= 0 || max_len <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || num_splits < 0 ||
+      num_splits > DSA_MAX_SPLITS)
+    return false;
+  WsLayout w;
+  w.ld = static_cast<int>(align_up(static_cast<size_t>(max_len), 64));
+  w.S = choose_splits(Q, topk, num_splits);
+  size_t off = 0;
+  w.err = off;      off = align_up(off + 256, 256);
+  w.scores = off;   off = align_up(off + static_cast<size_t>(Q) * w.ld * 4, 256);
+  w.hist = off;     off = align_up(off + static_cast<size_t>(Q) * TOPK_BINS * 4, 256);
+  w.meta = off;     off = align_up(off + static_cast<size_t>(Q) * TOPK_META * 4, 256);
+  w.cand = off;     off = align_up(off + static_cast<size_t>(Q) * w.ld * 8, 256);
+  w.cand2 = off;    off = align_up(off + static_cast<size_t>(Q) * w.ld * 8, 256);
+  w.o_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * DSA_DIM_V * 4, 256);
+  w.l_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * 4, 256);
+  w.total = off;
+  *L = w;
+  return true;
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return B200_SMS;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = B200_SMS;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+template <typename T>
+T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+dsa_status check_common(const int64_t* seq_offsets, const int32_t* q_offsets,
+                        const int32_t* q_vis, int B, int Q, int max_len, int topk) {
+  if (!seq_offsets || !q_offsets || !q_vis) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || max_len <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (Q > B * DSA_MAX_Q_PER_SEQ) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status indexer_checks(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                          int64_t total_keys) {
+  if (!q_idx || !w || !k_idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  if (total_keys <= 0) return DSA_ERR_INVALID_ARG;
+  if (total_keys >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                           int64_t total_keys, const int64_t* seq_offsets,
+                           const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                           int max_len, int topk, int first_only, int32_t* out_idx,
+                           float* out_scores, void* ws, const WsLayout& L, cudaStream_t st) {
+  uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
+  float* scores = ws_ptr<float>(ws, L.scores);
+  cudaError_t e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B,
+                                 Q, first_only, scores, L.ld, err, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
+                  out_scores, ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.meta),
+                  ws_ptr<uint64_t>(ws, L.cand), ws_ptr<uint64_t>(ws, L.cand2), err, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  if (first_only) {
+    e = launch_expand_idx(q_offsets, B, Q, topk, out_idx, out_scores, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
+                         const int32_t* page_table, int max_pages, const int32_t* q_offsets,
+                         const int32_t* q_vis, const int32_t* idx, int B, int Q, int topk,
+                         float scale, int S, float* out, float* lse, void* ws,
+                         const WsLayout& L, cudaStream_t st) {
+  uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
+  float* o_part = ws_ptr<float>(ws, L.o_part);
+  float* l_part = ws_ptr<float>(ws, L.l_part);
+  cudaError_t e = launch_sparse_mla(static_cast<const __nv_bfloat16*>(q),
+                                    static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
+                                    page_table, max_pages, q_offsets, q_vis, idx, B, Q, topk,
+                                    scale, S, out, lse, o_part, l_part, err, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  if (S > 1) {
+    e = launch_combine(o_part, l_part, Q, S, out, lse, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages,
+                      const int32_t* page_table, int max_pages, const int32_t* idx, float* out,
+                      float* lse, float scale) {
+  if (!q || !kv_pool || !page_table || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_pool) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
+                              const int32_t* page_table, int max_pages,
+                              const int32_t* q_offsets, const int32_t* q_vis,
+                              const int32_t* idx, int B, int Q, int topk, float scale, int S,
+                              float* out, float* lse, float* o_part, float* l_part,
+                              uint32_t* err, cudaStream_t st) {
+  return launch_sparse_mla_simt(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx,
+                                B, Q, topk, scale, S, out, lse, o_part, l_part, err, st);
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(int s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_DEVICE_BOUNDS: return "DSA_ERR_DEVICE_BOUNDS";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    default: return "DSA_ERR_UNKNOWN";
+  }
+}
+
+int dsa_version(void) { return 100; }
+
+size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits) {
+  WsLayout L;
+  if (!ws_layout(Q, max_len, topk, num_splits, &L)) return 0;
+  return L.total;
+}
+
+dsa_status dsa_indexer_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                              int64_t total_keys, const int64_t* seq_offsets,
+                              const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                              int max_len, int first_only, float* scores, int ld_scores,
+                              void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, 1);
+  if (s != DSA_OK) return s;
+  if ((s = indexer_checks(q_idx, w, k_idx, total_keys)) != DSA_OK) return s;
+  if (!scores || !ws || ld_scores < max_len || (ld_scores & 3) || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return DSA_ERR_WORKSPACE;
+  return cuda_status(launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis,
+                                    B, Q, first_only, scores, ld_scores,
+                                    static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_offsets,
+                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           int first_only, int32_t* out_idx, float* out_scores, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (!scores || !q_offsets || !q_vis || !out_idx || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || max_len <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (ld_scores < max_len || (ld_scores & 3) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  // the selector's candidate lists are sized by the score row stride
+  WsLayout L;
+  if (!ws_layout(Q, ld_scores, topk, 1, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_topk(scores, ld_scores, q_offsets, q_vis, B, Q, max_len, topk,
+                              first_only, out_idx, out_scores, ws_ptr<uint32_t>(ws, L.hist),
+                              ws_ptr<uint32_t>(ws, L.meta), ws_ptr<uint64_t>(ws, L.cand),
+                              ws_ptr<uint64_t>(ws, L.cand2), ws_ptr<uint32_t>(ws, L.err), st);
+  return cuda_status(e);
+}
+
+dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                            int64_t total_keys, const int64_t* seq_offsets,
+                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                            int max_len, int topk, int first_only, int32_t* out_idx,
+                            float* out_scores, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, topk);
+  if (s != DSA_OK) return s;
+  if ((s = indexer_checks(q_idx, w, k_idx, total_keys)) != DSA_OK) return s;
+  if (!out_idx || !ws) return DSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!ws_layout(Q, max_len, topk, 1, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  return do_indexer_topk(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
+                         max_len, topk, first_only, out_idx, out_scores, ws, L,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
+                                 const int32_t* page_table, int max_pages,
+                                 const int32_t* q_offsets, const int32_t* q_vis,
+                                 const int32_t* idx, int B, int Q, int topk, float scale,
+                                 int num_splits, float* out, float* lse, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (!q_offsets || !q_vis || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
+  dsa_status s = mla_checks(q, kv_pool, num_pages, page_table, max_pages, idx, out, lse, scale);
+  if (s != DSA_OK) return s;
+  WsLayout L;
+  if (!ws_layout(Q, 1, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  return do_sparse_mla(q, kv_pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
+                       topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, float* out,
+                           float* lse, void* stream) {
+  if (!o_parts || !lse_parts || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (Q <= 0 || S <= 0) return DSA_ERR_INVALID_ARG;
+  if (Q > 65535 * 8 || S > 1024) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(o_parts, lse_parts, Q, S, out, lse,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
+                           const uint8_t* const* q_idx_layers, const float* const* w_layers,
+                           const uint8_t* const* k_idx_layers, int64_t total_keys,
+                           const int64_t* seq_offsets, const int32_t* q_offsets,
+                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           const void* const* q_layers, const void* const* pool_layers,
+                           int num_pages, const int32_t* const* page_table_layers,
+                           int max_pages, float scale, int num_splits,
+                           float* const* out_layers, float* const* lse_layers,
+                           int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  if (n_layers <= 0 || index_share <= 0) return DSA_ERR_INVALID_ARG;
+  if (!q_idx_layers || !w_layers || !k_idx_layers || !q_layers || !pool_layers ||
+      !page_table_layers || !out_layers || !lse_layers || !idx_out || !ws)
+    return DSA_ERR_INVALID_ARG;
+  dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, topk);
+  if (s != DSA_OK) return s;
+  if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
+  for (int l = 0; l < n_layers; ++l) {
+    if (l % index_share == 0 &&
+        (s = indexer_checks(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys)) != DSA_OK)
+      return s;
+    if ((s = mla_checks(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
+                        idx_out, out_layers[l], lse_layers[l], scale)) != DSA_OK)
+      return s;
+  }
+  WsLayout L;
+  if (!ws_layout(Q, max_len, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l = 0; l < n_layers; ++l) {
+    const int g = l / index_share;
+    int32_t* idx_g = idx_out + static_cast<size_t>(g) * Q * topk;
+    if (l % index_share == 0) {
+      s = do_indexer_topk(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys, seq_offsets,
+                          q_offsets, q_vis, B, Q, max_len, topk, mtp_index_share, idx_g, nullptr,
+                          ws, L, st);
+      if (s != DSA_OK) return s;
+    }
+    s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
+                      q_offsets, q_vis, idx_g, B, Q, topk, scale, L.S, out_layers[l],
+                      lse_layers[l], ws, L, st);
+    if (s != DSA_OK) return s;
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_check_error(void* ws, void* stream) {
+  if (!ws) return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t flag = 0;
+  if (cudaMemcpy(&flag, ws, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (flag) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  if (flag & DEVERR_TIMEOUT) return DSA_ERR_TIMEOUT;
+  if (flag & DEVERR_BOUNDS) return DSA_ERR_DEVICE_BOUNDS;
+  return DSA_OK;
+}
+
+}  // extern "C"

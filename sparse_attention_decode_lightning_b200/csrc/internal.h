@@ -1,0 +1,63 @@
+// Host-side declarations shared by the libdsa translation units: the
+// workspace carve-up and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+constexpr int TOPK_BINS = 4096;   // first-level histogram: top 12 bits of the score key
+constexpr int TOPK_META = 4;      // per-query counters: [0] above-threshold, [1] candidates
+
+// Byte offsets of the workspace regions (all 256-byte aligned).
+struct WsLayout {
+  size_t err = 0;      // uint32 error flag (+ padding)
+  size_t scores = 0;   // fp32 [Q, ld]
+  size_t hist = 0;     // uint32 [Q, TOPK_BINS]
+  size_t meta = 0;     // uint32 [Q, TOPK_META]
+  size_t cand = 0;     // uint64 [Q, ld]   candidate (key, position) pairs
+  size_t cand2 = 0;    // uint64 [Q, ld]   ping-pong for the refinement passes
+  size_t o_part = 0;   // fp32 [Q, S, 128, 512]
+  size_t l_part = 0;   // fp32 [Q, S, 128]
+  size_t total = 0;
+  int ld = 0;          // score row stride (elements)
+  int S = 0;           // split-K parts the partial buffers hold
+};
+
+bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* out);
+int device_sm_count();
+int choose_splits(int Q, int topk, int requested);
+
+// kernel launchers (return cudaSuccess or the launch error)
+cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                           int64_t total_keys, const int64_t* seq_offsets,
+                           const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                           int first_only, float* scores, int ld, uint32_t* err,
+                           cudaStream_t st);
+
+cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
+                        const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                        int first_only, int32_t* out_idx, float* out_scores, uint32_t* hist,
+                        uint32_t* meta, uint64_t* cand, uint64_t* cand2, uint32_t* err,
+                        cudaStream_t st);
+
+cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,
+                              int32_t* out_idx, float* out_scores, cudaStream_t st);
+
+cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
+                              const int32_t* page_table, int max_pages,
+                              const int32_t* q_offsets, const int32_t* q_vis,
+                              const int32_t* idx, int B, int Q, int topk, float scale, int S,
+                              float* out, float* lse, float* o_part, float* l_part,
+                              uint32_t* err, cudaStream_t st);
+
+cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, float* out,
+                           float* lse, cudaStream_t st);
+
+}  // namespace dsa

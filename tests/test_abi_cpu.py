@@ -1,0 +1,105 @@
+"""The C-ABI library loads without a GPU, exports every declared symbol, and
+rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_attention_decode_lightning_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from sparse_attention_decode_lightning_b200.build import build
+    build()
+
+
+def declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared()
+    assert len(names) >= 9
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if l.strip())
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    # the binding wraps exactly the declared entry points
+    assert set(dsa.SIGNATURES) == set(names)
+
+
+def test_library_loads_and_reports_version_and_status_names():
+    L = dsa.lib()
+    assert L.dsa_version() == 100
+    for code, name in dsa.STATUS.items():
+        assert dsa.dsa_status_string(code) == name
+    assert dsa.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
+
+
+def test_workspace_bytes_arithmetic():
+    f = dsa.dsa_workspace_bytes
+    assert f(0, 10, 2048, 0) == 0
+    assert f(1, 0, 2048, 0) == 0
+    assert f(1, 10, 4096, 0) == 0
+    assert f(1, 10, 2048, 33) == 0
+    small = f(1, 8192, 2048, 1)
+    # scores fp32 + two candidate lists of 8 bytes per key, histogram, one partial output
+    assert small >= 8192 * 4 + 2 * 8192 * 8 + 4096 * 4 + 128 * 512 * 4
+    assert f(32, 131072, 2048, 1) > 32 * 131072 * 20
+    assert f(4, 1 << 20, 2048, 16) > f(4, 1 << 20, 2048, 1)
+    assert f(4, 1 << 20, 2048, 16) - f(4, 1 << 20, 2048, 1) >= 4 * 15 * 128 * 512 * 4
+
+
+def test_host_checks_reject_bad_arguments_without_a_device():
+    L = dsa.lib()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)          # never dereferenced: checks fail first
+    null = P(0)
+    # null pointers
+    assert L.dsa_indexer_topk(null, fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048, 0, fake,
+                              null, fake, 1 << 30, null) == 1
+    # top-k above the supported maximum
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 100, 4096, 0, fake,
+                              null, fake, 1 << 30, null) == 2
+    # more queries than sequences allow
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 9, 100, 2048, 0, fake,
+                              null, fake, 1 << 30, null) == 2
+    # misaligned pointer
+    assert L.dsa_indexer_topk(P((1 << 20) + 4), fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048,
+                              0, fake, null, fake, 1 << 30, null) == 1
+    # workspace too small
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048, 0, fake,
+                              null, fake, 16, null) == 6
+    # sparse MLA: bad scale, bad split count, null page table
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 2048,
+                                   ctypes.c_float(0.0), 0, fake, fake, fake, 1 << 30, null) == 1
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 2048,
+                                   ctypes.c_float(0.07), 33, fake, fake, fake, 1 << 30, null) == 2
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, null, 4, fake, fake, fake, 1, 1, 2048,
+                                   ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30, null) == 1
+    # decode step: no layers, zero share group
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    arr = (ctypes.c_void_p * 1)(1 << 20)
+    assert L.dsa_decode_step(0, 1, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 100, 2048, arr,
+                             arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake, fake,
+                             1 << 30, null) == 1
+    assert L.dsa_decode_step(1, 0, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 100, 2048, arr,
+                             arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake, fake,
+                             1 << 30, null) == 1
+    # check_error without a workspace
+    assert L.dsa_check_error(null, null) == 1
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        dsa._ptr(torch.zeros(4))

@@ -1,0 +1,274 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+the same seeded inputs, at sizes the oracle finishes in seconds that still
+span several tiles and ragged tails."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import sparse_attention_decode_lightning_b200 as dsa
+from synth import get_workload, make_inputs
+from tests._helpers import np_bits, oracle_inputs
+from tests._parity import check_attention, check_topk_row, oracle_attention_for_idx
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _e4m3(x: torch.Tensor) -> torch.Tensor:
+    return x.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def run_decode_step(inp, num_splits=None, ws=None):
+    n, G, Q = inp.n_layers, inp.index_share, inp.Q
+    qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
+    wl = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
+    kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
+    outs = [torch.empty(Q, 128, 512, dtype=torch.float32, device=DEV) for _ in range(n)]
+    lses = [torch.empty(Q, 128, dtype=torch.float32, device=DEV) for _ in range(n)]
+    ng = (n + G - 1) // G
+    idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=DEV)
+    S = inp.num_splits if num_splits is None else num_splits
+    if ws is None:
+        ws = dsa.workspace(Q, inp.max_len, inp.topk, S)
+    dsa.dsa_decode_step(qi, wl, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B, inp.max_len,
+                        inp.topk, [L["q"] for L in inp.layers], [L["pool"] for L in inp.layers],
+                        [inp.page_table] * n, inp.scale, outs, lses, idx, ws, index_share=G,
+                        mtp_index_share=inp.mtp_index_share, num_splits=S)
+    dsa.dsa_check_error(ws)
+    return outs, lses, idx
+
+
+# ------------------------------------------------------------------ indexer
+@pytest.mark.parametrize("T,first_only", [(1, False), (8, False), (8, True)])
+def test_indexer_scores_match_oracle(T, first_only):
+    torch.manual_seed(0)
+    lens = [1000, 300, 129, 4096 + 77]
+    B = len(lens)
+    Q = B * T
+    seq_off = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int64, device=DEV)
+    q_off = torch.arange(B + 1, dtype=torch.int32, device=DEV) * T
+    vis = torch.tensor([lens[b] - (T - 1 - t) for b in range(B) for t in range(T)],
+                       dtype=torch.int32, device=DEV)
+    k = _e4m3(torch.randn(int(sum(lens)), 128, device=DEV))
+    qi = _e4m3(torch.randn(Q, 64, 128, device=DEV))
+    w = torch.randn(Q, 64, device=DEV) / 8
+    ld = max(lens) + 60
+    ld += (-ld) % 4
+    scores = torch.full((Q, ld), float("nan"), device=DEV)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8, device=DEV)
+    dsa.dsa_indexer_scores(qi, w, k, seq_off, q_off, vis, B, max(lens), scores, ws,
+                           first_only=first_only)
+    dsa.dsa_check_error(ws)
+    sc = scores.cpu().numpy()
+    kb, qb, wb = np_bits(k), np_bits(qi), w.cpu().numpy()
+    so = seq_off.cpu().numpy()
+    vv = vis.cpu().numpy()
+    for q in range(Q):
+        b, t = divmod(q, T)
+        if first_only and t > 0:
+            assert np.isnan(sc[q]).all()
+            continue
+        keys = kb[so[b]:so[b] + vv[q]]
+        ref = O.indexer_scores(qb[q], wb[q], keys)
+        # fp32 summation bound for the 64-head reduction (products are exact)
+        d = O.e4m3_decode(keys) @ O.e4m3_decode(qb[q]).T
+        mag = np.abs(np.maximum(d, 0) * wb[q].astype(np.float64)).sum(1)
+        tol = 64 * 2.0 ** -24 * mag + 1e-30
+        got = sc[q, :vv[q]].astype(np.float64)
+        bad = np.abs(got - ref) > tol
+        assert not bad.any(), (q, np.flatnonzero(bad)[:5], got[bad][:5], ref[bad][:5])
+        assert np.isnan(sc[q, vv[q]:]).all()
+
+
+# ------------------------------------------------------------------ selector
+def _topk_case(name, rng):
+    if name == "normal":
+        return rng.standard_normal(5000).astype(np.float32)
+    if name == "int_ties":
+        return rng.integers(-3, 4, 6000).astype(np.float32)
+    if name == "all_equal":
+        return np.full(3000, 1.5, dtype=np.float32)
+    if name == "signed_zero":
+        x = np.where(rng.random(4000) < 0.5, 0.0, -0.0).astype(np.float32)
+        x[rng.choice(4000, 100, replace=False)] = -1.0
+        return x
+    if name == "narrow_band":
+        return (10.0 + rng.random(40000) * 1e-3).astype(np.float32)
+    if name == "long":
+        return (rng.standard_normal(200000) * 7).astype(np.float32)
+    raise KeyError(name)
+
+
+@pytest.mark.parametrize("case", ["normal", "int_ties", "all_equal", "signed_zero", "narrow_band", "long"])
+def test_topk_select_exact_on_fixed_scores(case):
+    rng = np.random.default_rng(7)
+    x = _topk_case(case, rng)
+    L = x.shape[0]
+    rows = [x, x[: 2048], x[: 2049], x[: 1], x[: 2047]]
+    Q = len(rows)
+    ld = L + (-L) % 4
+    s = np.zeros((Q, ld), dtype=np.float32)
+    vis = np.zeros(Q, dtype=np.int32)
+    for i, r in enumerate(rows):
+        s[i, : r.shape[0]] = r
+        vis[i] = r.shape[0]
+    scores = torch.from_numpy(s).to(DEV)
+    q_off = torch.arange(Q + 1, dtype=torch.int32, device=DEV)
+    out = torch.empty(Q, 2048, dtype=torch.int32, device=DEV)
+    osc = torch.empty(Q, 2048, dtype=torch.float32, device=DEV)
+    ws = dsa.workspace(Q, ld, 2048, 1)
+    dsa.dsa_topk_select(scores, q_off, torch.from_numpy(vis).to(DEV), Q, L, 2048, out, ws,
+                        out_scores=osc)
+    dsa.dsa_check_error(ws)
+    out = out.cpu().numpy()
+    osc = osc.cpu().numpy()
+    for i, r in enumerate(rows):
+        ref = O.topk_select(r.astype(np.float64), 2048)
+        n = min(2048, r.shape[0])
+        assert set(out[i][out[i] >= 0].tolist()) == set(ref[:n].tolist())   # exact
+        assert (out[i][n:] == -1).all()
+        sel = out[i][:n]
+        assert np.array_equal(osc[i][:n], r[sel])
+        assert np.isneginf(osc[i][n:]).all()
+
+
+# ------------------------------------------------------------------ sparse MLA
+@pytest.mark.parametrize("S", [1, 3, 16])
+def test_sparse_mla_matches_oracle(S):
+    w = get_workload("decode_b32_ctx128k", B=3, L=1500, topk=2048)
+    inp = make_inputs(w, seed=11, device=DEV)
+    Q = inp.Q
+    g = torch.Generator(device="cpu").manual_seed(5)
+    idx = torch.full((Q, 2048), -1, dtype=torch.int32)
+    for q in range(Q):
+        n = [1500, 700, 1][q]
+        idx[q, :n] = torch.randperm(1500, generator=g)[:n].to(torch.int32)
+    idx = idx.to(DEV)
+    out = torch.empty(Q, 128, 512, device=DEV)
+    lse = torch.empty(Q, 128, device=DEV)
+    ws = dsa.workspace(Q, 1, 2048, S)
+    dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], inp.page_table,
+                              inp.q_offsets, inp.q_vis, idx, inp.B, inp.scale, out, lse, ws,
+                              num_splits=S)
+    dsa.dsa_check_error(ws)
+    pool, pt, qb = np_bits(inp.layers[0]["pool"]), np_bits(inp.page_table), np_bits(inp.layers[0]["q"])
+    ix = idx.cpu().numpy()
+    for q in range(Q):
+        o_ref, l_ref = oracle_attention_for_idx(pool, pt[q], qb[q], ix[q], inp.scale)
+        check_attention(out[q].cpu().numpy(), lse[q].cpu().numpy(), o_ref, l_ref)
+
+
+def test_sparse_mla_all_padding_gives_zero_and_neg_inf():
+    inp = make_inputs(get_workload("decode_b1_ctx8k", L=256), seed=2, device=DEV)
+    idx = torch.full((1, 2048), -1, dtype=torch.int32, device=DEV)
+    out = torch.full((1, 128, 512), 7.0, device=DEV)
+    lse = torch.zeros(1, 128, device=DEV)
+    for S in (1, 4):
+        ws = dsa.workspace(1, 1, 2048, S)
+        dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], inp.page_table,
+                                  inp.q_offsets, inp.q_vis, idx, 1, inp.scale, out, lse, ws,
+                                  num_splits=S)
+        dsa.dsa_check_error(ws)
+        assert (out == 0).all() and torch.isneginf(lse).all()
+
+
+def test_lse_combine_matches_oracle():
+    rng = np.random.default_rng(3)
+    Q, S = 3, 5
+    o = rng.standard_normal((Q, S, 128, 512)).astype(np.float32)
+    l = (rng.standard_normal((Q, S, 128)) * 4).astype(np.float32)
+    l[0, 2] = -np.inf
+    l[1, :, :7] = -np.inf
+    out = torch.empty(Q, 128, 512, device=DEV)
+    lse = torch.empty(Q, 128, device=DEV)
+    dsa.dsa_lse_combine(torch.from_numpy(o).to(DEV), torch.from_numpy(l).to(DEV), out, lse)
+    torch.cuda.synchronize()
+    for q in range(Q):
+        o_ref, l_ref = O.lse_combine(o[q].astype(np.float64), l[q].astype(np.float64))
+        assert np.allclose(out[q].cpu().numpy(), o_ref, rtol=1e-5, atol=1e-5)
+        fin = np.isfinite(l_ref)
+        assert np.allclose(lse[q].cpu().numpy()[fin], l_ref[fin], atol=1e-5)
+        assert np.isneginf(lse[q].cpu().numpy()[~fin]).all()
+
+
+# ------------------------------------------------------------------ whole step
+SMALL = {
+    "decode_b1_ctx8k": dict(),
+    "decode_b32_ctx128k": dict(B=4, L=9000),
+    "indexshare4_b64_ctx16k_128k": dict(B=5, L_range=(1500, 7000)),
+    "mtp_verify_b16_t8_ctx128k": dict(B=2, L=5000),
+    "mtp_verify_reuse_b16_t8_ctx128k": dict(B=2, L=5000),
+    "decode_b4_ctx1m_split16": dict(B=2, L=40000),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_step_matches_oracle(name):
+    w = get_workload(name, **SMALL[name])
+    inp = make_inputs(w, seed=0, device=DEV)
+    outs, lses, idx = run_decode_step(inp)
+    host = oracle_inputs(inp)
+    ix = idx.cpu().numpy()
+    T, G = inp.T, inp.index_share
+    swaps = 0
+    for g in range(ix.shape[0]):
+        ind = host["indexer"][g]
+        for q in range(inp.Q):
+            b = q // T
+            src = b * T if inp.mtp_index_share else q
+            k0, vis = int(host["seq_offsets"][b]), int(host["q_vis"][src])
+            sc = O.indexer_scores(ind["q_idx"][src], ind["w"][src], ind["k_idx"][k0:k0 + vis])
+            swaps += check_topk_row(ix[g, q], sc, inp.topk)
+            if inp.mtp_index_share:
+                assert np.array_equal(ix[g, q], ix[g, src])
+    for l in range(inp.n_layers):
+        lay = host["layers"][l]
+        for q in range(inp.Q):
+            b = q // T
+            o_ref, l_ref = oracle_attention_for_idx(lay["pool"], host["page_table"][b], lay["q"][q],
+                                                    ix[l // G, q], inp.scale)
+            check_attention(outs[l][q].cpu().numpy(), lses[l][q].cpu().numpy(), o_ref, l_ref)
+
+
+def test_indexshare_layers_use_the_leader_indices():
+    inp = make_inputs(get_workload("indexshare4_b64_ctx16k_128k", B=3, L_range=(3000, 5000)),
+                      seed=4, device=DEV)
+    outs, lses, idx = run_decode_step(inp)
+    assert idx.shape[0] == 1
+    # the shared layers' outputs equal direct sparse-MLA calls on the leader's indices
+    for l in range(1, 4):
+        out = torch.empty_like(outs[l])
+        lse = torch.empty_like(lses[l])
+        ws = dsa.workspace(inp.Q, 1, inp.topk, 0)
+        dsa.dsa_sparse_mla_decode(inp.layers[l]["q"], inp.layers[l]["pool"], inp.page_table,
+                                  inp.q_offsets, inp.q_vis, idx[0], inp.B, inp.scale, out, lse, ws)
+        dsa.dsa_check_error(ws)
+        assert torch.equal(out, outs[l]) and torch.equal(lse, lses[l])
+
+
+def test_device_bounds_are_flagged_not_faulted():
+    inp = make_inputs(get_workload("decode_b32_ctx128k", B=2, L=3000), seed=9, device=DEV)
+    bad_pt = inp.page_table.clone()
+    bad_pt[0, 3] = inp.num_pages + 5          # page id out of range
+    idx = torch.arange(2048, dtype=torch.int32, device=DEV).repeat(inp.Q, 1)
+    out = torch.empty(inp.Q, 128, 512, device=DEV)
+    lse = torch.empty(inp.Q, 128, device=DEV)
+    ws = dsa.workspace(inp.Q, 1, 2048, 2)
+    dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], bad_pt, inp.q_offsets,
+                              inp.q_vis, idx, inp.B, inp.scale, out, lse, ws, num_splits=2)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.dsa_check_error(ws)
+    assert e.value.status == 4
+    assert torch.isfinite(out).all()
+    dsa.dsa_check_error(ws)                   # the flag was cleared
+    # an index beyond the visible length is flagged too
+    idx2 = idx.clone()
+    idx2[1, 5] = 2999 + 10
+    dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], inp.page_table,
+                              inp.q_offsets, inp.q_vis, idx2, inp.B, inp.scale, out, lse, ws,
+                              num_splits=2)
+    with pytest.raises(dsa.DSAError):
+        dsa.dsa_check_error(ws)
