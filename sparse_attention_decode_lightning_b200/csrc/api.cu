@@ -8,7 +8,7 @@
 
 namespace dsa {
 
-cudaError_t launch_sparse_mla_simt(const __nv_bfloat16* q, const __nv_bfloat16* pool,
+cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                                    int num_pages, const int32_t* page_table, int max_pages,
                                    const int32_t* q_offsets, const int32_t* q_vis,
                                    const int32_t* idx, int B, int Q, int topk, float scale,
@@ -28,12 +28,22 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int choose_splits(int Q, int topk, int requested) {
   int S = requested;
   if (S <= 0) {
-    // enough (query, split) work units to cover the SMs twice, each with at
-    // least 128 selected rows
-    S = (2 * B200_SMS + Q - 1) / (Q > 0 ? Q : 1);
-    const int cap = topk / 128 > 0 ? topk / 128 : 1;
-    if (S > cap) S = cap;
-    if (S > 16) S = 16;
+    // (query, split) units run on 2-SM clusters: pick the smallest S whose
+    // units fill the 74 SM pairs to at least 85% over whole waves, keeping
+    // >= 64 selected rows per split; otherwise the best-filling S.
+    const int pairs = B200_SMS / 2;
+    const int cap = topk / 64 > 0 ? (topk / 64 < 16 ? topk / 64 : 16) : 1;
+    int best = 1;
+    double best_eff = -1.0;
+    S = 0;
+    for (int s = 1; s <= cap; ++s) {
+      const long units = static_cast<long>(Q) * s;
+      const long waves = (units + pairs - 1) / pairs;
+      const double eff = static_cast<double>(units) / (static_cast<double>(pairs) * waves);
+      if (eff >= 0.85) { S = s; break; }
+      if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+    }
+    if (S == 0) S = best;
   }
   if (S < 1) S = 1;
   if (S > DSA_MAX_SPLITS) S = DSA_MAX_SPLITS;
@@ -161,8 +171,8 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               const int32_t* idx, int B, int Q, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st) {
-  return launch_sparse_mla_simt(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx,
-                                B, Q, topk, scale, S, out, lse, o_part, l_part, err, st);
+  return launch_sparse_mla_tc(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B,
+                              Q, topk, scale, S, out, lse, o_part, l_part, err, st);
 }
 
 }  // namespace dsa

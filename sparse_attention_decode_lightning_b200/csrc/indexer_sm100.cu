@@ -22,8 +22,6 @@
 #include "common.cuh"
 #include "internal.h"
 
-#include <cudaTypedefs.h>
-#include <mutex>
 
 namespace dsa {
 namespace {
@@ -320,32 +318,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D u8 tensor [rows, 128] with 128-byte rows, tile box [box_rows, 128], 128-byte swizzle
-bool encode_u8_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {128, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
@@ -355,8 +327,12 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
                            cudaStream_t st) {
   if (B <= 0 || Q <= 0 || total_keys <= 0) return cudaSuccess;
   CUtensorMap tk, tq;
-  if (!encode_u8_rows(&tk, k_idx, static_cast<uint64_t>(total_keys), KT)) return cudaErrorInvalidValue;
-  if (!encode_u8_rows(&tq, q_idx, static_cast<uint64_t>(Q) * DSA_IDX_HEADS, DSA_IDX_HEADS))
+  if (!encode_tiled_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, DSA_IDX_DIM,
+                       static_cast<uint64_t>(total_keys), DSA_IDX_DIM, DSA_IDX_DIM, KT))
+    return cudaErrorInvalidValue;
+  if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_idx, DSA_IDX_DIM,
+                       static_cast<uint64_t>(Q) * DSA_IDX_HEADS, DSA_IDX_DIM, DSA_IDX_DIM,
+                       DSA_IDX_HEADS))
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;

@@ -30,6 +30,11 @@ struct WsLayout {
   int S = 0;           // split-K parts the partial buffers hold
 };
 
+// 2-D tensor map, 128-byte swizzle, no OOB fill value (zeros)
+bool encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                     uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                     uint32_t box_inner, uint32_t box_rows);
+
 bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* out);
 int device_sm_count();
 int choose_splits(int Q, int topk, int requested);

@@ -12,6 +12,7 @@ import sparse_attention_decode_lightning_b200 as dsa
 from synth import get_workload, make_inputs
 from tests._helpers import np_bits, oracle_inputs
 from tests._parity import check_attention, check_topk_row, oracle_attention_for_idx
+from tests._gpu import run_decode_step
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -19,26 +20,6 @@ DEV = "cuda"
 
 def _e4m3(x: torch.Tensor) -> torch.Tensor:
     return x.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
-
-
-def run_decode_step(inp, num_splits=None, ws=None):
-    n, G, Q = inp.n_layers, inp.index_share, inp.Q
-    qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
-    wl = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
-    kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
-    outs = [torch.empty(Q, 128, 512, dtype=torch.float32, device=DEV) for _ in range(n)]
-    lses = [torch.empty(Q, 128, dtype=torch.float32, device=DEV) for _ in range(n)]
-    ng = (n + G - 1) // G
-    idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=DEV)
-    S = inp.num_splits if num_splits is None else num_splits
-    if ws is None:
-        ws = dsa.workspace(Q, inp.max_len, inp.topk, S)
-    dsa.dsa_decode_step(qi, wl, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B, inp.max_len,
-                        inp.topk, [L["q"] for L in inp.layers], [L["pool"] for L in inp.layers],
-                        [inp.page_table] * n, inp.scale, outs, lses, idx, ws, index_share=G,
-                        mtp_index_share=inp.mtp_index_share, num_splits=S)
-    dsa.dsa_check_error(ws)
-    return outs, lses, idx
 
 
 # ------------------------------------------------------------------ indexer
