@@ -42,6 +42,8 @@ def parse():
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's sequence count (small profiling cases)")
     return ap.parse_args()
 
 
@@ -193,7 +195,7 @@ def run_ours(args, rank, world, local_rank):
     dist = None
     if world > 1:
         import torch.distributed as dist
-    wl = get_workload(args.workload)
+    wl = get_workload(args.workload, **({"B": args.batch} if args.batch else {}))
     inp = make_inputs(wl, seed=args.seed + rank, device=dev)
     Q, G, n = inp.Q, inp.index_share, inp.n_layers
     S = inp.num_splits

@@ -8,7 +8,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/dsa.h"
+#include "dsa.h"
 
 namespace dsa {
 

@@ -9,10 +9,15 @@
 //   warp 0      TMA producer: 128-key x 128-byte e4m3 tiles (16 KB, 128-byte
 //               swizzle) into an 8-stage shared-memory ring; the queries of the
 //               current sequence (8 KB each) into a query buffer.
-//   warp 1      tcgen05 issuer: for every key tile and every query of its
+//   warps 1,2   two tcgen05 issuers, one per pipeline; pipeline p takes the
+//               CTA's key tiles of parity p: for every query of the tile's
 //               sequence, D[128 keys, 64 heads] = K_tile . q^T as 4 MMAs of
-//               kind::f8f6f4 (M=128, N=64, K=32) into one of 4 TMEM slots.
-//   warps 2..9  two epilogue warpgroups (alternating slots): each thread reads
+//               kind::f8f6f4 (M=128, N=64, K=32) into one of its 4 TMEM slots
+//               (64 columns each, all 512 columns in use).  A single issuer
+//               thread spends ~1500 cycles per tile on mbarrier waits, MMA
+//               issue and commits, which alone caps a CTA near 25 GB/s; two
+//               independent issuers double that.
+//   warps 3..10 two epilogue warpgroups, one per pipeline: each thread reads
 //               its key row (64 fp32 head dots) with tcgen05.ld and reduces
 //               sum_h w_h * max(d_h, 0) in registers; 128 consecutive fp32
 //               scores per warpgroup are written coalesced.
@@ -28,10 +33,11 @@ namespace {
 
 constexpr int KT = 128;                                // keys per tile (MMA M)
 constexpr int STAGES = 8;                              // key-tile ring depth
-constexpr int NACC = 4;                                // TMEM accumulator slots
+constexpr int NACC = 8;                                // TMEM accumulator slots (all 512 columns)
 constexpr int ACC_COLS = DSA_IDX_HEADS;                // 64 fp32 columns per slot
-constexpr int EPI_WG = 2;                              // epilogue warpgroups
-constexpr int THREADS = 64 + EPI_WG * 128;
+constexpr int PIPES = 2;                               // MMA issuer + epilogue warpgroup pairs
+constexpr int SLOTS_PER_PIPE = NACC / PIPES;
+constexpr int THREADS = 32 + PIPES * 32 + PIPES * 128;
 constexpr int KEY_TILE = KT * DSA_IDX_DIM;             // 16384 B
 constexpr int Q_TILE = DSA_IDX_HEADS * DSA_IDX_DIM;    // 8192 B
 constexpr int OFF_KEYS = 0;
@@ -39,7 +45,7 @@ constexpr int OFF_Q = OFF_KEYS + STAGES * KEY_TILE;
 constexpr int OFF_PREFIX = OFF_Q + DSA_MAX_Q_PER_SEQ * Q_TILE;
 constexpr int OFF_SCAN = OFF_PREFIX + ((DSA_MAX_BATCH + 1) * 4 + 15) / 16 * 16;
 constexpr int OFF_BAR = OFF_SCAN + 64 * 4;
-constexpr int NBAR = 2 * STAGES + 2 * NACC + 3;
+constexpr int NBAR = 2 * STAGES + 2 * NACC + 2 + PIPES;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;           // slack for 1024-byte alignment
@@ -129,7 +135,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* q_full = acc_empty + NACC;
   uint64_t* q_empty = q_full + 1;
-  uint64_t* mma_done = q_full + 2;
+  uint64_t* mma_done = q_full + 2;        // one per pipeline
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,8 +159,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < NACC; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    mbar_init(mma_done, 1);
+    mbar_init(q_empty, PIPES);        // every MMA issuer releases the query buffer
+    for (int p = 0; p < PIPES; ++p) mbar_init(&mma_done[p], 1);
     mbar_fence_init();
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_q);
@@ -219,12 +225,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1, a.err);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp <= 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // pipeline p = warp - 1 owns the CTA's tiles of parity p and TMEM slots
+    // 4p .. 4p+3; both walk every tile to keep the query-buffer hand-off in step
+    const int pipe = warp - 1;
     if (lane == 0 && t_begin < t_end) {
       constexpr uint32_t idesc = umma_idesc(0 /*E4M3*/, KT, ACC_COLS);
       int b = b_first, cur_b = -1, nq = 0;
-      uint32_t stage = 0, phase = 0, qphase = 0, acc = 0;
+      uint32_t qphase = 0, n = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
         while (prefix[b + 1] <= i) ++b;
@@ -235,12 +244,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           nq = seq_queries(a, b);
           cur_b = b;
         }
-        if (!mbar_wait(&full[stage], phase, a.err)) { ok = false; break; }
+        const int local = i - t_begin;
+        if ((local & 1) != pipe) continue;
+        const int stage = local % STAGES;
+        if (!mbar_wait(&full[stage], (local / STAGES) & 1, a.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(keys + stage * KEY_TILE);
-        for (int j = 0; j < nq; ++j, ++acc) {
-          const uint32_t slot = acc % NACC;
-          if (!mbar_wait(&acc_empty[slot], ((acc / NACC) & 1) ^ 1, a.err)) { ok = false; break; }
+        for (int j = 0; j < nq; ++j, ++n) {
+          const uint32_t slot = pipe * SLOTS_PER_PIPE + n % SLOTS_PER_PIPE;
+          if (!mbar_wait(&acc_empty[slot], ((n / SLOTS_PER_PIPE) & 1) ^ 1, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t b_base = smem_u32(qbuf + j * Q_TILE);
 #pragma unroll
@@ -252,31 +264,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (!ok) break;
         mma_commit(&empty[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       // every MMA this thread issued must finish before TMEM is released
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, a.err);
+      mma_commit(&mma_done[pipe]);
+      mbar_wait(&mma_done[pipe], 0, a.err);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     if (t_begin < t_end) {
-      const int g = (warp - 2) >> 2;           // warpgroup 0 / 1
+      const int g = (warp - 3) >> 2;           // warpgroup = pipeline 0 / 1
       const int quarter = warp & 3;            // TMEM lanes this warp may read
       const int row = quarter * 32 + lane;     // key row of the tile
       int b = b_first;
-      uint32_t acc = 0;
+      uint32_t n = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
         while (prefix[b + 1] <= i) ++b;
+        if (((i - t_begin) & 1) != g) continue;
         const int t = i - prefix[b];
         const int nq = seq_queries(a, b);
         const int q0 = a.q_offsets[b];
         const int64_t len = a.seq_offsets[b + 1] - a.seq_offsets[b];
-        for (int j = 0; j < nq; ++j, ++acc) {
-          if ((acc & 1u) != static_cast<uint32_t>(g)) continue;
-          const uint32_t slot = acc % NACC;
-          if (!mbar_wait(&acc_full[slot], (acc / NACC) & 1, a.err)) { ok = false; break; }
+        for (int j = 0; j < nq; ++j, ++n) {
+          const uint32_t slot = g * SLOTS_PER_PIPE + n % SLOTS_PER_PIPE;
+          if (!mbar_wait(&acc_full[slot], (n / SLOTS_PER_PIPE) & 1, a.err)) { ok = false; break; }
           tc_fence_after();
           float v[ACC_COLS];
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * ACC_COLS;

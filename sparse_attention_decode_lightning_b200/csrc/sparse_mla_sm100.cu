@@ -50,7 +50,8 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_ST = OFF_Q + MAXCH * CHUNK_Q;
 constexpr int OFF_P = OFF_ST + NST * STAGE_BYTES;
 constexpr int OFF_X = OFF_P + 2 * P_BYTES;
-constexpr int OFF_BAR = OFF_X + 2 * X_BYTES;
+constexpr int OFF_CRD = OFF_X + 2 * X_BYTES;    // pool row of every entry of the split
+constexpr int OFF_BAR = OFF_CRD + DSA_MAX_TOPK * 4;
 constexpr int NBAR = 2 * NST + 5 * 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -85,22 +86,6 @@ __device__ __forceinline__ int seq_of_query(const int32_t* q_offsets, int B, int
   return lo;
 }
 
-// pool row of entry j of the query's index row, or -1 (padding / out of range)
-__device__ __forceinline__ int pool_row(const MlaTcArgs& a, int q, int b, int vis, int j, int r1,
-                                        bool report) {
-  if (j >= r1) return -1;
-  const int s = a.idx[static_cast<size_t>(q) * a.topk + j];
-  if (s == -1) return -1;
-  bool ok = s >= 0 && s < vis && (s >> 6) < a.max_pages;
-  int pg = ok ? a.page_table[static_cast<size_t>(b) * a.max_pages + (s >> 6)] : -1;
-  ok = ok && pg >= 0 && pg < a.num_pages;
-  if (!ok) {
-    if (report) raise_error(a.err, DEVERR_BOUNDS);
-    return -1;
-  }
-  return pg * DSA_PAGE_SIZE + (s & (DSA_PAGE_SIZE - 1));
-}
-
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   const bool ok = mbar_wait(bar, parity, err);
   return __all_sync(0xffffffffu, ok);
@@ -116,6 +101,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint8_t* st = smem + OFF_ST;
   uint8_t* pb = smem + OFF_P;
   uint8_t* xb = smem + OFF_X;
+  int* crd = reinterpret_cast<int*>(smem + OFF_CRD);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
@@ -147,9 +133,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int i = 0; i < NST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&x_full[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_empty[i], 4);     // one arrival per softmax warp
+      mbar_init(&x_full[i], 4);      // one remote arrival per peer softmax warp
+      mbar_init(&p_full[i], 4);
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_done, 1);
@@ -163,28 +149,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();                 // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  if (tid == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_kv);
+    mbar_arrive_expect_tx(q_full, nch * CHUNK_Q);
+    for (int c = 0; c < nch; ++c)
+      tma_load_2d(qs + c * CHUNK_Q, &tmap_q, (gch0 + c) * 64, q * DSA_HEADS, q_full);
+  }
+  // pool row of every entry of this split, resolved once by all threads with
+  // many independent loads in flight (-1 = padding or out of range)
+  {
+    constexpr int PER = (DSA_MAX_TOPK + THREADS - 1) / THREADS;
+    int sv[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int j = r0 + tid + k * THREADS;
+      sv[k] = j < r1 ? a.idx[static_cast<size_t>(q) * a.topk + j] : -1;
+    }
+    int pg[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int sx = sv[k];
+      const bool ok = sx >= 0 && sx < vis && (sx >> 6) < a.max_pages;
+      pg[k] = ok ? a.page_table[static_cast<size_t>(b) * a.max_pages + (sx >> 6)] : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int jj = tid + k * THREADS;
+      if (r0 + jj < r1) {
+        const int sx = sv[k];
+        const bool ok = pg[k] >= 0 && pg[k] < a.num_pages;
+        if (!ok && sx != -1 && rank == 0) raise_error(a.err, DEVERR_BOUNDS);
+        crd[jj] = ok ? pg[k] * DSA_PAGE_SIZE + (sx & (DSA_PAGE_SIZE - 1)) : -1;
+      }
+    }
+  }
+  __syncthreads();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol = l2_policy_evict_first();
-    if (lane == 0) {
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_kv);
-      mbar_arrive_expect_tx(q_full, nch * CHUNK_Q);
-      for (int c = 0; c < nch; ++c)
-        tma_load_2d(qs + c * CHUNK_Q, &tmap_q, (gch0 + c) * 64, q * DSA_HEADS, q_full);
-    }
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % NST;
       if (!warp_wait(&empty[s], ((t / NST) & 1) ^ 1, a.err)) break;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], nch * CHUNK_T);
       __syncwarp();
       if (lane < NR / 4) {
-        const int j = r0 + t * NR + 4 * lane;
-        const int c0 = pool_row(a, q, b, vis, j + 0, r1, rank == 0);
-        const int c1 = pool_row(a, q, b, vis, j + 1, r1, rank == 0);
-        const int c2 = pool_row(a, q, b, vis, j + 2, r1, rank == 0);
-        const int c3 = pool_row(a, q, b, vis, j + 3, r1, rank == 0);
+        const int j = t * NR + 4 * lane;        // entry within the split
+        const int n = r1 - r0;
+        const int c0 = j + 0 < n ? crd[j + 0] : -1;
+        const int c1 = j + 1 < n ? crd[j + 1] : -1;
+        const int c2 = j + 2 < n ? crd[j + 2] : -1;
+        const int c3 = j + 3 < n ? crd[j + 3] : -1;
         for (int c = 0; c < nch; ++c)
           tma_gather4(st + s * STAGE_BYTES + c * CHUNK_T + 4 * lane * 128, &tmap_kv,
                       (gch0 + c) * 64, c0, c1, c2, c3, &full[s], pol);
@@ -245,21 +261,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int t = 0; t < ntiles && ok; ++t) {
       const int sb = t & 1;
       const uint32_t ph = (t >> 1) & 1;
-      const uint32_t vmask =
-          __ballot_sync(0xffffffffu, pool_row(a, q, b, vis, r0 + t * NR + lane, r1, false) >= 0);
+      const int jrow = t * NR + lane;
+      const uint32_t vmask = __ballot_sync(0xffffffffu, jrow < r1 - r0 && crd[jrow] >= 0);
       if (!(ok = warp_wait(&s_full[sb], ph, a.err))) break;
       tc_fence_after();
       float v[NR];
       tmem_ld32(lane_base + S_COL + sb * NR, v);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&s_empty[sb]);
-      // my partial scores -> the peer's exchange slot, then signal it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      // my partial scores -> the peer's exchange slot; the warp barrier orders
+      // all lanes' stores before lane 0's cluster-scope release arrive
       const uint32_t dst = peer_x + sb * X_BYTES + h * NR * 4;
 #pragma unroll
       for (int i = 0; i < NR / 4; ++i)
         st_cluster_v4(dst + 16 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      mbar_arrive_remote(map_to_rank(smem_u32(&x_full[sb]), peer));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&x_full[sb]), peer));
       const bool got = mbar_wait_cluster(&x_full[sb], ph, a.err);
       if (!(ok = __all_sync(0xffffffffu, got))) break;
       const float4* src = reinterpret_cast<const float4*>(xb + sb * X_BYTES + h * NR * 4);
@@ -333,7 +352,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&p_full[sb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
     }
     // ---- epilogue: O / l for this CTA's 256 value columns; LSE from CTA 0
     const bool have = ok && ntiles > 0 && warp_wait(o_final, 0, a.err);

@@ -19,7 +19,7 @@
 namespace dsa {
 namespace {
 
-constexpr int CHUNK = 16384;    // scores per CTA in passes 1 and 2
+constexpr int CHUNK = 8192;     // scores per CTA in passes 1 and 2
 constexpr int PT = 512;         // threads for passes 1 and 2
 constexpr int RT = 1024;        // threads for pass 3
 
@@ -52,24 +52,6 @@ __device__ __forceinline__ int clamped_vis(const TopkArgs& a, int q) {
     v = v < 0 ? 0 : a.max_len;
   }
   return v;
-}
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
-// warp-aggregated atomic slot reservation: every lane calls, `pred` lanes get a slot
-__device__ __forceinline__ uint32_t warp_reserve(uint32_t* ctr, bool pred) {
-  const uint32_t m = __ballot_sync(0xffffffffu, pred);
-  if (m == 0) return 0;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(ctr, static_cast<uint32_t>(__popc(m)));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  return base + __popc(m & lanemask_lt());
 }
 
 __global__ void __launch_bounds__(PT) topk_hist_kernel(TopkArgs a) {
@@ -139,7 +121,7 @@ __device__ void find_threshold(const uint32_t* hist, uint32_t k, uint32_t* s_bin
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(PT) topk_filter_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(PT, 2) topk_filter_kernel(TopkArgs a) {
   __shared__ uint32_t s_tmp[32];
   __shared__ uint32_t s_bin, s_above;
   const int q = row_query(a, blockIdx.y);
@@ -165,25 +147,71 @@ __global__ void __launch_bounds__(PT) topk_filter_kernel(TopkArgs a) {
   uint32_t* meta = a.meta + static_cast<size_t>(q) * TOPK_META;
   if (blockIdx.x == 0 && threadIdx.x == 0) { meta[2] = tb; meta[3] = s_above; }
   uint64_t* cand = a.cand + static_cast<size_t>(q) * a.ld;
-  for (int base = beg; base < end; base += 4 * PT) {
-    const int i = base + 4 * threadIdx.x;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < end) v = *reinterpret_cast<const float4*>(row + i);
-    const float vv[4] = {v.x, v.y, v.z, v.w};
+  // each thread holds its CHUNK / PT scores in registers; slots are reserved
+  // with one block scan and one global atomic per counter per CTA
+  constexpr int PER4 = CHUNK / (4 * PT);
+  float4 v[PER4];
+  uint32_t na = 0, nc = 0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const bool valid = i + k < end;
-      const uint32_t key = float_key(vv[k]);
+  for (int k = 0; k < PER4; ++k) {
+    const int i = beg + 4 * (threadIdx.x + k * PT);
+    v[k] = i < end ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t bin = float_key(vv[e]) >> 20;
+      const bool valid = i + e < end;
+      na += (valid && bin > tb);
+      nc += (valid && bin == tb);
+    }
+  }
+  // block exclusive scan of (na << 16 | nc); totals stay below 2^16 per CTA
+  const uint32_t packed = (na << 16) | nc;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = packed;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  __shared__ uint32_t s_warp[PT / 32];
+  __shared__ uint32_t s_base_a, s_base_c;
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t x = lane < PT / 32 ? s_warp[lane] : 0;
+    uint32_t xi = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, xi, off);
+      if (lane >= off) xi += y;
+    }
+    if (lane < PT / 32) s_warp[lane] = xi - x;
+    if (lane == 31) {
+      s_base_a = (xi >> 16) ? atomicAdd(&meta[0], xi >> 16) : 0;
+      s_base_c = (xi & 0xFFFFu) ? atomicAdd(&meta[1], xi & 0xFFFFu) : 0;
+    }
+  }
+  __syncthreads();
+  const uint32_t pre = s_warp[warp] + incl - packed;
+  uint32_t pa = s_base_a + (pre >> 16), pc = s_base_c + (pre & 0xFFFFu);
+#pragma unroll
+  for (int k = 0; k < PER4; ++k) {
+    const int i = beg + 4 * (threadIdx.x + k * PT);
+    const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t key = float_key(vv[e]);
       const uint32_t bin = key >> 20;
-      const bool above = valid && bin > tb;
-      const bool inbin = valid && bin == tb;
-      const uint32_t p = warp_reserve(&meta[0], above);
-      if (above) {
-        oi[p] = i + k;
-        if (os) os[p] = vv[k];
+      if (i + e < end) {
+        if (bin > tb) {
+          oi[pa] = i + e;
+          if (os) os[pa] = vv[e];
+          ++pa;
+        } else if (bin == tb) {
+          cand[pc++] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i + e));
+        }
       }
-      const uint32_t c = warp_reserve(&meta[1], inbin);
-      if (inbin) cand[c] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i + k));
     }
   }
 }
