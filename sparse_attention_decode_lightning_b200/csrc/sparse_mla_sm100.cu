@@ -5,63 +5,75 @@
 //   z_j = scale * q[h,:] . C[j,:],  O[h] = sum_j softmax(z)_j C[j,:512],
 //   LSE[h] = ln sum_j exp(z_j).
 //
-// Work unit: (query, split) on a cluster of two CTAs.  The 128 x 512 fp32
-// output alone fills one SM's tensor memory, and the 128 x 576 bf16 query
-// (147 KB) would crowd out the gather pipeline, so the pair divides both:
-//   CTA 0 holds q[:, 0:256) and computes S0 = q[:,0:256) C[:,0:256)^T and
-//         O[:, 0:256);
-//   CTA 1 holds q[:, 256:576) and computes S1 = q[:,256:576) C[:,256:576)^T
-//         and O[:, 256:512).
-// Each CTA gathers only the latent columns it uses (0:256 or 256:576), so
-// every latent byte crosses HBM once.  Per 32-row tile the CTAs swap their
-// fp32 partial scores through distributed shared memory; both form
-// S = S0 + S1 (bitwise equal on both sides), run the same online softmax and
-// feed the same P to their half of O += P V.
+// Work unit: (query, split) on a cluster of two CTAs that divide the
+// contraction dims and the output:
+//   CTA 0: S0 = q[:, 0:256) C[:, 0:256)^T + q[:, 512:544) C[:, 512:544)^T, O[:, 0:256)
+//   CTA 1: S1 = q[:, 256:512) C[:, 256:512)^T + q[:, 544:576) C[:, 544:576)^T, O[:, 256:512)
+// so each CTA gathers the latent columns it uses (the 64 RoPE columns go to
+// both; each contracts half of them, which keeps the pair in balance).  Per tile of 64 selected rows the CTAs swap their fp32
+// partial scores through distributed shared memory; both form S0 + S1
+// (bitwise equal on both sides), run the same online softmax and apply the
+// same P to their half of O.
 //
-// Roles per CTA (192 threads):
-//   warp 0      producer: page-table lookups and TMA tile::gather4 row
-//               gathers (4 rows x 128 B per op, 128-byte swizzle) into a
-//               3-stage ring; the query slice once.
-//   warp 1      tcgen05 issuer: S (M=128 heads, N=32 rows, K=256|320) into a
-//               double-buffered TMEM slot; O += P V (M=128, N=256, V read
-//               MN-major straight from the gathered tile).
-//   warps 2..5  softmax: one head row per thread; exchange, online softmax
-//               in the exp2 domain with a lazy rescale of O (only when the
-//               running max grows by more than 2^8), P into shared memory as
-//               a bf16 hi + lo pair (about 16 significant bits: a single bf16
-//               P costs ~1% of the output RMS once the running max is stale),
-//               final O / l and LSE.
+// Tensor memory (512 columns): O half [0,256) | S/P slot 0 [256,320) |
+// S/P slot 1 [320,384) | the CTA's 256 latent query dims [384,512) (bf16
+// pairs).  The scores MMA reads those from tensor memory and the RoPE query
+// dims from shared memory; the softmax overwrites a slot's scores with P as bf16
+// hi + lo halves (p ~= hi + lo to ~16 significant bits: a single bf16 P
+// costs ~1% of the output RMS once the running max is stale), which the PV
+// MMA reads from tensor memory against V (MN-major, N = 256) in shared
+// memory.
+//
+// Latent rows are gathered through the page table with 16-byte cp.async by
+// four producer warps (4 rows x 128 bytes per warp instruction, written in
+// the 128-byte swizzle the MMA descriptors expect; a single warp cannot keep
+// enough copies in flight) into a 3-stage ring; completion is signalled by
+// cp.async.mbarrier.arrive so no producer ever waits for its own copies
+// (waiting for them coupled a tile's arrival to the PV of an earlier tile).  Each stage holds one tile
+// (64 rows x 256 or 320 dims) until its PV is done.  The partial scores are
+// exchanged by pull (local write, remote loads): remote stores from four
+// warps drained at a few KB per microsecond.
+//
+// Roles (416 threads): warps 0, 10..12 producers, warp 1 tcgen05 issuer,
+// warps 2..9 softmax + epilogue as two warpgroups that take rows 0..31 and
+// 32..63 of each tile (one head per thread, TMEM lane = head; the row maxima
+// meet through shared memory).  A single warp per scheduler left the
+// softmax arithmetic latency-bound on the critical path.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dsa {
 namespace {
 
-constexpr int NR = 32;                         // selected rows per tile
-constexpr int NST = 3;                         // gather ring depth
-constexpr int THREADS = 192;
-constexpr int MAXCH = 5;                       // 64-column chunks per CTA (CTA 1)
-constexpr int CHUNK_Q = DSA_HEADS * 128;       // 16 KB: 128 heads x 64 bf16
-constexpr int CHUNK_T = NR * 128;              // 4 KB: 32 rows x 64 bf16
-constexpr int STAGE_BYTES = MAXCH * CHUNK_T;
-constexpr int P_BYTES = DSA_HEADS * 128;       // 128 rows of 32 bf16 hi + 32 bf16 lo
-constexpr int X_BYTES = DSA_HEADS * NR * 4;    // one tile of fp32 partial scores
-constexpr int OFF_Q = 0;
-constexpr int OFF_ST = OFF_Q + MAXCH * CHUNK_Q;
-constexpr int OFF_P = OFF_ST + NST * STAGE_BYTES;
-constexpr int OFF_X = OFF_P + 2 * P_BYTES;
-constexpr int OFF_CRD = OFF_X + 2 * X_BYTES;    // pool row of every entry of the split
+constexpr int NR = 64;                         // selected rows per tile
+constexpr int NST = 3;                         // tile ring depth
+constexpr int PRODUCERS = 4;                   // gather warps (cp.async parallelism)
+constexpr int SMX_WARPS = 8;                   // softmax warps (two warpgroups)
+constexpr int THREADS = 32 * (2 + SMX_WARPS + PRODUCERS - 1);   // warp 0 + warps 10.. produce
+constexpr int MAXCH = 5;                       // 64-dim chunks per CTA (CTA 1)
+constexpr int CHUNK_T = NR * 128;              // 8 KB: 64 rows x 64 bf16
+constexpr int STAGE_BYTES = MAXCH * CHUNK_T;   // 40 KB
+constexpr int QROPE_BYTES = DSA_HEADS * 128;   // 16 KB: 128 heads x 64 bf16
+constexpr int X_BYTES = DSA_HEADS * NR * 4;    // 32 KB: one tile of fp32 partial scores
+constexpr int OFF_QR = 0;
+constexpr int OFF_ST = OFF_QR + QROPE_BYTES;
+constexpr int OFF_X = OFF_ST + NST * STAGE_BYTES;
+constexpr int OFF_MX = OFF_X + 2 * X_BYTES;    // [2 tiles][2 warpgroups][128 heads] partial maxima
+constexpr int OFF_CRD = OFF_MX + 2 * 2 * DSA_HEADS * 4;
 constexpr int OFF_BAR = OFF_CRD + DSA_MAX_TOPK * 4;
-constexpr int NBAR = 2 * NST + 5 * 2 + 3;
+constexpr int NBAR = 2 * NST + 4 * 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "sparse MLA shared memory exceeds the sm_100 limit");
-static_assert(OFF_ST % 1024 == 0 && OFF_P % 1024 == 0 && OFF_X % 1024 == 0, "swizzle atoms");
-constexpr uint32_t O_COL = 0;                  // TMEM columns [0,256): O half
-constexpr uint32_t S_COL = 256;                // [256,320): two 32-column score slots
+static_assert(OFF_ST % 1024 == 0 && OFF_X % 1024 == 0, "swizzle atoms");
+constexpr uint32_t O_COL = 0;
+constexpr uint32_t S_COL = 256;
+constexpr uint32_t Q_COL = 384;
 constexpr uint32_t TMEM_COLS = 512;
 
 struct MlaTcArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* pool;
   const int32_t* page_table;
   int max_pages;
   int num_pages;
@@ -91,56 +103,59 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __all_sync(0xffffffffu, ok);
 }
 
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                         const __grid_constant__ CUtensorMap tmap_kv, MlaTcArgs a) {
+    sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* qs = smem + OFF_Q;
+  uint8_t* qrope = smem + OFF_QR;
   uint8_t* st = smem + OFF_ST;
-  uint8_t* pb = smem + OFF_P;
   uint8_t* xb = smem + OFF_X;
   int* crd = reinterpret_cast<int*>(smem + OFF_CRD);
+  float* mx = reinterpret_cast<float*>(smem + OFF_MX);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
-  uint64_t* s_full = bars + 2 * NST;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* x_full = s_empty + 2;
-  uint64_t* p_full = x_full + 2;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_done = p_empty + 2;
-  uint64_t* o_final = o_done + 1;
-  uint64_t* q_full = o_final + 1;
+  uint64_t* s_full = bars + 2 * NST;     // [2] scores of a tile are in its slot
+  uint64_t* p_full = s_full + 2;         // [2] P of a tile is in its slot
+  uint64_t* slot_free = p_full + 2;      // [2] PV of the slot's tile is done
+  uint64_t* x_full = slot_free + 2;      // [2] the peer's partial scores arrived
+  uint64_t* o_done = x_full + 2;         // every PV
+  uint64_t* o_final = o_done + 1;        // last PV
+  uint64_t* q_ready = o_final + 1;       // query slice in TMEM / shared memory
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const int unit = blockIdx.x >> 1;
   const int q = unit / a.S, split = unit % a.S;
-  const int nch = rank ? 5 : 4;                 // 64-column chunks gathered by this CTA
-  const int gch0 = rank ? 4 : 0;                // first global chunk
   const int b = seq_of_query(a.q_offsets, a.B, q);
   int vis = a.q_vis[q];
   if (vis < 0) vis = 0;
   const int per = (a.topk + a.S - 1) / a.S;
   const int r0 = split * per;
   const int r1 = min(a.topk, r0 + per);
-  const int ntiles = r1 > r0 ? (r1 - r0 + NR - 1) / NR : 0;
+  const int nrows = r1 > r0 ? r1 - r0 : 0;
+  const int ntiles = (nrows + NR - 1) / NR;
 
   if (tid == 0) {
-    for (int i = 0; i < NST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 32 * PRODUCERS);   // one copy-completion arrival per producer lane
+      mbar_init(&empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);     // one arrival per softmax warp
-      mbar_init(&x_full[i], 4);      // one remote arrival per peer softmax warp
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_empty[i], 1);
+      mbar_init(&p_full[i], SMX_WARPS);  // one arrival per softmax warp
+      mbar_init(&slot_free[i], 1);
+      mbar_init(&x_full[i], SMX_WARPS);  // the peer's softmax warps: its partial is readable
     }
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
-    mbar_init(q_full, 1);
+    mbar_init(q_ready, 5);             // 4 query-loading warps + thread 0 with the RoPE bytes
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, TMEM_COLS);
@@ -151,10 +166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_holder;
   if (tid == 0) {
     tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_kv);
-    mbar_arrive_expect_tx(q_full, nch * CHUNK_Q);
-    for (int c = 0; c < nch; ++c)
-      tma_load_2d(qs + c * CHUNK_Q, &tmap_q, (gch0 + c) * 64, q * DSA_HEADS, q_full);
+    mbar_arrive_expect_tx(q_ready, QROPE_BYTES);
+    tma_load_2d(qrope, &tmap_q, 8 * 64, q * DSA_HEADS, q_ready);
   }
   // pool row of every entry of this split, resolved once by all threads with
   // many independent loads in flight (-1 = padding or out of range)
@@ -176,7 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int jj = tid + k * THREADS;
-      if (r0 + jj < r1) {
+      if (jj < nrows) {
         const int sx = sv[k];
         const bool ok = pg[k] >= 0 && pg[k] < a.num_pages;
         if (!ok && sx != -1 && rank == 0) raise_error(a.err, DEVERR_BOUNDS);
@@ -186,116 +199,186 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
   __syncthreads();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const uint64_t pol = l2_policy_evict_first();
-    for (int t = 0; t < ntiles; ++t) {
-      const int s = t % NST;
-      if (!warp_wait(&empty[s], ((t / NST) & 1) ^ 1, a.err)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], nch * CHUNK_T);
-      __syncwarp();
-      if (lane < NR / 4) {
-        const int j = t * NR + 4 * lane;        // entry within the split
-        const int n = r1 - r0;
-        const int c0 = j + 0 < n ? crd[j + 0] : -1;
-        const int c1 = j + 1 < n ? crd[j + 1] : -1;
-        const int c2 = j + 2 < n ? crd[j + 2] : -1;
-        const int c3 = j + 3 < n ? crd[j + 3] : -1;
-        for (int c = 0; c < nch; ++c)
-          tma_gather4(st + s * STAGE_BYTES + c * CHUNK_T + 4 * lane * 128, &tmap_kv,
-                      (gch0 + c) * 64, c0, c1, c2, c3, &full[s], pol);
+  if (warp == 0 || warp >= 2 + SMX_WARPS) {
+    // ------------------------------------------------------------ producers
+    // producer p copies rows [16p, 16p+16) of every tile; its warp instruction
+    // i copies row 16p + 4i + (lane >> 3), 16-byte piece (lane & 7); piece u
+    // of row r lands at r*128 + ((u ^ (r & 7)) * 16)
+    const int pw = warp == 0 ? 0 : warp - (1 + SMX_WARPS);
+    const int pu = lane & 7;
+    const uint8_t* pool = reinterpret_cast<const uint8_t*>(a.pool);
+    bool ok = true;
+    for (int k = 0; k < ntiles && ok; ++k) {
+      const int s = k % NST;
+      if (!(ok = warp_wait(&empty[s], ((k / NST) & 1) ^ 1, a.err))) break;
+      uint8_t* stage = st + s * STAGE_BYTES;
+#pragma unroll
+      for (int i = 0; i < NR / (4 * PRODUCERS); ++i) {
+        const int r = (NR / PRODUCERS) * pw + 4 * i + (lane >> 3);
+        const int j = k * NR + r;
+        const int row = j < nrows ? crd[j] : -1;
+        const uint8_t* src = row >= 0 ? pool + static_cast<size_t>(row) * (DSA_DIM * 2) + pu * 16 : pool;
+        const uint32_t nb = row >= 0 ? 16u : 0u;
+        const int sh = row >= 0 ? 1 : 0;      // address step only for real rows
+        uint8_t* dst = stage + r * 128 + ((pu ^ (r & 7)) * 16);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cp_async16(dst + c * CHUNK_T, src + sh * (4 * rank + c) * 128, nb);
+        cp_async16(dst + 4 * CHUNK_T, src + sh * 8 * 128, nb);
       }
+      // arrives once this lane's copies of the tile have landed; the producer
+      // never blocks on its own copies
+      cp_async_arrive_noinc(&full[s]);
     }
+    cp_async_wait<0>();                 // nothing in flight when the CTA retires
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = umma_idesc(1 /*BF16*/, DSA_HEADS, NR);
       constexpr uint32_t idesc_pv = umma_idesc(1 /*BF16*/, DSA_HEADS, 256, 0, 1);
-      bool ok = mbar_wait(q_full, 0, a.err);
-      for (int t = 0; t <= ntiles && ok; ++t) {
-        if (t < ntiles) {
-          const int s = t % NST, sb = t & 1;
-          if (!mbar_wait(&full[s], (t / NST) & 1, a.err)) break;
-          if (!mbar_wait(&s_empty[sb], ((t >> 1) & 1) ^ 1, a.err)) break;
+      bool ok = mbar_wait(q_ready, 0, a.err);
+      tc_fence_after();
+      const uint32_t qra = smem_u32(qrope);
+      for (int u = 0; u <= ntiles && ok; ++u) {
+        if (u < ntiles) {
+          const int sb = u & 1, s = u % NST;
+          if (!(ok = mbar_wait(&slot_free[sb], ((u >> 1) & 1) ^ 1, a.err))) break;
+          if (!(ok = mbar_wait(&full[s], (u / NST) & 1, a.err))) break;
+          // the tile was written by cp.async (generic proxy); order it before
+          // the tensor core's shared-memory reads (async proxy)
+          fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t qa = smem_u32(qs), ta = smem_u32(st + s * STAGE_BYTES);
-          for (int c = 0; c < nch; ++c) {
+          const uint32_t ta = smem_u32(st + s * STAGE_BYTES);
+          const uint32_t d = tmem + S_COL + sb * NR;
+          // 256 dims with q from tensor memory: k-step kk reads chunk kk/4
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_f16(tmem + S_COL + sb * NR,
-                      umma_desc_sw128(qa + c * CHUNK_Q + kk * 32, 1024, 16),
-                      umma_desc_sw128(ta + c * CHUNK_T + kk * 32, 1024, 16), idesc_s,
-                      (c | kk) != 0);
-            }
-          }
+          for (int kk = 0; kk < 16; ++kk)
+            mma_f16_ts(d, tmem + Q_COL + kk * 8,
+                       umma_desc_sw128(ta + (kk >> 2) * CHUNK_T + (kk & 3) * 32, 1024, 16),
+                       idesc_s, kk > 0);
+          // this CTA's 32 of the 64 RoPE dims: q from shared memory
+#pragma unroll
+          for (int kk = 2 * rank; kk < 2 * rank + 2; ++kk)
+            mma_f16(d, umma_desc_sw128(qra + kk * 32, 1024, 16),
+                    umma_desc_sw128(ta + 4 * CHUNK_T + kk * 32, 1024, 16), idesc_s, 1u);
           mma_commit(&s_full[sb]);
         }
-        if (t >= 1) {
-          const int u = t - 1, ub = u & 1, us = u % NST;
-          if (!mbar_wait(&p_full[ub], (u >> 1) & 1, a.err)) break;
+        if (u >= 1) {
+          const int t = u - 1, pbuf = t & 1, s = t % NST;
+          if (!(ok = mbar_wait(&p_full[pbuf], (t >> 1) & 1, a.err))) break;
           tc_fence_after();
-          const uint32_t pa = smem_u32(pb + ub * P_BYTES), va = smem_u32(st + us * STAGE_BYTES);
-          // k-steps 0,1: P_hi x V rows 0-15, 16-31; k-steps 2,3: P_lo x the same rows
+          const uint32_t pa = tmem + S_COL + pbuf * NR;   // P_hi cols [0,32), P_lo [32,64)
+          const uint32_t va = smem_u32(st + s * STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 2 * (NR / 16); ++kk) {
-            mma_f16(tmem + O_COL, umma_desc_sw128(pa + kk * 32, 1024, 16),
-                    umma_desc_sw128_mn(va + (kk % (NR / 16)) * 2048, CHUNK_T, 1024), idesc_pv,
-                    (u > 0 || kk > 0) ? 1u : 0u);
+            // k-steps 0..3: P_hi x rows 16kk..; 4..7: P_lo x the same rows
+            mma_f16_ts(tmem + O_COL, pa + kk * 8,
+                       umma_desc_sw128_mn(va + (kk & 3) * 2048, CHUNK_T, 1024), idesc_pv,
+                       (t > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&p_empty[ub]);
+          mma_commit(&slot_free[pbuf]);
+          mma_commit(&empty[s]);
           mma_commit(o_done);
-          mma_commit(&empty[us]);
-          if (u == ntiles - 1) mma_commit(o_final);
+          if (t == ntiles - 1) mma_commit(o_final);
         }
       }
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int g = (warp - 2) >> 2;                 // warpgroup: tile rows [32g, 32g+32)
+    const int gt = tid - 64;                       // 0..255 within the softmax warps
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t peer = rank ^ 1u;
     const uint32_t peer_x = map_to_rank(smem_u32(xb), peer);
-    float m_use = -INFINITY, l = 0.f;
+    // partial scores are exchanged by pull: each CTA writes its own partial
+    // into its own shared memory, signals the peer, and reads the peer's with
+    // remote loads (all in flight at once)
+    if (g == 0) {
+      // this CTA's 256 latent query dims of head h -> tensor memory (bf16 pairs)
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(src + c * 8 + i);
+          w[4 * i + 0] = __uint_as_float(v.x);
+          w[4 * i + 1] = __uint_as_float(v.y);
+          w[4 * i + 2] = __uint_as_float(v.z);
+          w[4 * i + 3] = __uint_as_float(v.w);
+        }
+        tmem_st32(lane_base + Q_COL + c * 32, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    float m_use = -INFINITY, l = 0.f;                // l: this warpgroup's rows only
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
       const int sb = t & 1;
       const uint32_t ph = (t >> 1) & 1;
-      const int jrow = t * NR + lane;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, jrow < r1 - r0 && crd[jrow] >= 0);
+      const int j = t * NR + 32 * g + lane;
+      const uint32_t vm = __ballot_sync(0xffffffffu, j < nrows && crd[j] >= 0);
       if (!(ok = warp_wait(&s_full[sb], ph, a.err))) break;
       tc_fence_after();
-      float v[NR];
-      tmem_ld32(lane_base + S_COL + sb * NR, v);
+      float z[32];
+      tmem_ld32(lane_base + S_COL + sb * NR + 32 * g, z);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
-      // my partial scores -> the peer's exchange slot; the warp barrier orders
-      // all lanes' stores before lane 0's cluster-scope release arrive
-      const uint32_t dst = peer_x + sb * X_BYTES + h * NR * 4;
+      // my partial -> my own exchange slot; the warp barrier orders all lanes'
+      // stores before lane 0's cluster-scope release arrive at the peer
+      // layout [row group of 4][head] in float4s: consecutive heads touch
+      // consecutive 16-byte words (a [head][row] layout made every access an
+      // 8-way bank conflict)
+      float4* mine = reinterpret_cast<float4*>(xb + sb * X_BYTES) + (8 * g) * DSA_HEADS + h;
 #pragma unroll
-      for (int i = 0; i < NR / 4; ++i)
-        st_cluster_v4(dst + 16 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 8; ++i)
+        mine[i * DSA_HEADS] = make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&x_full[sb]), peer));
       const bool got = mbar_wait_cluster(&x_full[sb], ph, a.err);
       if (!(ok = __all_sync(0xffffffffu, got))) break;
-      const float4* src = reinterpret_cast<const float4*>(xb + sb * X_BYTES + h * NR * 4);
-      float mt = -INFINITY;
+      float4 xs[8];
+      const uint32_t src = peer_x + sb * X_BYTES + ((8 * g) * DSA_HEADS + h) * 16;
 #pragma unroll
-      for (int i = 0; i < NR / 4; ++i) {
-        const float4 pv = src[i];
-        const float s4[4] = {pv.x, pv.y, pv.z, pv.w};
+      for (int i = 0; i < 8; ++i) xs[i] = ld_cluster_v4(src + i * DSA_HEADS * 16);
+      // own + peer: rank 0 adds S0 + S1, rank 1 adds S1 + S0; fp32 addition
+      // commutes, so both CTAs hold the same z
+      float mt0 = -INFINITY, mt1 = -INFINITY;
+      const float sl = a.scale_log2;
+      if (vm == 0xffffffffu) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int r = 4 * i + k;
-          const float z = ((vmask >> r) & 1u) ? (v[r] + s4[k]) * a.scale_log2 : -INFINITY;
-          v[r] = z;
-          mt = fmaxf(mt, z);
+        for (int i = 0; i < 8; ++i) {
+          z[4 * i + 0] = (z[4 * i + 0] + xs[i].x) * sl;
+          z[4 * i + 1] = (z[4 * i + 1] + xs[i].y) * sl;
+          z[4 * i + 2] = (z[4 * i + 2] + xs[i].z) * sl;
+          z[4 * i + 3] = (z[4 * i + 3] + xs[i].w) * sl;
+          mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
+          mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float s4[4] = {xs[i].x, xs[i].y, xs[i].z, xs[i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = 4 * i + e;
+            z[r] = ((vm >> r) & 1u) ? (z[r] + s4[e]) * sl : -INFINITY;
+          }
+          mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
+          mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
         }
       }
-      // running max, moved only when it grows by more than 8 (a factor 2^8)
+      // tile maximum over both warpgroups' rows
+      float* mxt = mx + (t & 1) * 2 * DSA_HEADS;
+      mxt[g * DSA_HEADS + h] = fmaxf(mt0, mt1);
+      named_barrier(1, 32 * SMX_WARPS);
+      const float mt = fmaxf(mxt[h], mxt[DSA_HEADS + h]);
+      // running max, moved only when it grows by more than 8 (a factor 2^8);
+      // identical in both warpgroups and both CTAs
       float alpha = 1.f;
       bool resc = false;
       if (mt > m_use + 8.f) {
@@ -305,19 +388,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         m_use = mt;
       }
-      float ps = 0.f;
+      const float m_eff = m_use == -INFINITY ? 0.f : m_use;   // exp2(-inf - m_eff) = 0
+      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const float p = (v[r] == -INFINITY) ? 0.f : fast_exp2(v[r] - m_use);
-        v[r] = p;
-        ps += p;
+      for (int r = 0; r < 32; r += 4) {
+        z[r + 0] = fast_exp2(z[r + 0] - m_eff);
+        z[r + 1] = fast_exp2(z[r + 1] - m_eff);
+        z[r + 2] = fast_exp2(z[r + 2] - m_eff);
+        z[r + 3] = fast_exp2(z[r + 3] - m_eff);
+        ps0 += z[r + 0];
+        ps1 += z[r + 1];
+        ps2 += z[r + 2];
+        ps3 += z[r + 3];
       }
-      l = l * alpha + ps;
-      // the P slot is free once PV(t-2) is done
-      if (!(ok = warp_wait(&p_empty[sb], ph ^ 1, a.err))) break;
-      if (__any_sync(0xffffffffu, resc)) {
-        // O must not move under a running PV: wait for PV(t-1)
-        if (t >= 1 && !(ok = warp_wait(o_done, (t - 1) & 1, a.err))) break;
+      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
+      // PV(t-1) done (needed before O may be rescaled).  Waited on every tile
+      // before P(t) is published, so o_done has completed t-1 or t phases
+      // here and the parity test is exact.
+      if (t >= 1 && !(ok = warp_wait(o_done, (t - 1) & 1, a.err))) break;
+      if (g == 0 && __any_sync(0xffffffffu, resc)) {
         tc_fence_after();
         for (int c = 0; c < 256 / 32; ++c) {
           float o[32];
@@ -327,61 +416,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
           tmem_st32(lane_base + O_COL + c * 32, o);
         }
-        tmem_st_wait();
-        tc_fence_before();
       }
-      // P row h as bf16 hi + lo (p ~= hi + lo to ~16 bits): hi in 16-byte
-      // chunks 0..3, lo in chunks 4..7 of the 128-byte row, 128-byte swizzle
-      // (chunk u stored at u ^ (h & 7)).  PV then runs over K = 64 =
-      // [P_hi | P_lo] against [V ; V].
-      uint8_t* prow = pb + sb * P_BYTES + h * 128;
+      // P as bf16 hi (slot columns [16g, 16g+16)) + lo ([32+16g, 32+16g+16)),
+      // two rows per column
+      {
+        float hi[16], lo[16];
 #pragma unroll
-      for (int u = 0; u < NR / 8; ++u) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __nv_bfloat162 hv = __floats2bfloat162_rn(v[8 * u + 2 * k], v[8 * u + 2 * k + 1]);
+        for (int jj = 0; jj < 16; ++jj) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(z[2 * jj], z[2 * jj + 1]);
           const float2 hf = __bfloat1622float2(hv);
-          const __nv_bfloat162 lv =
-              __floats2bfloat162_rn(v[8 * u + 2 * k] - hf.x, v[8 * u + 2 * k + 1] - hf.y);
-          hw[k] = *reinterpret_cast<const uint32_t*>(&hv);
-          lw[k] = *reinterpret_cast<const uint32_t*>(&lv);
+          const __nv_bfloat162 lv = __floats2bfloat162_rn(z[2 * jj] - hf.x, z[2 * jj + 1] - hf.y);
+          hi[jj] = __uint_as_float(bf16x2_bits(hv));
+          lo[jj] = __uint_as_float(bf16x2_bits(lv));
         }
-        *reinterpret_cast<uint4*>(prow + ((u ^ (h & 7)) * 16)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(prow + (((u + 4) ^ (h & 7)) * 16)) =
-            make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        tmem_st16(lane_base + S_COL + sb * NR + 16 * g, hi);
+        tmem_st16(lane_base + S_COL + sb * NR + 32 + 16 * g, lo);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
     }
-    // ---- epilogue: O / l for this CTA's 256 value columns; LSE from CTA 0
+    // ---- epilogue: l over both warpgroups, then O / l (warpgroup g writes
+    // columns [128g, 128g+128) of this CTA's 256); LSE from CTA 0
+    float* lsum = mx;                               // reuse: [2][128]
+    named_barrier(1, 32 * SMX_WARPS);
+    lsum[g * DSA_HEADS + h] = l;
+    named_barrier(1, 32 * SMX_WARPS);
+    const float lt = lsum[h] + lsum[DSA_HEADS + h];
     const bool have = ok && ntiles > 0 && warp_wait(o_final, 0, a.err);
     if (have) tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
     float* orow;
     float* lrow;
     if (a.S == 1) {
-      orow = a.out + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM_V + rank * 256;
+      orow = a.out + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM_V + rank * 256 + 128 * g;
       lrow = a.lse + static_cast<size_t>(q) * DSA_HEADS + h;
     } else {
-      orow = a.o_part + ((static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h) * DSA_DIM_V + rank * 256;
+      orow = a.o_part + ((static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h) * DSA_DIM_V +
+             rank * 256 + 128 * g;
       lrow = a.l_part + (static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h;
     }
-    for (int c = 0; c < 256 / 32; ++c) {
+    for (int c = 0; c < 128 / 32; ++c) {
       float o[32];
       if (have) {
-        tmem_ld32(lane_base + O_COL + c * 32, o);
+        tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
         tmem_ld_wait();
       }
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
-        float4 w = have && l > 0.f ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 w = have && lt > 0.f
+                             ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4*>(orow + c * 32 + i) = w;
       }
     }
-    if (rank == 0) *lrow = l > 0.f ? m_use * 0.69314718055994531f + logf(l) : -INFINITY;
+    if (rank == 0 && g == 0) *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
+    (void)gt;
   }
 
   tc_fence_before();
@@ -402,12 +493,9 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st) {
   if (Q <= 0) return cudaSuccess;
-  CUtensorMap tq, tkv;
+  CUtensorMap tq;
   if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, DSA_DIM,
                        static_cast<uint64_t>(Q) * DSA_HEADS, DSA_DIM * 2, 64, DSA_HEADS))
-    return cudaErrorInvalidValue;
-  if (!encode_tiled_2d(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pool, DSA_DIM,
-                       static_cast<uint64_t>(num_pages) * DSA_PAGE_SIZE, DSA_DIM * 2, 64, 1))
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -418,9 +506,9 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  MlaTcArgs a{page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
+  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
-  sparse_mla_tc_kernel<<<2 * Q * S, THREADS, SMEM_BYTES, st>>>(tq, tkv, a);
+  sparse_mla_tc_kernel<<<2 * Q * S, THREADS, SMEM_BYTES, st>>>(tq, a);
   return cudaGetLastError();
 }
 
