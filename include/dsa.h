@@ -170,6 +170,33 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
                                  void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Sparse MLA decode that allocates nothing and takes no workspace.  The
+ * pages have no counterpart of this call; it exists for callers that cannot
+ * hand the library device memory: a serving engine whose allocator already
+ * owns all of HBM (reserved up front for the paged KV cache and weights), or
+ * code that must not call cudaMalloc because it synchronises the device.
+ *   Arguments, layouts and results are those of dsa_sparse_mla_decode.
+ *   The split-K partial outputs live in a fixed 16 MiB array of device memory
+ *   owned by the library (every GPU that loads the library holds it until
+ *   the process exits), so Q * num_splits (after the library's choice when
+ *   num_splits = 0) may not exceed 63 when it is above 1; larger requests
+ *   return DSA_ERR_UNSUPPORTED and enqueue nothing.  num_splits = 1 uses no
+ *   scratch and has no limit on Q.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents; calls
+ *   whose work overlaps on the GPU (other streams, or several devices'
+ *   threads racing on one device) race on it.  Nothing in it needs to start
+ *   at zero.  Out-of-range indices or pages are skipped as in
+ *   dsa_sparse_mla_decode but are not reported (there is no error word).
+ */
+dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool, int num_pages,
+                                         const int32_t* page_table, int max_pages,
+                                         const int32_t* q_offsets, const int32_t* q_vis,
+                                         const int32_t* idx, int B, int Q, int topk, float scale,
+                                         int num_splits, float* out, float* lse, void* stream);
+
+/*
  * Merge of split-K partial attentions (exact LSE combine).
  *   o_parts fp32 [Q,S,128,512], lse_parts fp32 [Q,S,128] (-inf = empty part)
  *   out fp32 [Q,128,512], lse fp32 [Q,128].

@@ -38,6 +38,8 @@ SIGNATURES = {
     "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P,
                                    _SZ, _P]),
+    "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _F, _I, _P,
+                                           _P, _P]),
     "dsa_lse_combine": (_I, [_P, _P, _I, _I, _P, _P, _P]),
     "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _PP, _PP,
                              _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
@@ -148,6 +150,16 @@ def dsa_sparse_mla_decode(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scal
         _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], idx.shape[1], float(scale),
         num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
         "dsa_sparse_mla_decode")
+
+
+def dsa_sparse_mla_decode_noalloc(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scale, out,
+                                  lse, num_splits=0, stream=None):
+    """dsa_sparse_mla_decode without a workspace (split-K partials in the
+    library's own fixed device array; see include/dsa.h)."""
+    _check(lib().dsa_sparse_mla_decode_noalloc(
+        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
+        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], idx.shape[1], float(scale),
+        num_splits, _ptr(out), _ptr(lse), _stream(stream)), "dsa_sparse_mla_decode_noalloc")
 
 
 def dsa_lse_combine(o_parts, lse_parts, out, lse, stream=None):

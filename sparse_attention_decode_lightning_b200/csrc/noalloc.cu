@@ -1,0 +1,98 @@
+// Sparse MLA decode for callers that cannot allocate device memory.
+//
+// Some callers cannot hand this library a workspace: their device memory is
+// owned by another allocator (a serving engine that reserves the whole HBM up
+// front for its paged KV cache and weights has nothing left to give out), or
+// they must not call cudaMalloc at all because it synchronises the device and
+// would stall every stream in flight.  For them this entry point keeps the
+// split-K partial outputs in a fixed array of device memory that the library
+// itself owns, so the call allocates nothing.
+//
+// The array is a file-scope __device__ variable: every GPU that loads the
+// library holds its NOALLOC_SCRATCH_BYTES until the process exits.  In host
+// code its name is only a host-side stand-in, not a device address, so the
+// address is looked up once per device with cudaGetSymbolAddress (with that
+// device current) and cached; the first call on a device does that set-up.
+#include "common.cuh"
+#include "internal.h"
+
+#include <mutex>
+
+namespace dsa {
+
+cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
+                                 const int32_t* page_table, int max_pages,
+                                 const int32_t* q_offsets, const int32_t* q_vis,
+                                 const int32_t* idx, int B, int Q, int topk, float scale, int S,
+                                 float* out, float* lse, float* o_part, float* l_part,
+                                 uint32_t* err, cudaStream_t st);
+
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;   // 16 MiB per device
+constexpr size_t PART_O_BYTES = size_t(DSA_HEADS) * DSA_DIM_V * 4;   // one (query, split) output
+constexpr size_t PART_L_BYTES = size_t(DSA_HEADS) * 4;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// device address of g_noalloc_scratch, per device (nullptr until looked up)
+void* scratch_ptr(dsa_status* st) {
+  static void* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = DSA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      *st = DSA_ERR_CUDA;
+      return nullptr;
+    }
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool,
+                                                    int num_pages, const int32_t* page_table,
+                                                    int max_pages, const int32_t* q_offsets,
+                                                    const int32_t* q_vis, const int32_t* idx,
+                                                    int B, int Q, int topk, float scale,
+                                                    int num_splits, float* out, float* lse,
+                                                    void* stream) {
+  if (!q || !kv_pool || !page_table || !q_offsets || !q_vis || !idx || !out || !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_pool) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || topk <= 0 || num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
+  const int S = choose_splits(Q, topk, num_splits);
+  const size_t need = S > 1 ? static_cast<size_t>(Q) * S * (PART_O_BYTES + PART_L_BYTES) : 0;
+  if (need > NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;   // beyond the fixed array
+  dsa_status st = DSA_OK;
+  uint8_t* scratch = static_cast<uint8_t*>(scratch_ptr(&st));
+  if (!scratch) return st;
+  float* o_part = reinterpret_cast<float*>(scratch);
+  float* l_part = reinterpret_cast<float*>(scratch + static_cast<size_t>(Q) * S * PART_O_BYTES);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // every partial is written by the kernel before the merge reads it, so the
+  // array needs no clearing; range violations are skipped but not reported
+  if (launch_sparse_mla_tc(static_cast<const __nv_bfloat16*>(q),
+                           static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_table,
+                           max_pages, q_offsets, q_vis, idx, B, Q, topk, scale, S, out, lse, o_part,
+                           l_part, nullptr, s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (S > 1 && launch_combine(o_part, l_part, Q, S, out, lse, s) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
