@@ -57,6 +57,40 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_traffic(kernel_file: str, profile: str):
+    """Per-launch DRAM traffic (read + write bytes) recorded from an ncu capture
+    in profiles/, or None when the kernel source changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", profile)
+    src = os.path.join(ROOT, "sparse_attention_decode_lightning_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch", "source_sha256_16"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if fields.get("source_sha256_16") != sha or "traffic_bytes_per_launch" not in fields:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
+def reduce_over_ranks(local_ms: float, world: int, dist=None, device=None) -> float:
+    """Slowest rank's device time (ms): the job finishes when its last rank does."""
+    if world <= 1 or dist is None:
+        return local_ms
+    import torch
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Units all ranks processed per second over the slowest rank's time."""
+    return units_per_rank * world * steps / (total_ms / 1e3)
+
+
 def algorithmic_bytes(inp):
     """Roofline bytes of one step: indexer FP8 keys read (once per sequence and
     indexer layer) + bf16 latent rows gathered (576 x 2 B per selected token,
@@ -245,11 +279,7 @@ def run_ours(args, rank, world, local_rank):
     clocks = clk.summary()
     dsa.dsa_check_error(ws, stream)
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_over_ranks(sum(step_ms), world, dist, dev)
 
     # ---- per-kernel breakdown of the same step, live (decomposed calls, same kernels)
     scores = torch.empty(Q, ((inp.max_len + 63) // 64) * 64, device=dev)
@@ -312,12 +342,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
             ev[i][1].record(stream)
         barrier()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in ev)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": Q * world * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        e2e_ms = reduce_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dist, dev)
+        e2e = {"value": job_throughput(Q, world, args.steps, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         dsa.dsa_check_error(ws, stream)
 
@@ -329,7 +355,7 @@ def run_ours(args, rank, world, local_rank):
     step_mean_ms = total_ms / args.steps
     launches_per_step = ng * (1 + 3 + (1 if inp.mtp_index_share else 0)) + n * (1 + (1 if S > 1 else 0))
     res = {
-        "metric": METRIC, "value": Q * world * args.steps / (total_ms / 1e3), "unit": UNIT,
+        "metric": METRIC, "value": job_throughput(Q, world, args.steps, total_ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_mean_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 indexer, bf16 attention, f32 accumulate", "data": "synthetic",
@@ -340,7 +366,9 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (FP8 keys) and a 256 MiB L2 flush before every step"},
         "roofline": {"bound": "hbm", "kernel": "indexer_kernel", "achieved": achieved, "peak": hbm,
                      "peak_source": hbm_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None},
+                     "traffic": (measured_traffic("indexer_sm100.cu", "indexer_kernel_decode_b8_ctx128k.md")
+                                 if wl.name == DEFAULT_WORKLOAD and not args.batch else None),
+                     "traffic_note": "ncu dram read+write of a batch-8 capture scaled x4 to the batch-32 launch"},
         "step_roofline": {"bytes_per_step": key_b + gat_b, "key_bytes": key_b, "gather_bytes": gat_b,
                           "achieved_gbs": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9,
                           "frac_of_measured": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9 / hbm,
