@@ -5,25 +5,25 @@
 // query one relevance scalar; it streams the whole key cache, which makes it
 // the HBM-bound part of the decode step.
 //
-// Design (persistent, warp-specialised, one CTA per SM):
-//   warp 0      TMA producer: 128-key x 128-byte e4m3 tiles (16 KB, 128-byte
-//               swizzle) into an 8-stage shared-memory ring; the queries of the
-//               current sequence (8 KB each) into a query buffer.
-//   warps 1,2   two tcgen05 issuers, one per pipeline; pipeline p takes the
-//               CTA's key tiles of parity p: for every query of the tile's
-//               sequence, D[128 keys, 64 heads] = K_tile . q^T as 4 MMAs of
-//               kind::f8f6f4 (M=128, N=64, K=32) into one of its 4 TMEM slots
-//               (64 columns each, all 512 columns in use).  A single issuer
-//               thread spends ~1500 cycles per tile on mbarrier waits, MMA
-//               issue and commits, which alone caps a CTA near 25 GB/s; two
-//               independent issuers double that.
-//   warps 3..10 two epilogue warpgroups, one per pipeline: each thread reads
-//               its key row (64 fp32 head dots) with tcgen05.ld and reduces
-//               sum_h w_h * max(d_h, 0) in registers; 128 consecutive fp32
-//               scores per warpgroup are written coalesced.
-// Work: the flattened list of (sequence, 128-key tile) items is cut into
-// equal contiguous ranges, one per CTA; a sequence's keys are read once for
-// all of its queries (MTP verify positions share the tile).
+// Design (persistent, one CTA per SM, two independent sub-pipelines):
+// the CTA's contiguous range of (sequence, 128-key tile) items is cut in two
+// halves, one per pipeline, and each pipeline has
+//   a producer warp   TMA loads of 128-key x 128-byte e4m3 tiles (16 KB,
+//                     128-byte swizzle, L2 evict-first) into its own ring,
+//                     and the queries of its current sequence (8 KB each);
+//   an issuer warp    for every query of the tile's sequence, D[128 keys, 64
+//                     heads] = K_tile . q^T as 4 MMAs of kind::f8f6f4 (M=128,
+//                     N=64, K=32) into one of its 4 TMEM slots;
+//   an epilogue warpgroup   each thread reads its key row (64 fp32 head
+//                     dots) with tcgen05.ld and reduces sum_h w_h max(d_h, 0)
+//                     in registers; scores are written coalesced.
+// A single issuer thread spends ~1500 cycles per tile on mbarrier waits, MMA
+// issue and commits (measured with per-role clock64 timelines), which alone
+// caps a CTA near 25 GB/s; two issuers that never wait on each other double
+// it.  The ring depth per pipeline is chosen at run time from the largest
+// number of queries per sequence (the query buffer holds them all).
+// A sequence's keys are read once for all of its queries (MTP verify
+// positions share each tile).
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,24 +32,25 @@ namespace dsa {
 namespace {
 
 constexpr int KT = 128;                                // keys per tile (MMA M)
-constexpr int STAGES = 8;                              // key-tile ring depth
-constexpr int NACC = 8;                                // TMEM accumulator slots (all 512 columns)
+constexpr int PIPES = 2;                               // independent sub-pipelines per CTA
+constexpr int SLOTS = 4;                               // TMEM accumulator slots per pipeline
 constexpr int ACC_COLS = DSA_IDX_HEADS;                // 64 fp32 columns per slot
-constexpr int PIPES = 2;                               // MMA issuer + epilogue warpgroup pairs
-constexpr int SLOTS_PER_PIPE = NACC / PIPES;
-constexpr int THREADS = 32 + PIPES * 32 + PIPES * 128;
+constexpr int WARPS_PER_PIPE = 6;                      // producer, MMA issuer, 4 epilogue warps
+constexpr int THREADS = 32 * WARPS_PER_PIPE * PIPES;
 constexpr int KEY_TILE = KT * DSA_IDX_DIM;             // 16384 B
 constexpr int Q_TILE = DSA_IDX_HEADS * DSA_IDX_DIM;    // 8192 B
-constexpr int OFF_KEYS = 0;
-constexpr int OFF_Q = OFF_KEYS + STAGES * KEY_TILE;
-constexpr int OFF_PREFIX = OFF_Q + DSA_MAX_Q_PER_SEQ * Q_TILE;
+constexpr int MAX_STAGES = 6;                          // per pipeline
+constexpr int OFF_PREFIX = 0;
 constexpr int OFF_SCAN = OFF_PREFIX + ((DSA_MAX_BATCH + 1) * 4 + 15) / 16 * 16;
+constexpr int NBAR_PIPE = 2 * MAX_STAGES + 2 * SLOTS + 3;
 constexpr int OFF_BAR = OFF_SCAN + 64 * 4;
-constexpr int NBAR = 2 * STAGES + 2 * NACC + 2 + PIPES;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;           // slack for 1024-byte alignment
+constexpr int OFF_MISC = OFF_BAR + PIPES * NBAR_PIPE * 8;
+constexpr int OFF_DATA = (OFF_MISC + 16 + 1023) / 1024 * 1024;   // per-pipeline rings + query buffers
+constexpr int SMEM_BYTES = 230400;                     // dynamic shared memory requested
+constexpr int DATA_BYTES = SMEM_BYTES - 1024 - OFF_DATA;
 static_assert(SMEM_BYTES <= 232448, "indexer shared memory exceeds the sm_100 limit");
+static_assert(DATA_BYTES >= PIPES * (2 * KEY_TILE + DSA_MAX_Q_PER_SEQ * Q_TILE),
+              "two stages and a full query buffer must fit per pipeline");
 
 struct IdxArgs {
   const float* w;
@@ -63,7 +64,7 @@ struct IdxArgs {
   uint32_t* err;
 };
 
-// queries of sequence b that this launch scores (0 if the entry is invalid)
+// queries of sequence b that this launch scores (-1 if the entry is invalid)
 __device__ __forceinline__ int seq_queries(const IdxArgs& a, int b) {
   const int n = a.q_offsets[b + 1] - a.q_offsets[b];
   if (n < 0 || n > DSA_MAX_Q_PER_SEQ) return -1;
@@ -118,30 +119,33 @@ __device__ void block_exclusive_scan(int* x, int n, int* tmp) {
   __syncthreads();
 }
 
+// largest b with prefix[b] <= t (prefix non-decreasing over [0, B])
+__device__ __forceinline__ int seq_of_tile(const int* prefix, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_q, IdxArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* keys = smem + OFF_KEYS;
-  uint8_t* qbuf = smem + OFF_Q;
   int* prefix = reinterpret_cast<int*>(smem + OFF_PREFIX);
   int* scan_tmp = reinterpret_cast<int*>(smem + OFF_SCAN);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;
-  uint64_t* acc_empty = acc_full + NACC;
-  uint64_t* q_full = acc_empty + NACC;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* mma_done = q_full + 2;        // one per pipeline
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  int* s_maxq = reinterpret_cast<int*>(smem + OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = a.B;
 
-  // ---- tiles per sequence -> exclusive prefix over the batch
+  // ---- tiles per sequence -> exclusive prefix over the batch; largest query count
+  if (tid == 0) *s_maxq = 1;
+  __syncthreads();
   for (int b = tid; b < B; b += THREADS) {
     const int nq = seq_queries(a, b);
     bool bad = nq < 0;
@@ -151,47 +155,65 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < nq; ++j) mv = max(mv, query_vis(a, a.q_offsets[b] + j, len < 0 ? 0 : len, &bad));
     if (bad) raise_error(a.err, DEVERR_BOUNDS);
     prefix[b] = (nq <= 0 || len < 0) ? 0 : (mv + KT - 1) / KT;
+    if (nq > 1) atomicMax(s_maxq, nq);
   }
   __syncthreads();
   block_exclusive_scan(prefix, B, scan_tmp);
+  const int maxq = *s_maxq;
+  // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of maxq tiles]
+  const int pipe_bytes = (DATA_BYTES / PIPES) / 1024 * 1024;
+  const int stages = min(MAX_STAGES, (pipe_bytes - maxq * Q_TILE) / KEY_TILE);
 
-  if (tid == 0) {
-    for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < NACC; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, PIPES);        // every MMA issuer releases the query buffer
-    for (int p = 0; p < PIPES; ++p) mbar_init(&mma_done[p], 1);
+  const int pipe = warp / WARPS_PER_PIPE;          // 0 / 1
+  const int pw = warp % WARPS_PER_PIPE;            // role within the pipeline
+  uint8_t* keys = smem + OFF_DATA + pipe * pipe_bytes;
+  uint8_t* qbuf = keys + stages * KEY_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR) + pipe * NBAR_PIPE;
+  uint64_t* full = bars;
+  uint64_t* empty = bars + MAX_STAGES;
+  uint64_t* acc_full = bars + 2 * MAX_STAGES;
+  uint64_t* acc_empty = acc_full + SLOTS;
+  uint64_t* q_full = acc_empty + SLOTS;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* mma_done = q_full + 2;
+
+  if (tid < PIPES) {
+    uint64_t* pb = reinterpret_cast<uint64_t*>(smem + OFF_BAR) + tid * NBAR_PIPE;
+    for (int i = 0; i < MAX_STAGES; ++i) { mbar_init(&pb[i], 1); mbar_init(&pb[MAX_STAGES + i], 1); }
+    for (int i = 0; i < SLOTS; ++i) {
+      mbar_init(&pb[2 * MAX_STAGES + i], 1);
+      mbar_init(&pb[2 * MAX_STAGES + SLOTS + i], 4);
+    }
+    mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 0], 1);   // q_full
+    mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 1], 1);   // q_empty
+    mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 2], 1);   // mma_done
     mbar_fence_init();
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_q);
+    if (tid == 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+    }
   }
-  if (warp == 1) tmem_alloc(tmem_holder, NACC * ACC_COLS);
+  if (warp == 1) tmem_alloc(tmem_holder, PIPES * SLOTS * ACC_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem = *tmem_holder + pipe * SLOTS * ACC_COLS;
 
+  // this CTA's tiles, then this pipeline's contiguous half of them
   const int total = prefix[B];
-  const int t_begin = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
-  const int t_end = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+  const int c_begin = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
+  const int c_end = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+  const int c_mid = c_begin + (c_end - c_begin + 1) / 2;
+  const int t_begin = pipe == 0 ? c_begin : c_mid;
+  const int t_end = pipe == 0 ? c_mid : c_end;
+  const int b_first = t_begin < t_end ? seq_of_tile(prefix, B, t_begin) : 0;
 
-  // first sequence of this CTA's range: largest b with prefix[b] <= t_begin
-  int b_first = 0;
-  if (t_begin < t_end) {
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (prefix[mid] <= t_begin) lo = mid; else hi = mid - 1;
-    }
-    b_first = lo;
-  }
-
-  if (warp == 0) {
+  if (pw == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && t_begin < t_end) {
       const uint64_t pol = l2_policy_evict_first();
       int b = b_first, cur_b = -1;
-      uint32_t stage = 0, phase = 0, qphase = 0, issued = 0, q_issued = 0;
+      uint32_t issued = 0, q_issued = 0, qphase = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
         while (prefix[b + 1] <= i) ++b;
@@ -208,34 +230,31 @@ __global__ void __launch_bounds__(THREADS, 1)
           ++q_issued;
           cur_b = b;
         }
-        if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], KEY_TILE);
+        const uint32_t s = issued % stages;
+        if (!mbar_wait(&empty[s], ((issued / stages) & 1) ^ 1, a.err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[s], KEY_TILE);
         const int64_t row = a.seq_offsets[b] + static_cast<int64_t>(t) * KT;
-        tma_load_2d_hint(keys + stage * KEY_TILE, &tmap_k, 0, static_cast<int>(row), &full[stage], pol);
+        tma_load_2d_hint(keys + s * KEY_TILE, &tmap_k, 0, static_cast<int>(row), &full[s], pol);
         ++issued;
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) {
         // drain the copies still in flight before the CTA's memory goes away
-        const uint32_t n = issued < STAGES ? issued : STAGES;
+        const uint32_t n = issued < static_cast<uint32_t>(stages) ? issued : stages;
         for (uint32_t k = 0; k < n; ++k) {
           const uint32_t it = issued - 1 - k;
-          mbar_wait(&full[it % STAGES], (it / STAGES) & 1, a.err);
+          mbar_wait(&full[it % stages], (it / stages) & 1, a.err);
         }
         if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1, a.err);
       }
     }
-  } else if (warp <= 2) {
-    // ------------------------------------------------------------ MMA issuers
-    // pipeline p = warp - 1 owns the CTA's tiles of parity p and TMEM slots
-    // 4p .. 4p+3; both walk every tile to keep the query-buffer hand-off in step
-    const int pipe = warp - 1;
+  } else if (pw == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && t_begin < t_end) {
       constexpr uint32_t idesc = umma_idesc(0 /*E4M3*/, KT, ACC_COLS);
       int b = b_first, cur_b = -1, nq = 0;
-      uint32_t qphase = 0, n = 0;
+      uint32_t qphase = 0, n = 0, k = 0;
       bool ok = true;
-      for (int i = t_begin; i < t_end && ok; ++i) {
+      for (int i = t_begin; i < t_end && ok; ++i, ++k) {
         while (prefix[b + 1] <= i) ++b;
         if (b != cur_b) {
           if (cur_b >= 0) mma_commit(q_empty);
@@ -244,15 +263,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           nq = seq_queries(a, b);
           cur_b = b;
         }
-        const int local = i - t_begin;
-        if ((local & 1) != pipe) continue;
-        const int stage = local % STAGES;
-        if (!mbar_wait(&full[stage], (local / STAGES) & 1, a.err)) { ok = false; break; }
+        const uint32_t s = k % stages;
+        if (!mbar_wait(&full[s], (k / stages) & 1, a.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(keys + stage * KEY_TILE);
+        const uint32_t a_base = smem_u32(keys + s * KEY_TILE);
         for (int j = 0; j < nq; ++j, ++n) {
-          const uint32_t slot = pipe * SLOTS_PER_PIPE + n % SLOTS_PER_PIPE;
-          if (!mbar_wait(&acc_empty[slot], ((n / SLOTS_PER_PIPE) & 1) ^ 1, a.err)) { ok = false; break; }
+          const uint32_t slot = n % SLOTS;
+          if (!mbar_wait(&acc_empty[slot], ((n / SLOTS) & 1) ^ 1, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t b_base = smem_u32(qbuf + j * Q_TILE);
 #pragma unroll
@@ -263,31 +280,33 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_commit(&acc_full[slot]);
         }
         if (!ok) break;
-        mma_commit(&empty[stage]);
+        mma_commit(&empty[s]);
       }
       // every MMA this thread issued must finish before TMEM is released
-      mma_commit(&mma_done[pipe]);
-      mbar_wait(&mma_done[pipe], 0, a.err);
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.err);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     if (t_begin < t_end) {
-      const int g = (warp - 3) >> 2;           // warpgroup = pipeline 0 / 1
       const int quarter = warp & 3;            // TMEM lanes this warp may read
       const int row = quarter * 32 + lane;     // key row of the tile
-      int b = b_first;
+      int b = b_first, cur_b = -1, nq = 0, q0 = 0;
+      int64_t len = 0;
       uint32_t n = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
         while (prefix[b + 1] <= i) ++b;
-        if (((i - t_begin) & 1) != g) continue;
+        if (b != cur_b) {
+          nq = seq_queries(a, b);
+          q0 = a.q_offsets[b];
+          len = a.seq_offsets[b + 1] - a.seq_offsets[b];
+          cur_b = b;
+        }
         const int t = i - prefix[b];
-        const int nq = seq_queries(a, b);
-        const int q0 = a.q_offsets[b];
-        const int64_t len = a.seq_offsets[b + 1] - a.seq_offsets[b];
         for (int j = 0; j < nq; ++j, ++n) {
-          const uint32_t slot = g * SLOTS_PER_PIPE + n % SLOTS_PER_PIPE;
-          if (!mbar_wait(&acc_full[slot], (n / SLOTS_PER_PIPE) & 1, a.err)) { ok = false; break; }
+          const uint32_t slot = n % SLOTS;
+          if (!mbar_wait(&acc_full[slot], (n / SLOTS) & 1, a.err)) { ok = false; break; }
           tc_fence_after();
           float v[ACC_COLS];
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * ACC_COLS;
@@ -325,7 +344,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NACC * ACC_COLS);
+    tmem_dealloc(*tmem_holder, PIPES * SLOTS * ACC_COLS);
   }
 }
 
