@@ -92,8 +92,8 @@ int dsa_version(void);
  * Bytes of device workspace the calls below need for Q queries, contexts of at
  * most max_len keys, `topk` selected tokens and `num_splits` split-K parts
  * (0 = let the library choose).  The workspace holds the fp32 score rows
- * [Q, max_len], the selector's histograms and candidate lists, the split-K
- * partial outputs and the device error flag.  The same workspace may be
+ * [Q, max_len], the split-K partial outputs and the device error flag (the
+ * selector keeps its histograms and candidate lists in on-chip memory).  The same workspace may be
  * reused by consecutive calls on one stream; it must be zeroed once
  * (cudaMemset) before its first use so the error flag starts clear.
  * Returns 0 for invalid sizes.
@@ -125,7 +125,8 @@ dsa_status dsa_indexer_scores(const uint8_t* q_idx, const float* w, const uint8_
  *   first_only != 0: only the first query of each sequence (rows
  *           q_offsets[b]) is selected; other rows are untouched.
  * Exact: the set equals a full sort by (score desc, position asc); -0 == +0.
- * Scores must not be NaN.  ws: dsa_workspace_bytes(Q, ld_scores, topk, 1) bytes.
+ * Scores must not be NaN.  ws: at least 256 bytes (only the error flag at its
+ * start is used; any workspace from dsa_workspace_bytes qualifies).
  */
 dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_offsets,
                            const int32_t* q_vis, int B, int Q, int max_len, int topk,

@@ -61,10 +61,6 @@ bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* L) {
   size_t off = 0;
   w.err = off;      off = align_up(off + 256, 256);
   w.scores = off;   off = align_up(off + static_cast<size_t>(Q) * w.ld * 4, 256);
-  w.hist = off;     off = align_up(off + static_cast<size_t>(Q) * TOPK_BINS * 4, 256);
-  w.meta = off;     off = align_up(off + static_cast<size_t>(Q) * TOPK_META * 4, 256);
-  w.cand = off;     off = align_up(off + static_cast<size_t>(Q) * w.ld * 8, 256);
-  w.cand2 = off;    off = align_up(off + static_cast<size_t>(Q) * w.ld * 8, 256);
   w.o_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * DSA_DIM_V * 4, 256);
   w.l_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * 4, 256);
   w.total = off;
@@ -123,8 +119,7 @@ dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* 
                                  Q, first_only, scores, L.ld, err, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
-                  out_scores, ws_ptr<uint32_t>(ws, L.hist), ws_ptr<uint32_t>(ws, L.meta),
-                  ws_ptr<uint64_t>(ws, L.cand), ws_ptr<uint64_t>(ws, L.cand2), err, st);
+                  out_scores, err, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (first_only) {
     e = launch_expand_idx(q_offsets, B, Q, topk, out_idx, out_scores, st);
@@ -226,15 +221,11 @@ dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_
   if (B <= 0 || Q <= 0 || max_len <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
   if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
   if (ld_scores < max_len || (ld_scores & 3) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
-  // the selector's candidate lists are sized by the score row stride
-  WsLayout L;
-  if (!ws_layout(Q, ld_scores, topk, 1, &L)) return DSA_ERR_INVALID_ARG;
-  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  // the selector keeps its working set on chip; the workspace holds the error flag
+  if (ws_bytes < 256) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_topk(scores, ld_scores, q_offsets, q_vis, B, Q, max_len, topk,
-                              first_only, out_idx, out_scores, ws_ptr<uint32_t>(ws, L.hist),
-                              ws_ptr<uint32_t>(ws, L.meta), ws_ptr<uint64_t>(ws, L.cand),
-                              ws_ptr<uint64_t>(ws, L.cand2), ws_ptr<uint32_t>(ws, L.err), st);
+                              first_only, out_idx, out_scores, static_cast<uint32_t*>(ws), st);
   return cuda_status(e);
 }
 

@@ -12,17 +12,10 @@
 
 namespace dsa {
 
-constexpr int TOPK_BINS = 4096;   // first-level histogram: top 12 bits of the score key
-constexpr int TOPK_META = 4;      // per-query counters: [0] above-threshold, [1] candidates
-
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct WsLayout {
   size_t err = 0;      // uint32 error flag (+ padding)
   size_t scores = 0;   // fp32 [Q, ld]
-  size_t hist = 0;     // uint32 [Q, TOPK_BINS]
-  size_t meta = 0;     // uint32 [Q, TOPK_META]
-  size_t cand = 0;     // uint64 [Q, ld]   candidate (key, position) pairs
-  size_t cand2 = 0;    // uint64 [Q, ld]   ping-pong for the refinement passes
   size_t o_part = 0;   // fp32 [Q, S, 128, 512]
   size_t l_part = 0;   // fp32 [Q, S, 128]
   size_t total = 0;
@@ -48,8 +41,7 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
                         const int32_t* q_vis, int B, int Q, int max_len, int topk,
-                        int first_only, int32_t* out_idx, float* out_scores, uint32_t* hist,
-                        uint32_t* meta, uint64_t* cand, uint64_t* cand2, uint32_t* err,
+                        int first_only, int32_t* out_idx, float* out_scores, uint32_t* err,
                         cudaStream_t st);
 
 cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,

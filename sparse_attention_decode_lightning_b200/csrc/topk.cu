@@ -2,26 +2,58 @@
 // lower position ("大语言模型结构总览", section 2.2: the token selector keeps the
 // k = 2048 best-scoring tokens; section 7.2: causal top-2048).
 //
-// Exact radix select over 64-bit keys  (order-preserving u32 of the fp32
-// score) << 32 | (0xFFFFFFFF - position), which are all distinct, so "the k
-// largest keys" is exactly the top-k with the lower-position tie rule.
-//   pass 1 (hist):    many CTAs per query build a 4096-bin histogram of the top
-//                     12 key bits (shared-memory atomics, merged in global).
-//   pass 2 (filter):  every CTA finds the bin holding the k-th key; keys above
-//                     it are written out, keys inside it become candidates.
-//   pass 3 (resolve): one CTA per query refines the candidates 8 bits at a
-//                     time until the remaining candidates are exactly needed.
-// Scores are read twice (from L2 when the indexer just wrote them); the
-// candidate set is the small slice of the distribution at the threshold.
+// One kernel launch, one thread-block cluster of C CTAs per query row.  The
+// row's visible positions are cut into C contiguous slices; every CTA copies
+// its slice into shared memory with bulk copies (a slice longer than
+// SLICE_CAP keeps its head there and re-reads the rest from global memory)
+// and turns the scores into order-preserving u32 keys in place.
+//
+// Exact radix select on the composite key of position s
+//     V(s) = (u(s) << pb) | s,   u(s) = kmax - key(I[s]),   pb = bits(vis - 1)
+// with kmax the largest key of the row.  V is distinct per position and a
+// smaller V is a better position (higher score, then lower position), so the
+// topk smallest V are exactly the top-k with the lower-position tie rule.
+// Measuring u from the row's own maximum makes the first 12-bit digit span
+// the row's score range [kmin, kmax] only: the 4096 first-level bins are
+// narrow and the bin holding the k-th score has few positions.
+//
+// Steps ('|' is a cluster barrier):
+//   bulk copy, keys, local min/max | row min/max
+//   pass 1: 4096-bin histogram of the top digit of V | every CTA sums the C
+//           histograms through distributed shared memory (1024 bins at a
+//           time, stopping at the chunk that holds the threshold digit t:
+//           the smallest d with count(digits <= d) >= k)
+//   then one of
+//   exact:  bin t holds exactly the positions still needed: every CTA writes
+//           its positions with digit <= t to the output | done
+//   gather: bin t has at most CAND_CAP positions over the row: every CTA
+//           writes its positions with digit < t to the output and pushes its
+//           bin-t positions into rank 0's shared memory | rank 0 finishes the
+//           selection among them alone (12-bit passes, block barriers only)
+//   rescan: (degenerate score sets) further 12-bit passes over the slices
+//           with a cluster merge each, then as "exact".
+// Output slots are handed out by an atomic on a counter in rank 0's shared
+// memory, so the index row is in no particular order.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dsa {
 namespace {
 
-constexpr int CHUNK = 8192;     // scores per CTA in passes 1 and 2
-constexpr int PT = 512;         // threads for passes 1 and 2
-constexpr int RT = 1024;        // threads for pass 3
+constexpr int THREADS = 1024;
+constexpr int DIGIT = 12;                     // bits per radix pass
+constexpr int BINS = 1 << DIGIT;
+constexpr int CHUNK = 4 * THREADS;            // scores per bulk copy: one float4 per thread
+constexpr int NCHUNK = 10;
+constexpr int SLICE_CAP = NCHUNK * CHUNK;     // 40960 scores a CTA keeps in shared memory
+constexpr int CAND_CAP = 4096;                // bin-t positions rank 0 gathers
+constexpr int MAX_CLUSTER = 8;                // portable cluster size
+constexpr int MIN_SLICE = 2048;               // rows are not cut finer than this
+static_assert(BINS == 4 * THREADS, "bins are merged THREADS at a time, scanned 4 per thread");
+
+constexpr size_t smem_bytes(int scap) {
+  return static_cast<size_t>(scap) * 4 + 2 * BINS * 4 + CAND_CAP * 8;
+}
 
 struct TopkArgs {
   const float* scores;
@@ -31,11 +63,8 @@ struct TopkArgs {
   int B, Q, max_len, topk, first_only;
   int32_t* out_idx;
   float* out_scores;
-  uint32_t* hist;
-  uint32_t* meta;
-  uint64_t* cand;
-  uint64_t* cand2;
   uint32_t* err;
+  int scap;             // slice elements held in shared memory (multiple of 4)
 };
 
 // query handled by grid row y, or -1
@@ -54,262 +83,414 @@ __device__ __forceinline__ int clamped_vis(const TopkArgs& a, int q) {
   return v;
 }
 
-__global__ void __launch_bounds__(PT) topk_hist_kernel(TopkArgs a) {
-  __shared__ uint32_t h[TOPK_BINS];
-  const int q = row_query(a, blockIdx.y);
-  if (q < 0) return;
-  const int vis = clamped_vis(a, q);
-  if (vis <= a.topk) return;                         // every visible key is kept
-  const int beg = blockIdx.x * CHUNK;
-  if (beg >= vis) return;
-  const int end = min(vis, beg + CHUNK);
-  for (int i = threadIdx.x; i < TOPK_BINS; i += PT) h[i] = 0;
-  __syncthreads();
-  const float* row = a.scores + static_cast<size_t>(q) * a.ld;
-  for (int i = beg + 4 * threadIdx.x; i < end; i += 4 * PT) {
-    const float4 v = *reinterpret_cast<const float4*>(row + i);
-    atomicAdd(&h[float_key(v.x) >> 20], 1u);
-    if (i + 1 < end) atomicAdd(&h[float_key(v.y) >> 20], 1u);
-    if (i + 2 < end) atomicAdd(&h[float_key(v.z) >> 20], 1u);
-    if (i + 3 < end) atomicAdd(&h[float_key(v.w) >> 20], 1u);
+// Calls f(position, key, valid) for every element of the slice, in the same
+// order on every call.  Groups of four that lie wholly inside the on-chip copy
+// take the first loop, where valid is the constant true; the rest (the
+// ragged tail and any part beyond scap, read from global memory and
+// converted) take the second.
+template <class F>
+__device__ __forceinline__ void for_slice(const uint32_t* s_key, const float* grow, int beg, int n,
+                                          int scap, F&& f) {
+  const int full = min(n, scap) & ~(4 * THREADS - 1);   // whole steps of 4*THREADS on chip
+  const int j0 = 4 * static_cast<int>(threadIdx.x);
+  for (int base = 0; base < full; base += 4 * THREADS) {
+    const int j = base + j0;
+    const uint4 k = *reinterpret_cast<const uint4*>(s_key + j);
+    f(beg + j, k.x, true);
+    f(beg + j + 1, k.y, true);
+    f(beg + j + 2, k.z, true);
+    f(beg + j + 3, k.w, true);
   }
-  __syncthreads();
-  uint32_t* g = a.hist + static_cast<size_t>(q) * TOPK_BINS;
-  for (int i = threadIdx.x; i < TOPK_BINS; i += PT)
-    if (h[i]) atomicAdd(&g[i], h[i]);
+  for (int j = full + j0; j < n; j += 4 * THREADS) {
+    uint4 k;
+    if (j < scap) {
+      k = *reinterpret_cast<const uint4*>(s_key + j);
+    } else {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(grow + j));
+      k = make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w));
+    }
+    f(beg + j, k.x, true);
+    f(beg + j + 1, k.y, j + 1 < n);
+    f(beg + j + 2, k.z, j + 2 < n);
+    f(beg + j + 3, k.w, j + 3 < n);
+  }
 }
 
-// threshold bin of a histogram: largest bin b with count(bins >= b) >= k;
-// returns b and count(bins > b) through shared memory.  nthreads*per == bins.
-template <int NT, int BINS>
-__device__ void find_threshold(const uint32_t* hist, uint32_t k, uint32_t* s_bin,
-                               uint32_t* s_above, uint32_t* s_tmp) {
-  constexpr int PER = BINS / NT;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // thread t owns bins [BINS - PER*(t+1), BINS - PER*t), i.e. counted from the top
-  const int hi = BINS - PER * tid;
-  uint32_t c[PER];
-  uint32_t sum = 0;
-#pragma unroll
-  for (int j = 0; j < PER; ++j) { c[j] = hist[hi - 1 - j]; sum += c[j]; }
-  uint32_t incl = sum;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += y;
-  }
-  if (lane == 31) s_tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    constexpr int NW = NT / 32;
-    const uint32_t v = lane < NW ? s_tmp[lane] : 0;
-    uint32_t vi = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, vi, off);
-      if (lane >= off) vi += y;
-    }
-    if (lane < NW) s_tmp[lane] = vi - v;
-  }
-  __syncthreads();
-  uint32_t run = s_tmp[warp] + incl - sum;     // count in bins above this thread's range
-#pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    if (run < k && run + c[j] >= k) { *s_bin = static_cast<uint32_t>(hi - 1 - j); *s_above = run; }
-    run += c[j];
-  }
-  __syncthreads();
-}
-
-__global__ void __launch_bounds__(PT, 2) topk_filter_kernel(TopkArgs a) {
-  __shared__ uint32_t s_tmp[32];
-  __shared__ uint32_t s_bin, s_above;
-  const int q = row_query(a, blockIdx.y);
-  if (q < 0) return;
-  const int vis = clamped_vis(a, q);
-  const int beg = blockIdx.x * CHUNK;
-  const float* row = a.scores + static_cast<size_t>(q) * a.ld;
-  int32_t* oi = a.out_idx + static_cast<size_t>(q) * a.topk;
-  float* os = a.out_scores ? a.out_scores + static_cast<size_t>(q) * a.topk : nullptr;
-  if (vis <= a.topk) {                               // keep all visible positions
-    const int end = min(vis, beg + CHUNK);
-    for (int i = beg + threadIdx.x; i < end; i += PT) {
-      oi[i] = i;
-      if (os) os[i] = row[i];
-    }
-    return;
-  }
-  if (beg >= vis) return;
-  const int end = min(vis, beg + CHUNK);
-  find_threshold<PT, TOPK_BINS>(a.hist + static_cast<size_t>(q) * TOPK_BINS,
-                                static_cast<uint32_t>(a.topk), &s_bin, &s_above, s_tmp);
-  const uint32_t tb = s_bin;
-  uint32_t* meta = a.meta + static_cast<size_t>(q) * TOPK_META;
-  if (blockIdx.x == 0 && threadIdx.x == 0) { meta[2] = tb; meta[3] = s_above; }
-  uint64_t* cand = a.cand + static_cast<size_t>(q) * a.ld;
-  // each thread holds its CHUNK / PT scores in registers; slots are reserved
-  // with one block scan and one global atomic per counter per CTA
-  constexpr int PER4 = CHUNK / (4 * PT);
-  float4 v[PER4];
-  uint32_t na = 0, nc = 0;
-#pragma unroll
-  for (int k = 0; k < PER4; ++k) {
-    const int i = beg + 4 * (threadIdx.x + k * PT);
-    v[k] = i < end ? *reinterpret_cast<const float4*>(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t bin = float_key(vv[e]) >> 20;
-      const bool valid = i + e < end;
-      na += (valid && bin > tb);
-      nc += (valid && bin == tb);
-    }
-  }
-  // block exclusive scan of (na << 16 | nc); totals stay below 2^16 per CTA
-  const uint32_t packed = (na << 16) | nc;
+// Exclusive prefix sum of x over the CTA in thread order, and the CTA total.
+// Every thread calls it; s_warp holds one word per warp.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* s_warp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t incl = packed;
+  uint32_t incl = x;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += y;
   }
-  __shared__ uint32_t s_warp[PT / 32];
-  __shared__ uint32_t s_base_a, s_base_c;
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const uint32_t x = lane < PT / 32 ? s_warp[lane] : 0;
-    uint32_t xi = x;
+  const uint32_t wt = s_warp[lane];            // THREADS / 32 == 32 warp totals
+  uint32_t wi = wt;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, xi, off);
-      if (lane >= off) xi += y;
-    }
-    if (lane < PT / 32) s_warp[lane] = xi - x;
-    if (lane == 31) {
-      s_base_a = (xi >> 16) ? atomicAdd(&meta[0], xi >> 16) : 0;
-      s_base_c = (xi & 0xFFFFu) ? atomicAdd(&meta[1], xi & 0xFFFFu) : 0;
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
+    if (lane >= off) wi += y;
+  }
+  *total = __shfl_sync(0xffffffffu, wi, 31);
+  const uint32_t wbase = __shfl_sync(0xffffffffu, wi - wt, warp);
+  __syncthreads();                             // s_warp may be reused after this
+  return wbase + incl - x;
+}
+
+// Threshold digit of a histogram whose bins 4*tid .. 4*tid+3 this thread
+// holds in c: the smallest d with count(digits <= d) >= need.  Publishes d,
+// the count below it and its count through s_t, s_cb, s_cnt.
+__device__ __forceinline__ void find_threshold4(const uint32_t c[4], uint32_t need, uint32_t* s_warp,
+                                                uint32_t* s_t, uint32_t* s_cb, uint32_t* s_cnt) {
+  const uint32_t tot = c[0] + c[1] + c[2] + c[3];
+  uint32_t all;
+  uint32_t before = block_excl_scan(tot, s_warp, &all);
+  if (before < need && before + tot >= need) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (before < need && before + c[k] >= need) {
+        *s_t = 4 * threadIdx.x + k;
+        *s_cb = before;
+        *s_cnt = c[k];
+      }
+      before += c[k];
     }
   }
   __syncthreads();
-  const uint32_t pre = s_warp[warp] + incl - packed;
-  uint32_t pa = s_base_a + (pre >> 16), pc = s_base_c + (pre & 0xFFFFu);
-#pragma unroll
-  for (int k = 0; k < PER4; ++k) {
-    const int i = beg + 4 * (threadIdx.x + k * PT);
-    const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t key = float_key(vv[e]);
-      const uint32_t bin = key >> 20;
-      if (i + e < end) {
-        if (bin > tb) {
-          oi[pa] = i + e;
-          if (os) os[pa] = vv[e];
-          ++pa;
-        } else if (bin == tb) {
-          cand[pc++] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i + e));
-        }
-      }
-    }
-  }
 }
 
-__global__ void __launch_bounds__(RT) topk_resolve_kernel(TopkArgs a) {
-  __shared__ uint32_t h[256];
-  __shared__ uint32_t s_tmp[32];
-  __shared__ uint32_t s_digit, s_gt, s_out, s_n;
-  const int q = row_query(a, blockIdx.x);
-  if (q < 0) return;
+__global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(smem);                  // scores, then keys
+  uint32_t* s_hist = s_key + a.scap;                                     // [2][BINS]
+  uint64_t* s_cand = reinterpret_cast<uint64_t*>(s_hist + 2 * BINS);    // rank 0: gathered V
+  __shared__ __align__(8) uint64_t s_bar[NCHUNK];
+  __shared__ uint32_t s_red[64];
+  __shared__ uint32_t s_warp[32];
+  __shared__ __align__(8) uint32_t s_mm[2];     // this CTA's min and max key
+  __shared__ uint32_t s_gmm[2];                 // the row's
+  __shared__ uint32_t s_t, s_cb, s_cnt;         // threshold digit, count below it, its count
+  __shared__ __align__(8) uint64_t s_ctr;      // rank 0: output slots | gathered candidates << 32
+  __shared__ uint32_t s_obase, s_cbase;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = static_cast<int>(gridDim.x);    // cluster = one grid row
+  const uint32_t rank = cluster_ctarank();
+  const int q = row_query(a, blockIdx.y);
+  if (q < 0) return;                            // the whole cluster leaves
   const int vis = clamped_vis(a, q);
-  int32_t* oi = a.out_idx + static_cast<size_t>(q) * a.topk;
-  float* os = a.out_scores ? a.out_scores + static_cast<size_t>(q) * a.topk : nullptr;
-  if (vis <= a.topk) {
-    for (int i = vis + threadIdx.x; i < a.topk; i += RT) {
-      oi[i] = -1;
-      if (os) os[i] = -INFINITY;
+  const int topk = a.topk;
+  const float* row = a.scores + static_cast<size_t>(q) * a.ld;
+  int32_t* oi = a.out_idx + static_cast<size_t>(q) * topk;
+  float* os = a.out_scores ? a.out_scores + static_cast<size_t>(q) * topk : nullptr;
+
+  if (vis <= topk) {                            // every visible position, then padding
+    for (int i = static_cast<int>(rank) * THREADS + tid; i < topk; i += C * THREADS) {
+      oi[i] = i < vis ? i : -1;
+      if (os) os[i] = i < vis ? row[i] : -INFINITY;
     }
+    return;                                     // the whole cluster leaves
+  }
+
+  // This CTA's slice [beg, beg + n), beg a multiple of 4.  Every read (bulk
+  // copies and float4 loads) ends at round_up(beg + n, 4) <= ld, since beg
+  // and ld are multiples of 4 and beg + n <= vis <= ld.
+  const int L = (((vis + C - 1) / C) + 3) & ~3;
+  const int beg = min(vis, static_cast<int>(rank) * L);
+  const int n = max(0, min(vis, beg + L) - beg);
+  const float* grow = row + beg;
+  const int nsm = min(n, a.scap);               // elements copied on chip
+  const int nch = (nsm + CHUNK - 1) / CHUNK;
+
+  if (tid == 0) {
+    for (int c = 0; c < nch; ++c) mbar_init(&s_bar[c], 1);
+    mbar_fence_init();
+    for (int c = 0; c < nch; ++c) {
+      const int e0 = c * CHUNK;
+      const uint32_t bytes = static_cast<uint32_t>(((min(CHUNK, nsm - e0) + 3) & ~3) * 4);
+      mbar_arrive_expect_tx(&s_bar[c], bytes);
+      bulk_load(s_key + e0, grow + e0, bytes, &s_bar[c]);
+    }
+    s_ctr = 0;
+  }
+  for (int i = tid; i < 2 * BINS; i += THREADS) s_hist[i] = 0;
+  __syncthreads();                              // barriers initialised before any wait
+
+  // ---- keys in place and local min / max, chunk by chunk as the copies land
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  auto minmax4 = [&](uint4 k, int j, int lim) {
+    const uint32_t e[4] = {k.x, k.y, k.z, k.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (j + t < lim) {
+        kmin = min(kmin, e[t]);
+        kmax = max(kmax, e[t]);
+      }
+  };
+  for (int c = 0; c < nch; ++c) {
+    mbar_wait(&s_bar[c], 0, a.err);
+    const int j = c * CHUNK + 4 * tid;
+    if (j < nsm) {
+      const float4 v = *reinterpret_cast<const float4*>(s_key + j);
+      const uint4 k = make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w));
+      *reinterpret_cast<uint4*>(s_key + j) = k;
+      minmax4(k, j, nsm);
+    }
+  }
+  for (int j = a.scap + 4 * tid; j < n; j += 4 * THREADS) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(grow + j));
+    minmax4(make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w)), j, n);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) { s_red[warp] = kmin; s_red[32 + warp] = kmax; }
+  __syncthreads();
+  if (warp == 0) {
+    kmin = __reduce_min_sync(0xffffffffu, s_red[lane]);
+    kmax = __reduce_max_sync(0xffffffffu, s_red[32 + lane]);
+    if (lane == 0) { s_mm[0] = kmin; s_mm[1] = kmax; }
+  }
+  cluster_sync();            // min/max of every CTA, keys, zeroed histograms and counters
+  if (warp == 0) {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    if (lane < C) {
+      const uint2 r = ld_cluster_u2(map_to_rank(smem_u32(s_mm), static_cast<uint32_t>(lane)));
+      mn = r.x;
+      mx = r.y;
+    }
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) { s_gmm[0] = mn; s_gmm[1] = mx; }
+  }
+  __syncthreads();
+  const uint32_t gmax = s_gmm[1];
+  const uint32_t range = gmax - s_gmm[0];
+  const int pb = 32 - __clz(vis - 1);                   // vis >= 2 here
+  const uint64_t pos_mask = (1ull << pb) - 1ull;
+  auto make_v = [&](int pos, uint32_t key) -> uint64_t {
+    return (static_cast<uint64_t>(gmax - key) << pb) | static_cast<uint64_t>(pos);
+  };
+
+  // ---- pass 1: the top DIGIT bits of V.  When sh0 >= pb (a score range of
+  // at least 2^12 keys, the usual case) the digit is (kmax - key) >> (sh0 - pb)
+  // and every later test on it is a comparison of the key with a bound.
+  const int tb = (range ? 32 - __clz(range) : 0) + pb;  // significant bits of V
+  const int w0 = min(DIGIT, tb);
+  const int sh0 = tb - w0;
+  const uint32_t dmask0 = (1u << w0) - 1u;
+  const bool fast0 = sh0 >= pb;
+  const int us0 = fast0 ? sh0 - pb : 0;
+  auto digit0 = [&](int pos, uint32_t key) -> uint32_t {   // general form
+    return (((gmax - key) << (pb - sh0)) | (static_cast<uint32_t>(pos) >> sh0)) & dmask0;
+  };
+  if (fast0) {
+    for_slice(s_key, grow, beg, n, a.scap, [&](int, uint32_t key, bool valid) {
+      if (valid) atomicAdd(&s_hist[(gmax - key) >> us0], 1u);
+    });
+  } else {
+    for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+      if (valid) atomicAdd(&s_hist[digit0(pos, key)], 1u);
+    });
+  }
+  cluster_sync();            // every CTA's pass-1 histogram is complete
+
+  // threshold digit of the cluster's summed histograms; h = this pass's buffer
+  auto merged_threshold = [&](const uint32_t* h, uint32_t need) {
+    uint32_t carry = 0;
+    for (int c0 = 0; c0 < BINS; c0 += THREADS) {
+      const uint32_t a0 = smem_u32(h + c0 + tid);
+      uint32_t m = 0;
+      for (int r = 0; r < C; ++r) m += ld_cluster_u32(map_to_rank(a0, static_cast<uint32_t>(r)));
+      uint32_t tot;
+      const uint32_t ex = carry + block_excl_scan(m, s_warp, &tot);
+      if (ex < need && ex + m >= need) {
+        s_t = static_cast<uint32_t>(c0 + tid);
+        s_cb = ex;
+        s_cnt = m;
+      }
+      carry += tot;
+      if (carry >= need) break;
+    }
+    __syncthreads();
+  };
+  // "exact" / "rescan" ending: every slice position with sel(pos, key) is
+  // written to the output; slots from rank 0's counter, then a cluster barrier
+  auto write_selected = [&](auto sel) {
+    uint32_t cnt = 0;
+    for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+      cnt += valid && sel(pos, key);
+    });
+    uint32_t tot;
+    const uint32_t pre = block_excl_scan(cnt, s_warp, &tot);
+    if (tid == 0)
+      s_obase = static_cast<uint32_t>(atom_add_cluster_u64(map_to_rank(smem_u32(&s_ctr), 0u), tot));
+    __syncthreads();
+    uint32_t o = s_obase + pre;
+    for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+      if (valid && sel(pos, key)) {
+        if (o < static_cast<uint32_t>(topk)) {
+          oi[o] = pos;
+          if (os) os[o] = key_float(key);
+        } else {
+          raise_error(a.err, DEVERR_BOUNDS);
+        }
+        ++o;
+      }
+    });
+    cluster_sync();          // rank 0's counter stays alive until every CTA took its slots
+  };
+
+  reinterpret_cast<uint4*>(s_hist + BINS)[tid] = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t need = static_cast<uint32_t>(topk);
+  merged_threshold(s_hist, need);
+  const uint32_t t0 = s_t;
+  need -= s_cb;
+  const uint32_t cnt0 = s_cnt;
+
+  // digit < t0 ("better") and digit <= t0 ("in"): in the fast form
+  // key >= kb1 and key >= kin1, from u < t0 << us0 and u < (t0 + 1) << us0
+  const uint32_t kb1 = gmax - (t0 << us0) + 1u;              // t0 << us0 <= range <= gmax
+  const uint64_t u2 = static_cast<uint64_t>(t0 + 1u) << us0;
+  const uint32_t kin1 = u2 > gmax ? 0u : static_cast<uint32_t>(gmax - u2 + 1u);
+  auto fast_better = [&](int, uint32_t key) { return key >= kb1; };
+  auto fast_in = [&](int, uint32_t key) { return key >= kin1; };
+  auto gen_better = [&](int pos, uint32_t key) { return digit0(pos, key) < t0; };
+  auto gen_in = [&](int pos, uint32_t key) { return digit0(pos, key) <= t0; };
+
+  if (cnt0 == need) {
+    // ---- exact: positions with digit <= t0
+    if (fast0) write_selected(fast_in);
+    else write_selected(gen_in);
     return;
   }
-  const uint32_t* meta = a.meta + static_cast<size_t>(q) * TOPK_META;
-  uint32_t base = meta[3];                     // positions already written
-  uint32_t need = static_cast<uint32_t>(a.topk) - base;
-  uint32_t n = meta[1];                        // candidates in the threshold bin
-  uint64_t* src = a.cand + static_cast<size_t>(q) * a.ld;
-  uint64_t* dst = a.cand2 + static_cast<size_t>(q) * a.ld;
-  if (n < need || n > static_cast<uint32_t>(a.ld)) {   // inconsistent counters
-    if (threadIdx.x == 0) raise_error(a.err, DEVERR_BOUNDS);
-    n = min(n, need);
-  }
-  // 52 low bits remain undecided: 20 score bits below the 12-bit bin, 32 position bits
-  for (int pass = 0; pass <= 7; ++pass) {
-    if (n == need || pass == 7) {
-      for (uint32_t j = threadIdx.x; j < n && j < need; j += RT) {
-        const uint64_t e = src[j];
-        oi[base + j] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
-        if (os) os[base + j] = key_float(static_cast<uint32_t>(e >> 32));
+
+  if (cnt0 <= static_cast<uint32_t>(CAND_CAP)) {
+    // ---- gather: digit < t0 goes out now, digit == t0 goes to rank 0
+    auto gather = [&](auto better, auto in) {
+      uint32_t nb = 0, ni = 0;
+      for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+        nb += valid && better(pos, key);
+        ni += valid && in(pos, key);
+      });
+      // per CTA nb < topk and ni - nb <= cnt0 <= CAND_CAP: both halves stay below 2^16
+      uint32_t tot;
+      const uint32_t pre = block_excl_scan((nb << 16) | (ni - nb), s_warp, &tot);
+      const uint32_t nb_cta = tot >> 16;
+      if (tid == 0) {
+        // rank 0 also takes the slots of the `need` positions it will pick from bin t0
+        const uint64_t add =
+            (static_cast<uint64_t>(tot & 0xFFFFu) << 32) | (nb_cta + (rank == 0 ? need : 0u));
+        const uint64_t old = atom_add_cluster_u64(map_to_rank(smem_u32(&s_ctr), 0u), add);
+        s_obase = static_cast<uint32_t>(old) + (rank == 0 ? nb_cta : 0u);   // rank 0: its picks
+        s_cbase = static_cast<uint32_t>(old >> 32);
       }
-      break;
-    }
-    // digit positions 44, 36, 28, 20, 12, 4 (8 bits each), then bits 3..0
-    const int sh = pass < 6 ? 44 - 8 * pass : 0;
-    const uint32_t mask = pass < 6 ? 0xFFu : 0xFu;
-    for (int i = threadIdx.x; i < 256; i += RT) h[i] = 0;
-    if (threadIdx.x == 0) { s_out = 0; s_n = 0; s_digit = 0; s_gt = 0; }
-    __syncthreads();
-    for (uint32_t j = threadIdx.x; j < n; j += RT)
-      atomicAdd(&h[static_cast<uint32_t>(src[j] >> sh) & mask], 1u);
-    __syncthreads();
-    {
-      // threshold digit: largest d with count(digits >= d) >= need
-      uint32_t c = threadIdx.x < 256 ? h[255 - threadIdx.x] : 0;
-      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-      uint32_t incl = c;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      if (lane == 31) s_tmp[warp] = incl;
       __syncthreads();
-      if (warp == 0) {
-        const uint32_t v = s_tmp[lane];
-        uint32_t vi = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, vi, off);
-          if (lane >= off) vi += y;
+      uint32_t o = s_obase - (rank == 0 ? nb_cta : 0u) + (pre >> 16);
+      uint32_t ci = s_cbase + (pre & 0xFFFFu);
+      const uint32_t cand0 = map_to_rank(smem_u32(s_cand), 0u);
+      for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+        if (valid && in(pos, key)) {
+          if (better(pos, key)) {
+            if (o < static_cast<uint32_t>(topk)) {
+              oi[o] = pos;
+              if (os) os[o] = key_float(key);
+            } else {
+              raise_error(a.err, DEVERR_BOUNDS);
+            }
+            ++o;
+          } else {
+            if (ci < static_cast<uint32_t>(CAND_CAP)) st_cluster_u64(cand0 + ci * 8u, make_v(pos, key));
+            else raise_error(a.err, DEVERR_BOUNDS);
+            ++ci;
+          }
         }
-        s_tmp[lane] = vi - v;
+      });
+    };
+    if (fast0) gather(fast_better, fast_in);
+    else gather(gen_better, gen_in);
+    cluster_sync();          // bin t0 gathered in rank 0; the other CTAs are done
+    if (rank != 0) return;
+
+    // rank 0: the `need` smallest V among the cnt0 gathered candidates
+    const uint32_t picks = need;
+    uint64_t P = t0;
+    int rem = sh0;
+    for (;;) {
+      const int w = min(DIGIT, rem);
+      const int sh = rem - w;
+      const uint32_t dmask = (1u << w) - 1u;
+      reinterpret_cast<uint4*>(s_hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();
+      for (uint32_t i = tid; i < cnt0; i += THREADS) {
+        const uint64_t V = s_cand[i];
+        if ((V >> rem) == P) atomicAdd(&s_hist[static_cast<uint32_t>(V >> sh) & dmask], 1u);
       }
       __syncthreads();
-      const uint32_t before = s_tmp[warp] + incl - c;   // count in digits above
-      if (threadIdx.x < 256 && before < need && before + c >= need) {
-        s_digit = 255u - threadIdx.x;
-        s_gt = before;
-      }
-      __syncthreads();
+      const uint4 h4 = reinterpret_cast<const uint4*>(s_hist)[tid];
+      const uint32_t c4[4] = {h4.x, h4.y, h4.z, h4.w};
+      find_threshold4(c4, need, s_warp, &s_t, &s_cb, &s_cnt);
+      need -= s_cb;
+      P = (P << w) | s_t;
+      rem = sh;
+      if (s_cnt == need || rem == 0) break;   // rem == 0 implies s_cnt == need == 1
     }
-    const uint32_t d = s_digit, gt = s_gt;
-    for (uint32_t j = threadIdx.x; j < n; j += RT) {
-      const uint64_t e = src[j];
-      const uint32_t dg = static_cast<uint32_t>(e >> sh) & mask;
-      if (dg > d) {
-        const uint32_t p = base + atomicAdd(&s_out, 1u);
-        oi[p] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(e));
-        if (os) os[p] = key_float(static_cast<uint32_t>(e >> 32));
-      } else if (dg == d) {
-        dst[atomicAdd(&s_n, 1u)] = e;
+    const uint64_t VT = (P << rem) | ((1ull << rem) - 1ull);
+    uint32_t c = 0;
+    for (uint32_t i = tid; i < cnt0; i += THREADS) c += s_cand[i] <= VT;
+    uint32_t picked;
+    uint32_t op = s_obase + block_excl_scan(c, s_warp, &picked);
+    for (uint32_t i = tid; i < cnt0; i += THREADS) {
+      const uint64_t V = s_cand[i];
+      if (V <= VT) {
+        if (op < static_cast<uint32_t>(topk)) {
+          oi[op] = static_cast<int32_t>(V & pos_mask);
+          if (os) os[op] = key_float(gmax - static_cast<uint32_t>(V >> pb));
+        } else {
+          raise_error(a.err, DEVERR_BOUNDS);
+        }
+        ++op;
       }
     }
-    __syncthreads();
-    base += gt;
-    need -= gt;
-    n = h[d];
-    uint64_t* t = src; src = dst; dst = t;
-    __syncthreads();
+    if (tid == 0 && picked != picks) raise_error(a.err, DEVERR_BOUNDS);
+    return;
   }
+
+  // ---- rescan (bin t0 holds more than CAND_CAP positions): further passes
+  // over the slices, positions alive while V's decided bits equal P
+  uint64_t P = t0;
+  int rem = sh0;
+  for (int pass = 1;; ++pass) {
+    const int w = min(DIGIT, rem);
+    const int sh = rem - w;
+    const uint32_t dmask = (1u << w) - 1u;
+    uint32_t* h = s_hist + (pass & 1) * BINS;
+    for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+      if (valid) {
+        const uint64_t V = make_v(pos, key);
+        if ((V >> rem) == P) atomicAdd(&h[static_cast<uint32_t>(V >> sh) & dmask], 1u);
+      }
+    });
+    cluster_sync();          // every CTA's histogram of this pass is complete
+    // the other buffer was last read remotely before this barrier
+    reinterpret_cast<uint4*>(s_hist + ((pass + 1) & 1) * BINS)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    merged_threshold(h, need);
+    need -= s_cb;
+    P = (P << w) | s_t;
+    rem = sh;
+    if (s_cnt == need || rem == 0) break;     // rem == 0 implies s_cnt == need == 1
+  }
+  // V <= V_T as (u, position) <= (uT, pT); uT fits 32 bits since V_T < 2^(32 + pb)
+  const uint64_t VT = (P << rem) | ((1ull << rem) - 1ull);
+  const uint32_t uT = static_cast<uint32_t>(VT >> pb);
+  const uint32_t pT = static_cast<uint32_t>(VT & pos_mask);
+  write_selected([&](int pos, uint32_t key) {
+    const uint32_t u = gmax - key;
+    return u < uT || (u == uT && static_cast<uint32_t>(pos) <= pT);
+  });
 }
 
 __global__ void expand_idx_kernel(const int32_t* q_offsets, int Q, int topk, int32_t* out_idx,
@@ -326,26 +507,53 @@ __global__ void expand_idx_kernel(const int32_t* q_offsets, int Q, int topk, int
   }
 }
 
+// CTAs per query row: enough clusters to cover the SMs once, at most 8 (the
+// portable cluster size) and no slice shorter than MIN_SLICE
+int topk_cluster_size(int rows, int max_len) {
+  int C = device_sm_count() / (rows > 0 ? rows : 1);
+  C = C < 1 ? 1 : (C > MAX_CLUSTER ? MAX_CLUSTER : C);
+  const int by_len = max_len / MIN_SLICE;
+  if (C > by_len) C = by_len < 1 ? 1 : by_len;
+  return C;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
                         const int32_t* q_vis, int B, int Q, int max_len, int topk,
-                        int first_only, int32_t* out_idx, float* out_scores, uint32_t* hist,
-                        uint32_t* meta, uint64_t* cand, uint64_t* cand2, uint32_t* err,
+                        int first_only, int32_t* out_idx, float* out_scores, uint32_t* err,
                         cudaStream_t st) {
   const int rows = first_only ? B : Q;
   if (rows <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(Q) * TOPK_BINS * sizeof(uint32_t), st);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(meta, 0, static_cast<size_t>(Q) * TOPK_META * sizeof(uint32_t), st);
-  if (e != cudaSuccess) return e;
+  if (rows > 65535 || topk > DSA_MAX_TOPK) return cudaErrorInvalidValue;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes(SLICE_CAP)));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int C = topk_cluster_size(rows, max_len);
+  const int slice = (((max_len + C - 1) / C) + 3) & ~3;
+  const int scap = slice < SLICE_CAP ? slice : SLICE_CAP;
   TopkArgs a{scores, ld, q_offsets, q_vis, B, Q, max_len, topk, first_only,
-             out_idx, out_scores, hist, meta, cand, cand2, err};
-  const dim3 grid((max_len + CHUNK - 1) / CHUNK, rows);
-  topk_hist_kernel<<<grid, PT, 0, st>>>(a);
-  topk_filter_kernel<<<grid, PT, 0, st>>>(a);
-  topk_resolve_kernel<<<rows, RT, 0, st>>>(a);
-  return cudaGetLastError();
+             out_idx, out_scores, err, scap};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(C), static_cast<unsigned>(rows), 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes(scap);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a);
 }
 
 cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk, int32_t* out_idx,

@@ -52,9 +52,11 @@ def test_workspace_bytes_arithmetic():
     assert f(1, 10, 4096, 0) == 0
     assert f(1, 10, 2048, 33) == 0
     small = f(1, 8192, 2048, 1)
-    # scores fp32 + two candidate lists of 8 bytes per key, histogram, one partial output
-    assert small >= 8192 * 4 + 2 * 8192 * 8 + 4096 * 4 + 128 * 512 * 4
-    assert f(32, 131072, 2048, 1) > 32 * 131072 * 20
+    # error flag + fp32 score row + one partial output and its LSE row
+    assert small >= 256 + 8192 * 4 + 128 * 512 * 4 + 128 * 4
+    assert f(32, 131072, 2048, 1) >= 32 * 131072 * 4
+    # the selector's working set is on chip: nothing per key beyond the fp32 score
+    assert f(32, 131072, 2048, 1) < 32 * 131072 * 4 + (64 << 20)
     assert f(4, 1 << 20, 2048, 16) > f(4, 1 << 20, 2048, 1)
     assert f(4, 1 << 20, 2048, 16) - f(4, 1 << 20, 2048, 1) >= 4 * 15 * 128 * 512 * 4
 

@@ -80,10 +80,15 @@ def _topk_case(name, rng):
         return (10.0 + rng.random(40000) * 1e-3).astype(np.float32)
     if name == "long":
         return (rng.standard_normal(200000) * 7).astype(np.float32)
+    if name == "very_long":       # slices longer than the on-chip copy: tails re-read
+        return (rng.standard_normal(400000) * 7).astype(np.float32)
+    if name == "long_int_ties":   # threshold bin too large for the candidate lists
+        return rng.integers(-3, 4, 400000).astype(np.float32)
     raise KeyError(name)
 
 
-@pytest.mark.parametrize("case", ["normal", "int_ties", "all_equal", "signed_zero", "narrow_band", "long"])
+@pytest.mark.parametrize("case", ["normal", "int_ties", "all_equal", "signed_zero", "narrow_band",
+                                  "long", "very_long", "long_int_ties"])
 def test_topk_select_exact_on_fixed_scores(case):
     rng = np.random.default_rng(7)
     x = _topk_case(case, rng)
