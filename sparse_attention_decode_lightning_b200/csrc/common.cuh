@@ -399,6 +399,18 @@ __device__ __forceinline__ uint64_t atom_add_cluster_u64(uint32_t addr, uint64_t
   return old;
 }
 
+// 16-byte store into another CTA's shared memory that counts its bytes as
+// completed transactions on an mbarrier in that CTA (no separate arrive and
+// no release fence: the receiver's wait covers the data)
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                            uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          cluster_addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
+      : "memory");
+}
+
 // arrive (release at cluster scope) on an mbarrier that lives in another CTA of the cluster
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
