@@ -58,6 +58,7 @@ constexpr int CHUNK_T = NR * 128;              // 8 KB: 64 rows x 64 bf16
 constexpr int STAGE_BYTES = MAXCH * CHUNK_T;   // 40 KB
 constexpr int QROPE_BYTES = DSA_HEADS * 128;   // 16 KB: 128 heads x 64 bf16
 constexpr int X_BYTES = DSA_HEADS * NR * 4;    // 32 KB: one tile of fp32 partial scores
+constexpr int OBOX_BYTES = DSA_HEADS * 128;    // 16 KB: output box of 128 heads x 32 fp32
 constexpr int OFF_QR = 0;
 constexpr int OFF_ST = OFF_QR + QROPE_BYTES;
 constexpr int OFF_X = OFF_ST + NST * STAGE_BYTES;
@@ -69,6 +70,7 @@ constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "sparse MLA shared memory exceeds the sm_100 limit");
 static_assert(OFF_ST % 1024 == 0 && OFF_X % 1024 == 0, "swizzle atoms");
+static_assert(8 * OBOX_BYTES <= OFF_MX - OFF_ST, "output boxes reuse the stage ring and exchange slots");
 constexpr uint32_t O_COL = 0;
 constexpr uint32_t S_COL = 256;
 constexpr uint32_t Q_COL = 384;
@@ -111,7 +113,8 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, MlaTcArgs a) {
+    sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_o, MlaTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -451,29 +454,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const bool have = ok && ntiles > 0 && warp_wait(o_final, 0, a.err);
     if (have) tc_fence_after();
     const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    float* orow;
-    float* lrow;
-    if (a.S == 1) {
-      orow = a.out + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM_V + rank * 256 + 128 * g;
-      lrow = a.lse + static_cast<size_t>(q) * DSA_HEADS + h;
-    } else {
-      orow = a.o_part + ((static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h) * DSA_DIM_V +
-             rank * 256 + 128 * g;
-      lrow = a.l_part + (static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h;
-    }
+    // O / l leaves through shared memory: warpgroup g fills four boxes of
+    // [128 heads x 32 fp32] (its columns [128g, 128g+128) of this CTA's 256)
+    // in the 128-byte swizzle, then one thread stores them with TMA.  The
+    // stage ring and the exchange slots are idle once the last PV is done.
+    float* lrow = a.S == 1 ? a.lse + static_cast<size_t>(q) * DSA_HEADS + h
+                           : a.l_part + (static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h;
+    const int orow0 = (a.S == 1 ? q : q * a.S + split) * DSA_HEADS;
+    uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
     for (int c = 0; c < 128 / 32; ++c) {
       float o[32];
       if (have) {
         tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
         tmem_ld_wait();
       }
+      uint8_t* row = box0 + c * OBOX_BYTES + h * 128;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 w = have && lt > 0.f
-                             ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(orow + c * 32 + i) = w;
+      for (int j = 0; j < 8; ++j) {
+        const float4 w = have && lt > 0.f ? make_float4(o[4 * j] * inv, o[4 * j + 1] * inv,
+                                                        o[4 * j + 2] * inv, o[4 * j + 3] * inv)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(row + ((j ^ (h & 7)) << 4)) = w;
       }
+    }
+    fence_proxy_async_smem();
+    named_barrier(2 + g, 128);
+    if (gt == 128 * g) {
+      for (int c = 0; c < 128 / 32; ++c)
+        tma_store_2d(&tmap_o, box0 + c * OBOX_BYTES, static_cast<int>(rank) * 256 + 128 * g + 32 * c,
+                     orow0);
+      bulk_commit_group();
+      bulk_wait_all();
     }
     if (rank == 0 && g == 0) *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
     (void)gt;
@@ -510,9 +521,16 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  // output boxes of 128 heads x 32 fp32 into O [Q, 128, 512] (S = 1) or the
+  // split partials [Q, S, 128, 512]
+  CUtensorMap to;
+  if (!encode_tiled_2d(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S == 1 ? out : o_part, DSA_DIM_V,
+                       static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * DSA_HEADS, DSA_DIM_V * 4, 32,
+                       DSA_HEADS))
+    return cudaErrorInvalidValue;
   MlaTcArgs a{q, pool, page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
-  sparse_mla_tc_kernel<<<2 * Q * S, THREADS, SMEM_BYTES, st>>>(tq, a);
+  sparse_mla_tc_kernel<<<2 * Q * S, THREADS, SMEM_BYTES, st>>>(tq, to, a);
   return cudaGetLastError();
 }
 
