@@ -306,45 +306,69 @@ def run_ours(args, rank, world, local_rank):
         stage["mla"].append(e[2].elapsed_time(e[3]))
     dsa.dsa_check_error(ws, stream)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs from pinned host memory, runs the decode step and reads
+    # its outputs back.  Device buffers are double-buffered and the copies run
+    # on their own streams, so step i's H2D and step i-1's D2H overlap step i's
+    # compute; the L2 flush stays inside every step, and the timed region runs
+    # from the first H2D to the last D2H.
     e2e = None
     if not args.no_e2e:
-        h_qi = [t.cpu().pin_memory() if t is not None else None for t in qi]
-        h_w = [t.cpu().pin_memory() if t is not None else None for t in wl_]
-        h_q = [t.cpu().pin_memory() for t in qs]
-        h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-        h_lse = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lses]
-        d_qi = [torch.empty_like(t) if t is not None else None for t in qi]
-        d_w = [torch.empty_like(t) if t is not None else None for t in wl_]
-        d_q = [torch.empty_like(t) for t in qs]
-        h2d = sum(t.numel() * t.element_size() for t in h_qi + h_w + h_q if t is not None)
-        d2h = sum(t.numel() * t.element_size() for t in h_out + h_lse)
+        nb = 2
+        h_in = [t.cpu().pin_memory() if t is not None else None for t in qi + wl_ + qs]
+        h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs + lses]
+        d_in = [[torch.empty_like(t) if t is not None else None for t in qi + wl_ + qs]
+                for _ in range(nb)]
+        d_res = [[torch.empty_like(o) for o in outs + lses] for _ in range(nb)]
+        h2d = sum(t.numel() * t.element_size() for t in h_in if t is not None)
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+        s_h2d = torch.cuda.Stream(dev)
+        s_d2h = torch.cuda.Stream(dev)
 
-        def e2e_step():
-            for d, h in zip(d_qi + d_w + d_q, h_qi + h_w + h_q):
-                if h is not None:
-                    d.copy_(h, non_blocking=True)
-            dsa.dsa_decode_step(d_qi, d_w, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B,
-                                inp.max_len, inp.topk, d_q, pools, pts, inp.scale, outs, lses, idx,
-                                ws, index_share=G, mtp_index_share=inp.mtp_index_share,
-                                num_splits=S, stream=stream)
-            for h, d in zip(h_out + h_lse, outs + lses):
-                h.copy_(d, non_blocking=True)
+        def e2e_run(k):
+            ev = lambda: torch.cuda.Event()  # noqa: E731
+            h2d_ev, comp_ev, d2h_ev = ([ev() for _ in range(k)] for _ in range(3))
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            s_h2d.wait_event(t0)
+            for i in range(k):
+                b = i % nb
+                if i >= nb:
+                    s_h2d.wait_event(comp_ev[i - nb])      # buffer b's previous step is done
+                with torch.cuda.stream(s_h2d):
+                    for d, h in zip(d_in[b], h_in):
+                        if h is not None:
+                            d.copy_(h, non_blocking=True)
+                h2d_ev[i].record(s_h2d)
+                stream.wait_event(h2d_ev[i])
+                if i >= nb:
+                    stream.wait_event(d2h_ev[i - nb])      # result buffer b has been read
+                flush.zero_()
+                d = d_in[b]
+                dsa.dsa_decode_step(d[:n], d[n:2 * n], kl, inp.seq_offsets, inp.q_offsets, inp.q_vis,
+                                    inp.B, inp.max_len, inp.topk, d[2 * n:], pools, pts, inp.scale,
+                                    d_res[b][:n], d_res[b][n:], idx, ws, index_share=G,
+                                    mtp_index_share=inp.mtp_index_share, num_splits=S, stream=stream)
+                comp_ev[i].record(stream)
+                s_d2h.wait_event(comp_ev[i])
+                with torch.cuda.stream(s_d2h):
+                    for h, dd in zip(h_out, d_res[b]):
+                        h.copy_(dd, non_blocking=True)
+                d2h_ev[i].record(s_d2h)
+            stream.wait_event(d2h_ev[k - 1])
+            t1.record(stream)
+            return t0, t1
 
-        for _ in range(2):
-            e2e_step()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+        e2e_run(2)
         barrier()
-        for i in range(args.steps):
-            flush.zero_()
-            ev[i][0].record(stream)
-            e2e_step()
-            ev[i][1].record(stream)
+        t0, t1 = e2e_run(args.steps)
         barrier()
-        e2e_ms = reduce_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world, dist, dev)
+        e2e_ms = reduce_over_ranks(t0.elapsed_time(t1), world, dist, dev)
         e2e = {"value": job_throughput(Q, world, args.steps, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "pinned host buffers; copies on two copy streams overlap compute "
+                       "(double-buffered); 256 MiB L2 flush inside every step"}
         dsa.dsa_check_error(ws, stream)
 
     key_b, gat_b = algorithmic_bytes(inp)

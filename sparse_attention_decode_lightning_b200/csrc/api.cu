@@ -13,7 +13,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                    const int32_t* q_offsets, const int32_t* q_vis,
                                    const int32_t* idx, int B, int Q, int topk, float scale,
                                    int S, float* out, float* lse, float* o_part, float* l_part,
-                                   uint32_t* err, cudaStream_t st);
+                                   uint32_t* err, cudaStream_t st, bool pdl);
 
 namespace {
 
@@ -118,8 +118,9 @@ dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* 
   cudaError_t e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B,
                                  Q, first_only, scores, L.ld, err, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
+  // the selector starts while the indexer drains (its scores are waited for)
   e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
-                  out_scores, err, st);
+                  out_scores, err, st, true);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (first_only) {
     e = launch_expand_idx(q_offsets, B, Q, topk, out_idx, out_scores, st);
@@ -132,17 +133,17 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
                          const int32_t* page_table, int max_pages, const int32_t* q_offsets,
                          const int32_t* q_vis, const int32_t* idx, int B, int Q, int topk,
                          float scale, int S, float* out, float* lse, void* ws,
-                         const WsLayout& L, cudaStream_t st) {
+                         const WsLayout& L, cudaStream_t st, bool pdl) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* o_part = ws_ptr<float>(ws, L.o_part);
   float* l_part = ws_ptr<float>(ws, L.l_part);
   cudaError_t e = launch_sparse_mla(static_cast<const __nv_bfloat16*>(q),
                                     static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
                                     page_table, max_pages, q_offsets, q_vis, idx, B, Q, topk,
-                                    scale, S, out, lse, o_part, l_part, err, st);
+                                    scale, S, out, lse, o_part, l_part, err, st, pdl);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (S > 1) {
-    e = launch_combine(o_part, l_part, Q, S, out, lse, st);
+    e = launch_combine(o_part, l_part, Q, S, out, lse, st, true);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
   }
   return DSA_OK;
@@ -165,9 +166,9 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               const int32_t* q_offsets, const int32_t* q_vis,
                               const int32_t* idx, int B, int Q, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
-                              uint32_t* err, cudaStream_t st) {
+                              uint32_t* err, cudaStream_t st, bool pdl) {
   return launch_sparse_mla_tc(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B,
-                              Q, topk, scale, S, out, lse, o_part, l_part, err, st);
+                              Q, topk, scale, S, out, lse, o_part, l_part, err, st, pdl);
 }
 
 }  // namespace dsa
@@ -225,7 +226,8 @@ dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_
   if (ws_bytes < 256) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_topk(scores, ld_scores, q_offsets, q_vis, B, Q, max_len, topk,
-                              first_only, out_idx, out_scores, static_cast<uint32_t*>(ws), st);
+                              first_only, out_idx, out_scores, static_cast<uint32_t*>(ws), st,
+                              false);
   return cuda_status(e);
 }
 
@@ -262,7 +264,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
   if (!ws_layout(Q, 1, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   return do_sparse_mla(q, kv_pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
-                       topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream));
+                       topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream), false);
 }
 
 dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, float* out,
@@ -272,7 +274,7 @@ dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, 
   if (Q > 65535 * 8 || S > 1024) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(o_parts) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
   return cuda_status(launch_combine(o_parts, lse_parts, Q, S, out, lse,
-                                    static_cast<cudaStream_t>(stream)));
+                                    static_cast<cudaStream_t>(stream), false));
 }
 
 dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
@@ -315,7 +317,7 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
     }
     s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
                       q_offsets, q_vis, idx_g, B, Q, topk, scale, L.S, out_layers[l],
-                      lse_layers[l], ws, L, st);
+                      lse_layers[l], ws, L, st, true);
     if (s != DSA_OK) return s;
   }
   return DSA_OK;

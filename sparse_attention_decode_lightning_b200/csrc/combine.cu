@@ -14,6 +14,8 @@ __global__ void __launch_bounds__(128) lse_combine_kernel(const float* __restric
                                                           const float* __restrict__ l_part,
                                                           int S, float* __restrict__ out,
                                                           float* __restrict__ lse) {
+  pdl_trigger();
+  pdl_wait();                                   // the partials come from the previous kernel
   const int qh = blockIdx.x;                    // q * 128 + h
   const int q = qh / DSA_HEADS, h = qh % DSA_HEADS;
   const float* lp = l_part + static_cast<size_t>(q) * S * DSA_HEADS + h;
@@ -47,10 +49,18 @@ __global__ void __launch_bounds__(128) lse_combine_kernel(const float* __restric
 }  // namespace
 
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, float* out,
-                           float* lse, cudaStream_t st) {
+                           float* lse, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
-  lse_combine_kernel<<<Q * DSA_HEADS, 128, 0, st>>>(o_part, l_part, S, out, lse);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(Q) * DSA_HEADS, 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  unsigned int na = 0;
+  add_pdl_attr(attr, &na, pdl);
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, lse_combine_kernel, o_part, l_part, S, out, lse);
 }
 
 }  // namespace dsa

@@ -476,6 +476,17 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
   return umma_desc_sw128(saddr, sbo_bytes, lbo_bytes);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with the programmatic-serialization attribute may start
+// while the previous kernel on the stream is still running; it must call
+// pdl_wait() before it touches anything that kernel writes or reads.  Both
+// are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// lets the next kernel on the stream (if launched with the attribute) be
+// scheduled as SMs free up; it still waits for this grid in pdl_wait()
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // ------------------------------------------------------------------ misc
 // order-preserving map of fp32 to u32 (larger float -> larger key); -0 == +0
 __device__ __forceinline__ uint32_t float_key(float f) {

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = a.B;
+  pdl_trigger();   // the selector after this kernel may be scheduled as SMs free up
 
   // ---- tiles per sequence -> exclusive prefix over the batch; largest query count
   if (tid == 0) *s_maxq = 1;

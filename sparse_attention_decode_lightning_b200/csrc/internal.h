@@ -42,7 +42,7 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
                         const int32_t* q_vis, int B, int Q, int max_len, int topk,
                         int first_only, int32_t* out_idx, float* out_scores, uint32_t* err,
-                        cudaStream_t st);
+                        cudaStream_t st, bool pdl);
 
 cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,
                               int32_t* out_idx, float* out_scores, cudaStream_t st);
@@ -52,9 +52,20 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               const int32_t* q_offsets, const int32_t* q_vis,
                               const int32_t* idx, int B, int Q, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
-                              uint32_t* err, cudaStream_t st);
+                              uint32_t* err, cudaStream_t st, bool pdl);
 
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, float* out,
-                           float* lse, cudaStream_t st);
+                           float* lse, cudaStream_t st, bool pdl);
+
+// pdl = true: the kernel may start before the previous kernel on the stream
+// ends (programmatic dependent launch); it waits for it in pdl_wait().  Only
+// set where the previous kernel is one of this library's, launched by the same
+// entry point, so everything older on the stream has finished before it.
+inline void add_pdl_attr(cudaLaunchAttribute* attrs, unsigned int* n, bool pdl) {
+  if (!pdl) return;
+  attrs[*n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[*n].val.programmaticStreamSerializationAllowed = 1;
+  ++*n;
+}
 
 }  // namespace dsa

@@ -25,7 +25,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int topk, float scale, int S,
                                  float* out, float* lse, float* o_part, float* l_part,
-                                 uint32_t* err, cudaStream_t st);
+                                 uint32_t* err, cudaStream_t st, bool pdl);
 
 namespace {
 
@@ -91,8 +91,9 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
   if (launch_sparse_mla_tc(static_cast<const __nv_bfloat16*>(q),
                            static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_table,
                            max_pages, q_offsets, q_vis, idx, B, Q, topk, scale, S, out, lse, o_part,
-                           l_part, nullptr, s) != cudaSuccess)
+                           l_part, nullptr, s, false) != cudaSuccess)
     return DSA_ERR_CUDA;
-  if (S > 1 && launch_combine(o_part, l_part, Q, S, out, lse, s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (S > 1 && launch_combine(o_part, l_part, Q, S, out, lse, s, true) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return DSA_OK;
 }

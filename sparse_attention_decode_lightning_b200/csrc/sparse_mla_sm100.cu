@@ -137,6 +137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
+  pdl_trigger();
   const int unit = blockIdx.x >> 1;
   const int q = unit / a.S, split = unit % a.S;
   const int b = seq_of_query(a.q_offsets, a.B, q);
@@ -175,6 +176,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     mbar_arrive_expect_tx(q_ready, QROPE_BYTES);
     tma_load_2d(qrope, &tmap_q, 8 * 64, q * DSA_HEADS, q_ready);
   }
+  if (warp >= 2 && warp < 6) {
+    // softmax warpgroup 0: this CTA's 256 latent query dims of head h -> tensor
+    // memory (bf16 pairs).  The queries are inputs of the whole step, so this
+    // runs before pdl_wait() and overlaps the end of the selector.
+    const int quarter = warp & 3;
+    const int h = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float w[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(src + c * 8 + i);
+        w[4 * i + 0] = __uint_as_float(v.x);
+        w[4 * i + 1] = __uint_as_float(v.y);
+        w[4 * i + 2] = __uint_as_float(v.z);
+        w[4 * i + 3] = __uint_as_float(v.w);
+      }
+      tmem_st32(lane_base + Q_COL + c * 32, w);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
+  }
+  // the selected indices (and the error word) come from the kernel before
+  pdl_wait();
   // pool row of every entry of this split, resolved once by all threads with
   // many independent loads in flight (-1 = padding or out of range)
   {
@@ -300,28 +330,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
     // partial scores are exchanged by push: each CTA stores its partial into
     // the peer's shared memory with st.async and reads the peer's from its own
-    if (g == 0) {
-      // this CTA's 256 latent query dims of head h -> tensor memory (bf16 pairs)
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float w[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = __ldg(src + c * 8 + i);
-          w[4 * i + 0] = __uint_as_float(v.x);
-          w[4 * i + 1] = __uint_as_float(v.y);
-          w[4 * i + 2] = __uint_as_float(v.z);
-          w[4 * i + 3] = __uint_as_float(v.w);
-        }
-        tmem_st32(lane_base + Q_COL + c * 32, w);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_ready);
-    }
     float m_use = -INFINITY, l = 0.f;                // l: this warpgroup's rows only
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
@@ -506,7 +514,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int topk, float scale, int S,
                                  float* out, float* lse, float* o_part, float* l_part,
-                                 uint32_t* err, cudaStream_t st) {
+                                 uint32_t* err, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
   CUtensorMap tq;
   if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, DSA_DIM,
@@ -530,8 +538,17 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
     return cudaErrorInvalidValue;
   MlaTcArgs a{q, pool, page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
-  sparse_mla_tc_kernel<<<2 * Q * S, THREADS, SMEM_BYTES, st>>>(tq, to, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * Q * S), 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  unsigned int na = 0;
+  add_pdl_attr(attr, &na, pdl);
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel, tq, to, a);
 }
 
 }  // namespace dsa

@@ -180,8 +180,12 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = static_cast<int>(gridDim.x);    // cluster = one grid row
   const uint32_t rank = cluster_ctarank();
+  pdl_trigger();
+  // q_offsets and q_vis are inputs of the whole step; the scores, the
+  // outputs and the error word belong to the kernels before this one
   const int q = row_query(a, blockIdx.y);
   if (q < 0) return;                            // the whole cluster leaves
+  pdl_wait();
   const int vis = clamped_vis(a, q);
   const int topk = a.topk;
   const float* row = a.scores + static_cast<size_t>(q) * a.ld;
@@ -522,7 +526,7 @@ int topk_cluster_size(int rows, int max_len) {
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
                         const int32_t* q_vis, int B, int Q, int max_len, int topk,
                         int first_only, int32_t* out_idx, float* out_scores, uint32_t* err,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool pdl) {
   const int rows = first_only ? B : Q;
   if (rows <= 0) return cudaSuccess;
   if (rows > 65535 || topk > DSA_MAX_TOPK) return cudaErrorInvalidValue;
@@ -546,13 +550,15 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes(scap);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  unsigned int na = 1;
+  add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a);
 }
 
