@@ -65,7 +65,7 @@ constexpr int OFF_X = OFF_ST + NST * STAGE_BYTES;
 constexpr int OFF_MX = OFF_X + 2 * X_BYTES;    // [2 tiles][2 warpgroups][128 heads] partial maxima
 constexpr int OFF_CRD = OFF_MX + 2 * 2 * DSA_HEADS * 4;
 constexpr int OFF_BAR = OFF_CRD + DSA_MAX_TOPK * 4;
-constexpr int NBAR = 2 * NST + 4 * 2 + 3;
+constexpr int NBAR = 2 * NST + 4 * 2 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "sparse MLA shared memory exceeds the sm_100 limit");
@@ -130,8 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* p_full = s_full + 2;         // [2] P of a tile is in its slot
   uint64_t* slot_free = p_full + 2;      // [2] PV of the slot's tile is done
   uint64_t* x_full = slot_free + 2;      // [2] the peer's partial scores arrived
-  uint64_t* o_done = x_full + 2;         // every PV
-  uint64_t* o_final = o_done + 1;        // last PV
+  uint64_t* o_final = x_full + 2;        // last PV
   uint64_t* q_ready = o_final + 1;       // query slice in TMEM / shared memory
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
@@ -160,7 +159,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&slot_free[i], 1);
       mbar_init(&x_full[i], 1);   // armed with the tile's bytes; the peer's st.async complete them
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(q_ready, 5);             // 4 query-loading warps + thread 0 with the RoPE bytes
     mbar_fence_init();
@@ -175,33 +173,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmap_q);
     mbar_arrive_expect_tx(q_ready, QROPE_BYTES);
     tma_load_2d(qrope, &tmap_q, 8 * 64, q * DSA_HEADS, q_ready);
-  }
-  if (warp >= 2 && warp < 6) {
-    // softmax warpgroup 0: this CTA's 256 latent query dims of head h -> tensor
-    // memory (bf16 pairs).  The queries are inputs of the whole step, so this
-    // runs before pdl_wait() and overlaps the end of the selector.
-    const int quarter = warp & 3;
-    const int h = quarter * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint4* src = reinterpret_cast<const uint4*>(
-        a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float w[32];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 v = __ldg(src + c * 8 + i);
-        w[4 * i + 0] = __uint_as_float(v.x);
-        w[4 * i + 1] = __uint_as_float(v.y);
-        w[4 * i + 2] = __uint_as_float(v.z);
-        w[4 * i + 3] = __uint_as_float(v.w);
-      }
-      tmem_st32(lane_base + Q_COL + c * 32, w);
-    }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(q_ready);
   }
   // the selected indices (and the error word) come from the kernel before
   pdl_wait();
@@ -313,7 +284,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           mma_commit(&slot_free[pbuf]);
           mma_commit(&empty[s]);
-          mma_commit(o_done);
           if (t == ntiles - 1) mma_commit(o_final);
         }
       }
@@ -330,6 +300,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
     // partial scores are exchanged by push: each CTA stores its partial into
     // the peer's shared memory with st.async and reads the peer's from its own
+    if (g == 0) {
+      // this CTA's 256 latent query dims of head h -> tensor memory (bf16 pairs)
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(src + c * 8 + i);
+          w[4 * i + 0] = __uint_as_float(v.x);
+          w[4 * i + 1] = __uint_as_float(v.y);
+          w[4 * i + 2] = __uint_as_float(v.z);
+          w[4 * i + 3] = __uint_as_float(v.w);
+        }
+        tmem_st32(lane_base + Q_COL + c * 32, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
     float m_use = -INFINITY, l = 0.f;                // l: this warpgroup's rows only
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
@@ -417,11 +409,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         ps3 += z[r + 3];
       }
       l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
-      // PV(t-1) done (needed before O may be rescaled).  Waited on every tile
-      // before P(t) is published, so o_done has completed t-1 or t phases
-      // here and the parity test is exact.
-      if (t >= 1 && !(ok = warp_wait(o_done, (t - 1) & 1, a.err))) break;
+      // O is rescaled (rarely: only when the running max moves) after PV(t-1)
+      // has finished, which completes phase (t-1)/2 of slot_free[(t-1)&1];
+      // PV(t+1) needs P(t+1), so that barrier cannot have moved further.
+      // Without a rescale P(t) is published at once, and PV(t-1) runs
+      // behind the scores MMA of tile t+1 without holding up the softmax.
       if (g == 0 && __any_sync(0xffffffffu, resc)) {
+        if (t >= 1 && !(ok = warp_wait(&slot_free[(t - 1) & 1], ((t - 1) >> 1) & 1, a.err))) break;
         tc_fence_after();
         for (int c = 0; c < 256 / 32; ++c) {
           float o[32];
