@@ -1,49 +1,66 @@
 // Split-K merge of partial attentions by log-sum-exp:
 //   LSE = ln sum_c exp(LSE_c),  O = sum_c exp(LSE_c - LSE) O_c,
 // parts with LSE_c = -inf (no selected token) get weight 0; if every part is
-// empty O = 0 and LSE = -inf.  One CTA of 128 threads per (query, head): the
-// 512 outputs are one float4 per thread, the split weights are recomputed by
-// every thread from the S partial LSEs (S <= 32, L1-resident).
+// empty O = 0 and LSE = -inf.  One CTA of 256 threads per (query, 8 heads): a
+// warp per head, 16 outputs per thread; the split weights are recomputed by
+// every thread from the S partial LSEs (L1-resident).  One CTA per head (4096
+// CTAs of 128 threads for 32 queries) spent its time in CTA scheduling.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dsa {
 namespace {
 
-__global__ void __launch_bounds__(128) lse_combine_kernel(const float* __restrict__ o_part,
-                                                          const float* __restrict__ l_part,
-                                                          int S, float* __restrict__ out,
-                                                          float* __restrict__ lse) {
+constexpr int HEADS_PER_CTA = 8;               // 8 heads x 512 outputs, 16 per thread
+constexpr int CTHREADS = HEADS_PER_CTA * DSA_DIM_V / 16;
+
+__global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __restrict__ o_part,
+                                                               const float* __restrict__ l_part,
+                                                               int S, float* __restrict__ out,
+                                                               float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();                                   // the partials come from the previous kernel
-  const int qh = blockIdx.x;                    // q * 128 + h
-  const int q = qh / DSA_HEADS, h = qh % DSA_HEADS;
+  // CTA: query q, heads [h0, h0 + 8); thread: head h0 + tid / 32, outputs
+  // [16 * (tid % 32), +16) as four float4 spread 128 floats apart
+  const int q = blockIdx.x / (DSA_HEADS / HEADS_PER_CTA);
+  const int h = (blockIdx.x % (DSA_HEADS / HEADS_PER_CTA)) * HEADS_PER_CTA + (threadIdx.x >> 5);
+  const int c4 = threadIdx.x & 31;              // float4 column within each 128-float quarter
+  const size_t qh = static_cast<size_t>(q) * DSA_HEADS + h;
   const float* lp = l_part + static_cast<size_t>(q) * S * DSA_HEADS + h;
   float m = -INFINITY;
   for (int c = 0; c < S; ++c) m = fmaxf(m, lp[static_cast<size_t>(c) * DSA_HEADS]);
-  float4* o = reinterpret_cast<float4*>(out + static_cast<size_t>(qh) * DSA_DIM_V) + threadIdx.x;
+  float4* o = reinterpret_cast<float4*>(out + qh * DSA_DIM_V) + c4;
   if (m == -INFINITY) {
-    *o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (threadIdx.x == 0) lse[qh] = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[32 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c4 == 0) lse[qh] = -INFINITY;
     return;
   }
   float tot = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int c = 0; c < S; ++c) {
     const float lc = lp[static_cast<size_t>(c) * DSA_HEADS];
     if (lc == -INFINITY) continue;
     const float wc = expf(lc - m);
     tot += wc;
-    const float4 v = reinterpret_cast<const float4*>(
-        o_part + ((static_cast<size_t>(q) * S + c) * DSA_HEADS + h) * DSA_DIM_V)[threadIdx.x];
-    acc.x = fmaf(wc, v.x, acc.x);
-    acc.y = fmaf(wc, v.y, acc.y);
-    acc.z = fmaf(wc, v.z, acc.z);
-    acc.w = fmaf(wc, v.w, acc.w);
+    const float4* v = reinterpret_cast<const float4*>(
+                          o_part + ((static_cast<size_t>(q) * S + c) * DSA_HEADS + h) * DSA_DIM_V) + c4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 x = v[32 * k];
+      acc[k].x = fmaf(wc, x.x, acc[k].x);
+      acc[k].y = fmaf(wc, x.y, acc[k].y);
+      acc[k].z = fmaf(wc, x.z, acc[k].z);
+      acc[k].w = fmaf(wc, x.w, acc[k].w);
+    }
   }
   const float inv = 1.f / tot;
-  *o = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (threadIdx.x == 0) lse[qh] = m + logf(tot);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    o[32 * k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+  if (c4 == 0) lse[qh] = m + logf(tot);
 }
 
 }  // namespace
@@ -52,8 +69,8 @@ cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int 
                            float* lse, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(Q) * DSA_HEADS, 1, 1);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(Q) * (DSA_HEADS / HEADS_PER_CTA), 1, 1);
+  cfg.blockDim = dim3(CTHREADS, 1, 1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   unsigned int na = 0;
