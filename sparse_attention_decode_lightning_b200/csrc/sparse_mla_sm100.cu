@@ -536,7 +536,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tma_store_2d(&tmap_o, box0 + c * OBOX_BYTES, static_cast<int>(rank) * 256 + 128 * g + 32 * c,
                      orow0);
       bulk_commit_group();
-      bulk_wait_all();
+      bulk_wait_all_read();   // the shared-memory boxes may be released; the grid's end publishes O
     }
     if (rank == 0 && g == 0) *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
     (void)gt;
