@@ -49,7 +49,7 @@ constexpr int OFF_DATA = (OFF_MISC + 16 + 1023) / 1024 * 1024;   // per-pipeline
 constexpr int SMEM_BYTES = 230400;                     // dynamic shared memory requested
 constexpr int DATA_BYTES = SMEM_BYTES - 1024 - OFF_DATA;
 static_assert(SMEM_BYTES <= 232448, "indexer shared memory exceeds the sm_100 limit");
-static_assert(DATA_BYTES >= PIPES * (2 * KEY_TILE + DSA_MAX_Q_PER_SEQ * Q_TILE),
+static_assert(DATA_BYTES >= PIPES * (2 * KEY_TILE + (DSA_MAX_Q_PER_SEQ + 1) / 2 * 2 * Q_TILE),
               "two stages and a full query buffer must fit per pipeline");
 
 struct IdxArgs {
@@ -161,9 +161,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   block_exclusive_scan(prefix, B, scan_tmp);
   const int maxq = *s_maxq;
-  // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of maxq tiles]
+  // Sequences with several queries (MTP verify) take their queries two at a
+  // time: one MMA with N = 128 (two 64-head query tiles side by side) into one
+  // of 2 accumulator slots of 128 columns, instead of one N = 64 MMA per query
+  // into 4 slots of 64.  Halves the MMAs and commits per tile.
+  const int G = maxq >= 2 ? 2 : 1;
+  const int nslots = SLOTS / G;
+  const uint32_t slot_cols = ACC_COLS * G;
+  const int qtiles = (maxq + G - 1) / G * G;      // the last pair may read one tile past nq
+  // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of qtiles tiles]
   const int pipe_bytes = (DATA_BYTES / PIPES) / 1024 * 1024;
-  const int stages = min(MAX_STAGES, (pipe_bytes - maxq * Q_TILE) / KEY_TILE);
+  const int stages = min(MAX_STAGES, (pipe_bytes - qtiles * Q_TILE) / KEY_TILE);
 
   const int pipe = warp / WARPS_PER_PIPE;          // 0 / 1
   const int pw = warp % WARPS_PER_PIPE;            // role within the pipeline
@@ -251,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (pw == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && t_begin < t_end) {
-      constexpr uint32_t idesc = umma_idesc(0 /*E4M3*/, KT, ACC_COLS);
+      const uint32_t idesc = umma_idesc(0 /*E4M3*/, KT, static_cast<int>(slot_cols));
       int b = b_first, cur_b = -1, nq = 0;
       uint32_t qphase = 0, n = 0, k = 0;
       bool ok = true;
@@ -268,14 +276,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(&full[s], (k / stages) & 1, a.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(keys + s * KEY_TILE);
-        for (int j = 0; j < nq; ++j, ++n) {
-          const uint32_t slot = n % SLOTS;
-          if (!mbar_wait(&acc_empty[slot], ((n / SLOTS) & 1) ^ 1, a.err)) { ok = false; break; }
+        for (int j0 = 0; j0 < nq; j0 += G, ++n) {
+          const uint32_t slot = n % nslots;
+          if (!mbar_wait(&acc_empty[slot], ((n / nslots) & 1) ^ 1, a.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t b_base = smem_u32(qbuf + j * Q_TILE);
+          // G consecutive 64-row query tiles form one 64G-row B operand (the
+          // 128-byte swizzle atoms continue every 1024 bytes across tiles)
+          const uint32_t b_base = smem_u32(qbuf + j0 * Q_TILE);
 #pragma unroll
           for (int kk = 0; kk < DSA_IDX_DIM / 32; ++kk) {
-            mma_f8f6f4(tmem + slot * ACC_COLS, umma_desc_sw128(a_base + kk * 32, 1024, 16),
+            mma_f8f6f4(tmem + slot * slot_cols, umma_desc_sw128(a_base + kk * 32, 1024, 16),
                        umma_desc_sw128(b_base + kk * 32, 1024, 16), idesc, kk > 0 ? 1u : 0u);
           }
           mma_commit(&acc_full[slot]);
@@ -305,20 +315,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           cur_b = b;
         }
         const int t = i - prefix[b];
-        for (int j = 0; j < nq; ++j, ++n) {
-          const uint32_t slot = n % SLOTS;
-          if (!mbar_wait(&acc_full[slot], (n / SLOTS) & 1, a.err)) { ok = false; break; }
-          tc_fence_after();
+        for (int j = 0; j < nq; ++j) {
+          const uint32_t slot = n % nslots;
+          const int jj = j % G;                    // query within the slot's pair
+          if (jj == 0) {
+            if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
+            tc_fence_after();
+          }
           float v[ACC_COLS];
-          const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * ACC_COLS;
+          const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols +
+                                 static_cast<uint32_t>(jj * ACC_COLS);
           tmem_ld16(taddr + 0, v + 0);
           tmem_ld16(taddr + 16, v + 16);
           tmem_ld16(taddr + 32, v + 32);
           tmem_ld16(taddr + 48, v + 48);
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[slot]);
+          if (jj == G - 1 || j == nq - 1) {        // last query of the slot: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[slot]);
+            ++n;
+          }
           const int q = q0 + j;
           bool bad = false;
           const int vis = query_vis(a, q, len, &bad);
