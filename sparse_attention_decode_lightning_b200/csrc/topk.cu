@@ -48,6 +48,7 @@ constexpr int NCHUNK = 10;
 constexpr int SLICE_CAP = NCHUNK * CHUNK;     // 40960 scores a CTA keeps in shared memory
 constexpr int CAND_CAP = 4096;                // bin-t positions rank 0 gathers
 constexpr int MAX_CLUSTER = 8;                // portable cluster size
+constexpr int MAX_CLUSTER_NP = 16;            // non-portable size for a few long rows
 constexpr int MIN_SLICE = 2048;               // rows are not cut finer than this
 static_assert(BINS == 4 * THREADS, "bins are merged THREADS at a time, scanned 4 per thread");
 
@@ -511,14 +512,45 @@ __global__ void expand_idx_kernel(const int32_t* q_offsets, int Q, int topk, int
   }
 }
 
-// CTAs per query row: enough clusters to cover the SMs once, at most 8 (the
-// portable cluster size) and no slice shorter than MIN_SLICE
-int topk_cluster_size(int rows, int max_len) {
+// CTAs per query row: enough clusters to cover the SMs once, at most `cap`
+// and no slice shorter than MIN_SLICE
+int topk_cluster_size(int rows, int max_len, int cap) {
   int C = device_sm_count() / (rows > 0 ? rows : 1);
-  C = C < 1 ? 1 : (C > MAX_CLUSTER ? MAX_CLUSTER : C);
+  C = C < 1 ? 1 : (C > cap ? cap : C);
   const int by_len = max_len / MIN_SLICE;
   if (C > by_len) C = by_len < 1 ? 1 : by_len;
   return C;
+}
+
+// Largest cluster size the device schedules for this kernel: 16 (opt-in,
+// non-portable) when at least one such cluster fits, else 8.  Queried once
+// per device; a handful of long rows (1M context) then gets twice the CTAs.
+int max_cluster_for_device(size_t smem) {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAX_CLUSTER;
+  if (cached[dev]) return cached[dev];
+  int cap = MAX_CLUSTER;
+  if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(MAX_CLUSTER_NP, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = MAX_CLUSTER_NP;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) == cudaSuccess && n > 0)
+      cap = MAX_CLUSTER_NP;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error behind
+  cached[dev] = cap;
+  return cap;
 }
 
 }  // namespace
@@ -540,7 +572,8 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int C = topk_cluster_size(rows, max_len);
+  const int C = topk_cluster_size(rows, max_len,
+                                  max_cluster_for_device(smem_bytes(SLICE_CAP)));
   const int slice = (((max_len + C - 1) / C) + 3) & ~3;
   const int scap = slice < SLICE_CAP ? slice : SLICE_CAP;
   TopkArgs a{scores, ld, q_offsets, q_vis, B, Q, max_len, topk, first_only,
