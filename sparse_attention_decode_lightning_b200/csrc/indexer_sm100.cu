@@ -42,10 +42,14 @@ constexpr int Q_TILE = DSA_IDX_HEADS * DSA_IDX_DIM;    // 8192 B
 constexpr int MAX_STAGES = 6;                          // per pipeline
 constexpr int OFF_PREFIX = 0;
 constexpr int OFF_SCAN = OFF_PREFIX + ((DSA_MAX_BATCH + 1) * 4 + 15) / 16 * 16;
-constexpr int NBAR_PIPE = 2 * MAX_STAGES + 2 * SLOTS + 3;
+constexpr int NBAR_PIPE = 2 * MAX_STAGES + 2 * SLOTS + 5;
 constexpr int OFF_BAR = OFF_SCAN + 64 * 4;
 constexpr int OFF_MISC = OFF_BAR + PIPES * NBAR_PIPE * 8;
-constexpr int OFF_DATA = (OFF_MISC + 16 + 1023) / 1024 * 1024;   // per-pipeline rings + query buffers
+// per pipeline: the current sequence's head weights [queries][64] fp32 and
+// visible lengths, shared by its four epilogue warps
+constexpr int WS_PIPE = DSA_MAX_Q_PER_SEQ * DSA_IDX_HEADS * 4 + DSA_MAX_Q_PER_SEQ * 4;
+constexpr int OFF_WS = (OFF_MISC + 16 + 15) / 16 * 16;
+constexpr int OFF_DATA = (OFF_WS + PIPES * WS_PIPE + 1023) / 1024 * 1024;   // rings + query buffers
 constexpr int SMEM_BYTES = 230400;                     // dynamic shared memory requested
 constexpr int DATA_BYTES = SMEM_BYTES - 1024 - OFF_DATA;
 static_assert(SMEM_BYTES <= 232448, "indexer shared memory exceeds the sm_100 limit");
@@ -185,6 +189,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* q_full = acc_empty + SLOTS;
   uint64_t* q_empty = q_full + 1;
   uint64_t* mma_done = q_full + 2;
+  uint64_t* w_free = q_full + 3;                   // epilogue warps left the previous sequence
+  uint64_t* w_full = q_full + 4;                   // the sequence's weights are in w_s
+  float* w_s = reinterpret_cast<float*>(smem + OFF_WS + pipe * WS_PIPE);
+  int* vis_s = reinterpret_cast<int*>(w_s + DSA_MAX_Q_PER_SEQ * DSA_IDX_HEADS);
 
   if (tid < PIPES) {
     uint64_t* pb = reinterpret_cast<uint64_t*>(smem + OFF_BAR) + tid * NBAR_PIPE;
@@ -196,6 +204,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 0], 1);   // q_full
     mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 1], 1);   // q_empty
     mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 2], 1);   // mma_done
+    mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 3], 4);   // w_free: the 4 epilogue warps
+    mbar_init(&pb[2 * MAX_STAGES + 2 * SLOTS + 4], 4);   // w_full
     mbar_fence_init();
     if (tid == 0) {
       tma_prefetch_desc(&tmap_k);
@@ -303,15 +313,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int quarter = warp & 3;            // TMEM lanes this warp may read
       const int row = quarter * 32 + lane;     // key row of the tile
       int b = b_first, cur_b = -1, nq = 0, q0 = 0;
-      int64_t len = 0;
-      uint32_t n = 0;
+      uint32_t n = 0, wph = 0;
       bool ok = true;
       for (int i = t_begin; i < t_end && ok; ++i) {
         while (prefix[b + 1] <= i) ++b;
         if (b != cur_b) {
+          // new sequence: once all four epilogue warps are past the previous
+          // one, they copy its weights and visible lengths into w_s / vis_s
+          // (bounded mbarrier waits, not bar.sync, so a timed-out warp cannot
+          // leave the others waiting for ever)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(w_free);
+          if (!(ok = mbar_wait(w_free, wph, a.err))) break;
           nq = seq_queries(a, b);
           q0 = a.q_offsets[b];
-          len = a.seq_offsets[b + 1] - a.seq_offsets[b];
+          const int64_t len = a.seq_offsets[b + 1] - a.seq_offsets[b];
+          const int e = pw - 2;                  // 0..3
+          for (int x = e * 32 + lane; x < nq * DSA_IDX_HEADS; x += 128)
+            w_s[x] = __ldg(a.w + static_cast<size_t>(q0) * DSA_IDX_HEADS + x);
+          if (e == 0 && lane < nq) {
+            bool bad = false;
+            vis_s[lane] = query_vis(a, q0 + lane, len, &bad);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(w_full);
+          if (!(ok = mbar_wait(w_full, wph, a.err))) break;
+          wph ^= 1;
           cur_b = b;
         }
         const int t = i - prefix[b];
@@ -337,15 +364,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             ++n;
           }
           const int q = q0 + j;
-          bool bad = false;
-          const int vis = query_vis(a, q, len, &bad);
+          const int vis = vis_s[j];
           const int s = t * KT + row;
           if (s < vis) {
-            const float4* wp = reinterpret_cast<const float4*>(a.w + static_cast<size_t>(q) * DSA_IDX_HEADS);
+            const float4* wp = reinterpret_cast<const float4*>(w_s + j * DSA_IDX_HEADS);
             float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
             for (int h4 = 0; h4 < DSA_IDX_HEADS / 4; ++h4) {
-              const float4 ww = __ldg(wp + h4);
+              const float4 ww = wp[h4];
               s0 = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
               s1 = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
               s2 = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
