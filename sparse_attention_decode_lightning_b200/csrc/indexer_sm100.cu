@@ -342,6 +342,52 @@ __global__ void __launch_bounds__(THREADS, 1)
           cur_b = b;
         }
         const int t = i - prefix[b];
+        // query pairs: both queries' 128 columns are read with a single wait
+        // (the wait covers every outstanding TMEM load, so reading the second
+        // query later would cost a second full load latency)
+        if (G == 2) {
+          for (int j0 = 0; j0 < nq; j0 += 2, ++n) {
+            const uint32_t slot = n % nslots;
+            const bool two = j0 + 1 < nq;
+            if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
+            tc_fence_after();
+            float v[2 * ACC_COLS];
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols;
+            tmem_ld32(taddr + 0, v + 0);
+            tmem_ld32(taddr + 32, v + 32);
+            tmem_ld32(taddr + 64, v + 64);      // past nq for an odd last query: not used
+            tmem_ld32(taddr + 96, v + 96);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[slot]);
+            const int s = t * KT + row;
+            float r0 = 0.f, r1 = 0.f;
+            {
+              const float4* w0 = reinterpret_cast<const float4*>(w_s + j0 * DSA_IDX_HEADS);
+              const float4* w1 = reinterpret_cast<const float4*>(w_s + (two ? j0 + 1 : j0) * DSA_IDX_HEADS);
+              float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+              for (int h4 = 0; h4 < DSA_IDX_HEADS / 4; ++h4) {
+                const float4 x = w0[h4];
+                const float4 y = w1[h4];
+                a0 = fmaf(x.x, fmaxf(v[4 * h4 + 0], 0.f), a0);
+                a1 = fmaf(x.y, fmaxf(v[4 * h4 + 1], 0.f), a1);
+                a0 = fmaf(x.z, fmaxf(v[4 * h4 + 2], 0.f), a0);
+                a1 = fmaf(x.w, fmaxf(v[4 * h4 + 3], 0.f), a1);
+                b0 = fmaf(y.x, fmaxf(v[64 + 4 * h4 + 0], 0.f), b0);
+                b1 = fmaf(y.y, fmaxf(v[64 + 4 * h4 + 1], 0.f), b1);
+                b0 = fmaf(y.z, fmaxf(v[64 + 4 * h4 + 2], 0.f), b0);
+                b1 = fmaf(y.w, fmaxf(v[64 + 4 * h4 + 3], 0.f), b1);
+              }
+              r0 = a0 + a1;
+              r1 = b0 + b1;
+            }
+            if (s < vis_s[j0]) a.scores[static_cast<size_t>(q0 + j0) * a.ld + s] = r0;
+            if (two && s < vis_s[j0 + 1]) a.scores[static_cast<size_t>(q0 + j0 + 1) * a.ld + s] = r1;
+          }
+          continue;
+        }
         for (int j = 0; j < nq; ++j) {
           const uint32_t slot = n % nslots;
           const int jj = j % G;                    // query within the slot's pair
