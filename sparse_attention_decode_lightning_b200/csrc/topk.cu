@@ -572,8 +572,11 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int C = topk_cluster_size(rows, max_len,
-                                  max_cluster_for_device(smem_bytes(SLICE_CAP)));
+  // beyond the portable 8 CTAs only when 8 would leave slices longer than the
+  // on-chip copy (merging 16 histograms costs more than it saves otherwise)
+  int C = topk_cluster_size(rows, max_len, MAX_CLUSTER);
+  if (C == MAX_CLUSTER && (max_len + C - 1) / C > SLICE_CAP)
+    C = topk_cluster_size(rows, max_len, max_cluster_for_device(smem_bytes(SLICE_CAP)));
   const int slice = (((max_len + C - 1) / C) + 3) & ~3;
   const int scap = slice < SLICE_CAP ? slice : SLICE_CAP;
   TopkArgs a{scores, ld, q_offsets, q_vis, B, Q, max_len, topk, first_only,
