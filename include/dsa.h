@@ -161,6 +161,11 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
  *   out        fp32 [Q,128,512]      lse fp32 [Q,128] (natural log)
  * Entries with idx >= q_vis[q], a page id outside [0,num_pages) or a page
  * slot beyond max_pages are skipped and flagged (DSA_ERR_DEVICE_BOUNDS).
+ * Precision: bf16 products accumulate in fp32 on the tensor cores.  Each
+ * score is the sum of two partial dot products (latent dims split between a
+ * pair of SMs); one partial crosses to the other SM rounded to a 24-bit
+ * float (15 mantissa bits), which moves O by well under 1e-3 of its RMS.  P
+ * enters the value product as a bf16 high + low pair (~16 significant bits).
  * ws: at least dsa_workspace_bytes(Q, 1, topk, num_splits) bytes.
  */
 dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
@@ -219,6 +224,12 @@ dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, 
  *   idx_out          int32 [ceil(n_layers/G), Q, topk]: the index rows used.
  *   out_layers / lse_layers: per layer fp32 [Q,128,512] / [Q,128].
  * Other arguments as in dsa_indexer_topk and dsa_sparse_mla_decode.
+ * The kernels of one call (and of dsa_indexer_topk) are chained with
+ * programmatic dependent launch: a kernel may start its set-up while the
+ * previous kernel of the same call drains, and waits for it before reading
+ * what it wrote.  The first kernel of a call starts only after all earlier
+ * work on the stream, as usual.  The call allocates nothing and does not
+ * synchronise, so it can be captured into a CUDA graph.
  */
 dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                            const uint8_t* const* q_idx_layers, const float* const* w_layers,

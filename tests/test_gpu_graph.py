@@ -1,0 +1,91 @@
+"""dsa_decode_step captured into a CUDA graph and replayed.
+
+The step allocates nothing and never synchronises, and its kernels are
+chained with programmatic dependent launch; a captured step must give the
+same indices and attention as the same call run eagerly, and a replay must
+read the inputs as they are at replay time (not at capture time).  Index rows
+come out in no particular order (slots are handed out by atomics), so rows are
+compared as sets and the attention, whose tiles and split parts follow the
+row order, to fp32 reassociation."""
+import pytest
+import torch
+
+import sparse_attention_decode_lightning_b200 as dsa
+from synth import get_workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _args(inp, outs, lses, idx, ws, stream):
+    n, G = inp.n_layers, inp.index_share
+    qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
+    wl = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
+    kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
+    return dict(q_idx_layers=qi, w_layers=wl, k_idx_layers=kl, qs=[L["q"] for L in inp.layers],
+                pools=[L["pool"] for L in inp.layers], outs=outs, lses=lses, idx=idx, ws=ws,
+                stream=stream)
+
+
+def _step(inp, a):
+    n = inp.n_layers
+    dsa.dsa_decode_step(a["q_idx_layers"], a["w_layers"], a["k_idx_layers"], inp.seq_offsets,
+                        inp.q_offsets, inp.q_vis, inp.B, inp.max_len, inp.topk, a["qs"], a["pools"],
+                        [inp.page_table] * n, inp.scale, a["outs"], a["lses"], a["idx"], a["ws"],
+                        index_share=inp.index_share, mtp_index_share=inp.mtp_index_share,
+                        num_splits=inp.num_splits, stream=a["stream"])
+
+
+def _same(a_outs, a_lses, a_idx, b_outs, b_lses, b_idx):
+    assert torch.equal(torch.sort(a_idx, dim=-1).values, torch.sort(b_idx, dim=-1).values)
+    for o1, l1, o2, l2 in zip(a_outs, a_lses, b_outs, b_lses):
+        r = o1.square().mean().sqrt()
+        # same rows, another order: the tiles, running maxima and split parts
+        # regroup the fp32 sums (observed ~5e-5 of rms; parity's bar is 1e-2)
+        assert (o1 - o2).abs().max() <= 1e-3 * r
+        assert (l1 - l2).abs().max() <= 1e-4
+
+
+@pytest.mark.parametrize("name,over", [("decode_b32_ctx128k", dict(B=4, L=9000)),
+                                       ("indexshare4_b64_ctx16k_128k", dict(B=3, L_range=(1500, 7000)))])
+def test_captured_step_matches_eager_and_reads_inputs_at_replay(name, over):
+    inp = make_inputs(get_workload(name, **over), seed=3, device=DEV)
+    Q, n = inp.Q, inp.n_layers
+    ng = (n + inp.index_share - 1) // inp.index_share
+
+    def buffers():
+        return ([torch.empty(Q, 128, 512, device=DEV) for _ in range(n)],
+                [torch.empty(Q, 128, device=DEV) for _ in range(n)],
+                torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=DEV))
+
+    ws = dsa.workspace(Q, inp.max_len, inp.topk, inp.num_splits, device=DEV)
+    side = torch.cuda.Stream()
+    # eager reference (also the first call on the device: attributes, caches)
+    e_outs, e_lses, e_idx = buffers()
+    _step(inp, _args(inp, e_outs, e_lses, e_idx, ws, side))
+    torch.cuda.synchronize()
+    dsa.dsa_check_error(ws)
+
+    g_outs, g_lses, g_idx = buffers()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        _step(inp, _args(inp, g_outs, g_lses, g_idx, ws, side))
+    # capture records work without running it
+    graph.replay()
+    torch.cuda.synchronize()
+    dsa.dsa_check_error(ws)
+    _same(g_outs, g_lses, g_idx, e_outs, e_lses, e_idx)
+
+    # new query values in place: the replay must see them
+    for L in inp.layers:
+        L["q"].copy_(torch.flip(L["q"], dims=[0]))
+    for grp in inp.indexer:
+        grp["w"].mul_(-1.0)
+    e2_outs, e2_lses, e2_idx = buffers()
+    _step(inp, _args(inp, e2_outs, e2_lses, e2_idx, ws, side))
+    torch.cuda.synchronize()       # the eager step and the replay share the workspace
+    graph.replay()
+    torch.cuda.synchronize()
+    dsa.dsa_check_error(ws)
+    assert not torch.equal(torch.sort(e2_idx, dim=-1).values, torch.sort(e_idx, dim=-1).values)
+    _same(g_outs, g_lses, g_idx, e2_outs, e2_lses, e2_idx)
