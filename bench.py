@@ -416,11 +416,7 @@ def run_ours(args, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_mean_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 indexer, bf16 attention, f32 accumulate", "data": "synthetic",
-        "config": {"workload": wl.name, "B": inp.B, "T": inp.T, "L": wl.L,
-                   "L_range": list(wl.L_range) if wl.L_range else None, "layers": n,
-                   "index_share": G, "mtp_index_share": inp.mtp_index_share, "topk": inp.topk,
-                   "num_splits": S, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (FP8 keys) and a 256 MiB L2 flush before every step"},
+        "config": workload_config(wl, inp.B, S, world),
         "roofline": {"bound": "hbm", "kernel": "indexer_kernel", "achieved": achieved, "peak": hbm,
                      "peak_source": hbm_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": (measured_traffic("indexer_sm100.cu", "indexer_kernel_decode_b8_ctx128k.md")
@@ -439,6 +435,16 @@ def run_ours(args, rank, world, local_rank):
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
     return res
+
+
+def workload_config(wl, B, S, world):
+    """The `config` object of both arms' JSON lines: the workload by name and sizes."""
+    return {"workload": wl.name, "B": B, "T": wl.T, "L": wl.L,
+            "L_range": list(wl.L_range) if wl.L_range else None, "layers": wl.n_layers,
+            "index_share": wl.index_share, "mtp_index_share": wl.mtp_index_share,
+            "topk": wl.topk, "num_splits": S,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (FP8 keys) and a 256 MiB L2 flush before every step"}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -469,7 +475,7 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": wl.name, "sample": "one sequence of the workload per step"},
+        "config": workload_config(wl, wl.B, wl.num_splits, 1),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{args.steps} steps x 1 sequence ({inp.Q} query tokens, all layers)"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
