@@ -9,20 +9,23 @@
 // and turns the scores into order-preserving u32 keys in place.
 //
 // Exact radix select on the composite key of position s
-//     V(s) = (u(s) << pb) | s,   u(s) = kmax - key(I[s]),   pb = bits(vis - 1)
-// with kmax the largest key of the row.  V is distinct per position and a
-// smaller V is a better position (higher score, then lower position), so the
-// topk smallest V are exactly the top-k with the lower-position tie rule.
-// Measuring u from the row's own maximum makes the first 12-bit digit span
-// the row's score range [kmin, kmax] only: the 4096 first-level bins are
-// narrow and the bin holding the k-th score has few positions.
+//     V(s) = (u(s) << pb) | s,   u(s) = ~key(I[s]),   pb = bits(vis - 1)
+// (u measures the key down from the largest possible key).  V is distinct
+// per position and a smaller V is a better position (higher score, then
+// lower position), so the topk smallest V are exactly the top-k with the
+// lower-position tie rule.  The first 12-bit digit of V is the sign, exponent
+// and top three mantissa bits of the score: relative bins of 1/8 of an
+// octave, the same in every CTA without first agreeing on the row's range,
+// so the first histogram is built while the copies land.  (Measuring u from
+// the row's own maximum instead narrowed the bins but cost a cluster-wide
+// min/max round and a separate histogram pass.)  Rows whose scores sit in a
+// band narrower than a bin take the rescan path below.
 //
 // Steps ('|' is a cluster barrier):
-//   bulk copy, keys, local min/max | row min/max
-//   pass 1: 4096-bin histogram of the top digit of V | every CTA sums the C
-//           histograms through distributed shared memory (1024 bins at a
-//           time, stopping at the chunk that holds the threshold digit t:
-//           the smallest d with count(digits <= d) >= k)
+//   bulk copy, keys and the pass-1 histogram (4096 bins, top digit of V) |
+//           every CTA sums the C histograms through distributed shared
+//           memory (1024 bins at a time, stopping at the chunk that holds the
+//           threshold digit t: the smallest d with count(digits <= d) >= k)
 //   then one of
 //   exact:  bin t holds exactly the positions still needed: every CTA writes
 //           its positions with digit <= t to the output | done
@@ -170,15 +173,12 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   uint32_t* s_hist = s_key + a.scap;                                     // [2][BINS]
   uint64_t* s_cand = reinterpret_cast<uint64_t*>(s_hist + 2 * BINS);    // rank 0: gathered V
   __shared__ __align__(8) uint64_t s_bar[NCHUNK];
-  __shared__ uint32_t s_red[64];
   __shared__ uint32_t s_warp[32];
-  __shared__ __align__(8) uint32_t s_mm[2];     // this CTA's min and max key
-  __shared__ uint32_t s_gmm[2];                 // the row's
   __shared__ uint32_t s_t, s_cb, s_cnt;         // threshold digit, count below it, its count
   __shared__ __align__(8) uint64_t s_ctr;      // rank 0: output slots | gathered candidates << 32
   __shared__ uint32_t s_obase, s_cbase;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int C = static_cast<int>(gridDim.x);    // cluster = one grid row
   const uint32_t rank = cluster_ctarank();
   pdl_trigger();
@@ -225,16 +225,16 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   for (int i = tid; i < 2 * BINS; i += THREADS) s_hist[i] = 0;
   __syncthreads();                              // barriers initialised before any wait
 
-  // ---- keys in place and local min / max, chunk by chunk as the copies land
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  auto minmax4 = [&](uint4 k, int j, int lim) {
+  // ---- keys in place and the pass-1 histogram, chunk by chunk as the copies
+  // land.  V measures a key down from the largest possible key (u = ~key), so
+  // the pass-1 digit is the top DIGIT bits of ~key (sign, exponent and three
+  // mantissa bits of the score): every CTA bins alike with no agreement on
+  // the row's range first, and the histogram overlaps the copies.
+  auto hist4 = [&](uint4 k, int j, int lim) {
     const uint32_t e[4] = {k.x, k.y, k.z, k.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t)
-      if (j + t < lim) {
-        kmin = min(kmin, e[t]);
-        kmax = max(kmax, e[t]);
-      }
+      if (j + t < lim) atomicAdd(&s_hist[(~e[t]) >> (32 - DIGIT)], 1u);
   };
   for (int c = 0; c < nch; ++c) {
     mbar_wait(&s_bar[c], 0, a.err);
@@ -243,46 +243,24 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
       const float4 v = *reinterpret_cast<const float4*>(s_key + j);
       const uint4 k = make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w));
       *reinterpret_cast<uint4*>(s_key + j) = k;
-      minmax4(k, j, nsm);
+      hist4(k, j, nsm);
     }
   }
   for (int j = a.scap + 4 * tid; j < n; j += 4 * THREADS) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(grow + j));
-    minmax4(make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w)), j, n);
+    hist4(make_uint4(float_key(v.x), float_key(v.y), float_key(v.z), float_key(v.w)), j, n);
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  if (lane == 0) { s_red[warp] = kmin; s_red[32 + warp] = kmax; }
-  __syncthreads();
-  if (warp == 0) {
-    kmin = __reduce_min_sync(0xffffffffu, s_red[lane]);
-    kmax = __reduce_max_sync(0xffffffffu, s_red[32 + lane]);
-    if (lane == 0) { s_mm[0] = kmin; s_mm[1] = kmax; }
-  }
-  cluster_sync();            // min/max of every CTA, keys, zeroed histograms and counters
-  if (warp == 0) {
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-    if (lane < C) {
-      const uint2 r = ld_cluster_u2(map_to_rank(smem_u32(s_mm), static_cast<uint32_t>(lane)));
-      mn = r.x;
-      mx = r.y;
-    }
-    mn = __reduce_min_sync(0xffffffffu, mn);
-    mx = __reduce_max_sync(0xffffffffu, mx);
-    if (lane == 0) { s_gmm[0] = mn; s_gmm[1] = mx; }
-  }
-  __syncthreads();
-  const uint32_t gmax = s_gmm[1];
-  const uint32_t range = gmax - s_gmm[0];
+  cluster_sync();            // every CTA's keys and pass-1 histogram; counters zeroed
+  const uint32_t gmax = 0xFFFFFFFFu;                    // u = gmax - key = ~key
+  const uint32_t range = gmax;
   const int pb = 32 - __clz(vis - 1);                   // vis >= 2 here
   const uint64_t pos_mask = (1ull << pb) - 1ull;
   auto make_v = [&](int pos, uint32_t key) -> uint64_t {
     return (static_cast<uint64_t>(gmax - key) << pb) | static_cast<uint64_t>(pos);
   };
-
-  // ---- pass 1: the top DIGIT bits of V.  When sh0 >= pb (a score range of
-  // at least 2^12 keys, the usual case) the digit is (kmax - key) >> (sh0 - pb)
-  // and every later test on it is a comparison of the key with a bound.
+  // pass 1 took the top DIGIT bits of V = (~key << pb) | pos: with 32 + pb
+  // significant bits, sh0 - pb = 32 - DIGIT and every later test on the
+  // digit is a comparison of the key with a bound
   const int tb = (range ? 32 - __clz(range) : 0) + pb;  // significant bits of V
   const int w0 = min(DIGIT, tb);
   const int sh0 = tb - w0;
@@ -292,16 +270,6 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   auto digit0 = [&](int pos, uint32_t key) -> uint32_t {   // general form
     return (((gmax - key) << (pb - sh0)) | (static_cast<uint32_t>(pos) >> sh0)) & dmask0;
   };
-  if (fast0) {
-    for_slice(s_key, grow, beg, n, a.scap, [&](int, uint32_t key, bool valid) {
-      if (valid) atomicAdd(&s_hist[(gmax - key) >> us0], 1u);
-    });
-  } else {
-    for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
-      if (valid) atomicAdd(&s_hist[digit0(pos, key)], 1u);
-    });
-  }
-  cluster_sync();            // every CTA's pass-1 histogram is complete
 
   // threshold digit of the cluster's summed histograms; h = this pass's buffer
   auto merged_threshold = [&](const uint32_t* h, uint32_t need) {
@@ -358,10 +326,11 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
 
   // digit < t0 ("better") and digit <= t0 ("in"): in the fast form
   // key >= kb1 and key >= kin1, from u < t0 << us0 and u < (t0 + 1) << us0
-  const uint32_t kb1 = gmax - (t0 << us0) + 1u;              // t0 << us0 <= range <= gmax
+  // (64-bit: with t0 = 0 the bound is 2^32 and no key is better)
+  const uint64_t kb1 = static_cast<uint64_t>(gmax) - (static_cast<uint64_t>(t0) << us0) + 1u;
   const uint64_t u2 = static_cast<uint64_t>(t0 + 1u) << us0;
   const uint32_t kin1 = u2 > gmax ? 0u : static_cast<uint32_t>(gmax - u2 + 1u);
-  auto fast_better = [&](int, uint32_t key) { return key >= kb1; };
+  auto fast_better = [&](int, uint32_t key) { return static_cast<uint64_t>(key) >= kb1; };
   auto fast_in = [&](int, uint32_t key) { return key >= kin1; };
   auto gen_better = [&](int pos, uint32_t key) { return digit0(pos, key) < t0; };
   auto gen_in = [&](int pos, uint32_t key) { return digit0(pos, key) <= t0; };
