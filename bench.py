@@ -410,7 +410,8 @@ def run_ours(args, rank, world, local_rank):
     idx_bytes = key_b // ((n + G - 1) // G)
     achieved = idx_bytes / (idx_ms / 1e3) / 1e9
     step_mean_ms = total_ms / args.steps
-    launches_per_step = ng * (1 + 1 + (1 if inp.mtp_index_share else 0)) + n * (1 + (1 if S > 1 else 0))
+    S_used = dsa.dsa_choose_splits(Q, inp.topk, S)
+    launches_per_step = ng * (1 + 1 + (1 if inp.mtp_index_share else 0)) + n * (1 + (1 if S_used > 1 else 0))
     res = {
         "metric": METRIC, "value": job_throughput(Q, world, args.steps, total_ms), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_mean_ms,

@@ -101,6 +101,16 @@ int dsa_version(void);
 size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits);
 
 /*
+ * Split-K parts the sparse MLA calls use for Q queries and `topk` selected
+ * tokens: num_splits itself when it is 1..DSA_MAX_SPLITS (capped at topk),
+ * the library's choice for 0 (the fewest parts whose (query, part) units,
+ * each on a pair of SMs, fill the GPU's SM pairs to at least 85% over whole
+ * waves, with at least 64 tokens a part).  With more than one part the call
+ * also runs the LSE merge.  Returns 0 for invalid sizes.  Host only.
+ */
+int dsa_choose_splits(int Q, int topk, int num_splits);
+
+/*
  * Lightning indexer, scores only  (section 2.2: the indexer stage).
  *   q_idx  e4m3 [Q,64,128]     w [Q,64] fp32      k_idx e4m3 [total_keys,128]
  *   seq_offsets int64 [B+1], q_offsets int32 [B+1], q_vis int32 [Q] (device)

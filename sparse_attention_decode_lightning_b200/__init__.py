@@ -33,6 +33,7 @@ SIGNATURES = {
     "dsa_status_string": (ctypes.c_char_p, [_I]),
     "dsa_version": (_I, []),
     "dsa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "dsa_choose_splits": (_I, [_I, _I, _I]),
     "dsa_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _SZ, _P]),
     "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -105,6 +106,10 @@ def dsa_version() -> int:
 
 def dsa_status_string(s: int) -> str:
     return lib().dsa_status_string(s).decode()
+
+
+def dsa_choose_splits(Q: int, topk: int, num_splits: int = 0) -> int:
+    return lib().dsa_choose_splits(Q, topk, num_splits)
 
 
 def dsa_workspace_bytes(Q: int, max_len: int, topk: int, num_splits: int = 0) -> int:

@@ -192,6 +192,12 @@ const char* dsa_status_string(int s) {
 
 int dsa_version(void) { return 100; }
 
+int dsa_choose_splits(int Q, int topk, int num_splits) {
+  if (Q <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || num_splits < 0 || num_splits > DSA_MAX_SPLITS)
+    return 0;
+  return choose_splits(Q, topk, num_splits);
+}
+
 size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits) {
   WsLayout L;
   if (!ws_layout(Q, max_len, topk, num_splits, &L)) return 0;

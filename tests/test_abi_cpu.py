@@ -45,6 +45,19 @@ def test_library_loads_and_reports_version_and_status_names():
     assert dsa.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
 
 
+def test_split_choice():
+    f = dsa.dsa_choose_splits
+    assert f(0, 2048, 0) == 0 and f(1, 0, 0) == 0 and f(1, 2048, 33) == 0
+    assert f(32, 2048, 5) == 5 and f(4, 2048, 16) == 16
+    assert f(1, 8, 16) == 8                      # never more parts than tokens
+    # the library's choice: 32 queries on 74 SM pairs -> 2 parts (64 units, 86%)
+    assert f(32, 2048, 0) == 2
+    assert f(128, 2048, 0) == 1 and f(74, 2048, 0) == 1
+    for q in (1, 3, 16, 40, 500):
+        s = f(q, 2048, 0)
+        assert 1 <= s <= 16 and 2048 // s >= 64
+
+
 def test_workspace_bytes_arithmetic():
     f = dsa.dsa_workspace_bytes
     assert f(0, 10, 2048, 0) == 0
