@@ -236,8 +236,8 @@ def run_ours(args, rank, world, local_rank):
     S = inp.num_splits
     stream = torch.cuda.current_stream(dev)
     ws = dsa.workspace(Q, inp.max_len, inp.topk, S, device=dev)
-    outs = [torch.empty(Q, 128, 512, device=dev) for _ in range(n)]
-    lses = [torch.empty(Q, 128, device=dev) for _ in range(n)]
+    outs = [torch.empty(Q, inp.heads, 512, device=dev) for _ in range(n)]
+    lses = [torch.empty(Q, inp.heads, device=dev) for _ in range(n)]
     ng = (n + G - 1) // G
     idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=dev)
     qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
@@ -443,7 +443,7 @@ def workload_config(wl, B, S, world):
     return {"workload": wl.name, "B": B, "T": wl.T, "L": wl.L,
             "L_range": list(wl.L_range) if wl.L_range else None, "layers": wl.n_layers,
             "index_share": wl.index_share, "mtp_index_share": wl.mtp_index_share,
-            "topk": wl.topk, "num_splits": S,
+            "topk": wl.topk, "num_splits": S, "heads": wl.heads, "idx_heads": wl.idx_heads,
             "parallelism": f"replicas{world}" if world > 1 else "single",
             "l2": "inputs larger than L2 (FP8 keys) and a 256 MiB L2 flush before every step"}
 

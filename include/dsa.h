@@ -11,16 +11,23 @@
  *     512 plus a 64-d RoPE part (576 values), 128 attention heads.
  *   Same page, section 7.2 GLM-5.2 / Figure 7-2: IndexShare -- one indexer per
  *     group of sparse layers; the following layers reuse its top-k indices.
+ *     The same section gives GLM-5.2's shapes: 64 MLA heads (qk head dim
+ *     192 + 64 RoPE, kv rank 512) and a 32-head FP8 indexer of head dim 128,
+ *     top-2048 causal keys.  Absorbed into MQA form its cached latent is the
+ *     same 576-value row (512 kv rank + 64 RoPE), so the calls below take
+ *     the head counts as arguments: heads = 128 or 64, idx_heads = 64 or 32
+ *     (any other value returns DSA_ERR_UNSUPPORTED).
  *   "GLM-5.2 推理部署" (inference deployment), MTP draft + verify flow: top-K
  *     = 2048 indices computed once and reused across the MTP positions.
  *
  * Definitions used throughout (readings where the pages give no formula):
- *   indexer score   I[q,s] = sum_{h<64} w[q,h] * max(0, sum_{d<128} qi[q,h,d]*K[s,d])
+ *   indexer score   I[q,s] = sum_{h<HI} w[q,h] * max(0, sum_{d<128} qi[q,h,d]*K[s,d])
+ *                   with HI = idx_heads indexer heads;
  *                   qi and K are FP8 e4m3 bytes at scale 1, w is fp32;
  *   selector        the topk positions s < vis[q] with the largest I[q,s],
  *                   ties to the lower s; if vis[q] < topk every visible s is
  *                   kept and the remaining slots hold -1;
- *   sparse MLA      per head h:  z_j = scale * <q[h,0:576], C[idx_j,0:576]>,
+ *   sparse MLA      per head h < heads:  z_j = scale * <q[h,0:576], C[idx_j,0:576]>,
  *                   O[h] = sum_j softmax_j(z) * C[idx_j,0:512],
  *                   LSE[h] = ln sum_j exp(z_j)  (empty set: O = 0, LSE = -inf);
  *   split-K         the selected set is partitioned into num_splits parts, each
@@ -62,10 +69,12 @@ extern "C" {
 #endif
 
 #define DSA_PAGE_SIZE 64        /* latent-cache page (tokens) */
-#define DSA_HEADS 128           /* MLA query heads */
+#define DSA_HEADS 128           /* MLA query heads (DeepSeek-V3.2) */
+#define DSA_HEADS_GLM 64        /* MLA query heads (GLM-5.2) */
 #define DSA_DIM 576             /* latent row: 512 kv-rank + 64 RoPE */
 #define DSA_DIM_V 512           /* value dims (first 512 of the row) */
-#define DSA_IDX_HEADS 64        /* indexer heads */
+#define DSA_IDX_HEADS 64        /* indexer heads (DeepSeek-V3.2) */
+#define DSA_IDX_HEADS_GLM 32    /* indexer heads (GLM-5.2) */
 #define DSA_IDX_DIM 128         /* indexer head dim */
 #define DSA_MAX_TOPK 2048
 #define DSA_MAX_Q_PER_SEQ 8     /* 1 decode token + up to 7 MTP drafts */
@@ -92,7 +101,8 @@ int dsa_version(void);
  * Bytes of device workspace the calls below need for Q queries, contexts of at
  * most max_len keys, `topk` selected tokens and `num_splits` split-K parts
  * (0 = let the library choose).  The workspace holds the fp32 score rows
- * [Q, max_len], the split-K partial outputs and the device error flag (the
+ * [Q, max_len], the split-K partial outputs (sized for 128 heads, so one
+ * workspace serves both head counts) and the device error flag (the
  * selector keeps its histograms and candidate lists in on-chip memory).  The same workspace may be
  * reused by consecutive calls on one stream; it must be zeroed once
  * (cudaMemset) before its first use so the error flag starts clear.
@@ -112,7 +122,8 @@ int dsa_choose_splits(int Q, int topk, int num_splits);
 
 /*
  * Lightning indexer, scores only  (section 2.2: the indexer stage).
- *   q_idx  e4m3 [Q,64,128]     w [Q,64] fp32      k_idx e4m3 [total_keys,128]
+ *   q_idx  e4m3 [Q,idx_heads,128]   w [Q,idx_heads] fp32   k_idx e4m3 [total_keys,128]
+ *   idx_heads  64 (DeepSeek-V3.2) or 32 (GLM-5.2)
  *   seq_offsets int64 [B+1], q_offsets int32 [B+1], q_vis int32 [Q] (device)
  *   scores fp32 [Q, ld_scores]: row q gets I[q,s] for s < q_vis[q]; other
  *          entries are left untouched.  ld_scores >= max_len, multiple of 4.
@@ -122,8 +133,8 @@ int dsa_choose_splits(int Q, int topk, int num_splits);
 dsa_status dsa_indexer_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                               int64_t total_keys, const int64_t* seq_offsets,
                               const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                              int max_len, int first_only, float* scores, int ld_scores,
-                              void* ws, size_t ws_bytes, void* stream);
+                              int idx_heads, int max_len, int first_only, float* scores,
+                              int ld_scores, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Token selector on given scores  (section 2.2: the token selector stage).
@@ -153,13 +164,17 @@ dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_
 dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                             int64_t total_keys, const int64_t* seq_offsets,
                             const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                            int max_len, int topk, int first_only, int32_t* out_idx,
-                            float* out_scores, void* ws, size_t ws_bytes, void* stream);
+                            int idx_heads, int max_len, int topk, int first_only,
+                            int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /*
  * Sparse MLA decode in absorbed-MQA form over the selected tokens
- * (section 2.2: MLA in MQA mode; section 2.1: 576-d latent, 128 heads).
- *   q          bf16 [Q,128,576]  absorbed queries (512 latent + 64 RoPE)
+ * (section 2.2: MLA in MQA mode; section 2.1: 576-d latent, 128 heads;
+ * section 7.2: GLM-5.2's 64 heads).
+ *   q          bf16 [Q,heads,576]  absorbed queries (512 latent + 64 RoPE)
+ *   heads      128 (DeepSeek-V3.2) or 64 (GLM-5.2); 64 heads run on the same
+ *              128-row tensor-core tiles with the upper rows unused
  *   kv_pool    bf16 [num_pages,64,576]  paged latent cache shared by all heads
  *   page_table int32 [B,max_pages]: page of token s of sequence b is
  *              page_table[b*max_pages + s/64], row s%64 in that page.  A
@@ -168,7 +183,7 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
  *   scale      softmax scale applied to the 576-d dot product.
  *   num_splits split-K parts (1..DSA_MAX_SPLITS, 0 = library's choice); the
  *              idx row is cut into equal-count parts merged exactly by LSE.
- *   out        fp32 [Q,128,512]      lse fp32 [Q,128] (natural log)
+ *   out        fp32 [Q,heads,512]    lse fp32 [Q,heads] (natural log)
  * Entries with idx >= q_vis[q], a page id outside [0,num_pages) or a page
  * slot beyond max_pages are skipped and flagged (DSA_ERR_DEVICE_BOUNDS).
  * Precision: bf16 products accumulate in fp32 on the tensor cores.  Each
@@ -181,8 +196,8 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
 dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int topk, float scale,
-                                 int num_splits, float* out, float* lse,
+                                 const int32_t* idx, int B, int Q, int heads, int topk,
+                                 float scale, int num_splits, float* out, float* lse,
                                  void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -195,7 +210,8 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
  *   The split-K partial outputs live in a fixed 16 MiB array of device memory
  *   owned by the library (every GPU that loads the library holds it until
  *   the process exits), so Q * num_splits (after the library's choice when
- *   num_splits = 0) may not exceed 63 when it is above 1; larger requests
+ *   num_splits = 0) may not exceed 63 at 128 heads (127 at 64 heads) when it
+ *   is above 1; larger requests
  *   return DSA_ERR_UNSUPPORTED and enqueue nothing.  num_splits = 1 uses no
  *   scratch and has no limit on Q.
  *   The first call on a device looks up the array's device address (with
@@ -209,15 +225,16 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
 dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool, int num_pages,
                                          const int32_t* page_table, int max_pages,
                                          const int32_t* q_offsets, const int32_t* q_vis,
-                                         const int32_t* idx, int B, int Q, int topk, float scale,
-                                         int num_splits, float* out, float* lse, void* stream);
+                                         const int32_t* idx, int B, int Q, int heads, int topk,
+                                         float scale, int num_splits, float* out, float* lse,
+                                         void* stream);
 
 /*
  * Merge of split-K partial attentions (exact LSE combine).
- *   o_parts fp32 [Q,S,128,512], lse_parts fp32 [Q,S,128] (-inf = empty part)
- *   out fp32 [Q,128,512], lse fp32 [Q,128].
+ *   o_parts fp32 [Q,S,heads,512], lse_parts fp32 [Q,S,heads] (-inf = empty part)
+ *   out fp32 [Q,heads,512], lse fp32 [Q,heads]; heads = 128 or 64.
  */
-dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S,
+dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, int heads,
                            float* out, float* lse, void* stream);
 
 /*
@@ -232,7 +249,8 @@ dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, 
  *   mtp_index_share  != 0: the first query of each sequence supplies the
  *                    top-k of all its queries (draft positions reuse step 1).
  *   idx_out          int32 [ceil(n_layers/G), Q, topk]: the index rows used.
- *   out_layers / lse_layers: per layer fp32 [Q,128,512] / [Q,128].
+ *   out_layers / lse_layers: per layer fp32 [Q,heads,512] / [Q,heads].
+ *   heads / idx_heads: 128 / 64 (DeepSeek-V3.2) or 64 / 32 (GLM-5.2).
  * Other arguments as in dsa_indexer_topk and dsa_sparse_mla_decode.
  * The kernels of one call (and of dsa_indexer_topk) are chained with
  * programmatic dependent launch: a kernel may start its set-up while the
@@ -245,7 +263,8 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                            const uint8_t* const* q_idx_layers, const float* const* w_layers,
                            const uint8_t* const* k_idx_layers, int64_t total_keys,
                            const int64_t* seq_offsets, const int32_t* q_offsets,
-                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           const int32_t* q_vis, int B, int Q, int heads, int idx_heads,
+                           int max_len, int topk,
                            const void* const* q_layers, const void* const* pool_layers,
                            int num_pages, const int32_t* const* page_table_layers,
                            int max_pages, float scale, int num_splits,

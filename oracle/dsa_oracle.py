@@ -16,7 +16,10 @@ Sources (pages are cited by title and section):
           token, kv rank 512 plus a 64-d RoPE part; 128 attention heads.
   [ARCH-7.2] same page, section 7.2 GLM-5.2 and Figure 7-2: IndexShare, one
           indexer per 4 sparse layers whose top-k indices the next 3 layers
-          reuse; causal top-2048.
+          reuse; causal top-2048.  GLM-5.2's shapes: 64 MLA heads over a
+          kv rank of 512 with a 64-d RoPE part, a 32-head FP8 indexer of head
+          dim 128.  Every function below takes its head counts from the
+          arrays it is given, so both models' shapes go through the same code.
   [GLM-INF] "GLM-5.2 推理部署" (inference deployment), MTP draft + verify flow:
           top-K = 2048 indices computed at draft step 1 and reused by later
           steps; verify appends the drafts and runs one prefill-style forward.
@@ -95,14 +98,14 @@ def bf16_decode(bits: np.ndarray) -> np.ndarray:
 def indexer_scores(q_idx: np.ndarray, w: np.ndarray, keys: np.ndarray) -> np.ndarray:
     """Scores of every key for one query.
 
-    q_idx: e4m3 bytes [64,128] (one query's indexer heads)
-    w:     float [64] head weights
+    q_idx: e4m3 bytes [HI,128] (one query's indexer heads: 64, or GLM-5.2's 32)
+    w:     float [HI] head weights
     keys:  e4m3 bytes [n,128] (the query's visible indexer keys)
     returns float64 [n]: I[s] = sum_h w[h] * max(0, sum_d q[h,d] * K[s,d])
     """
-    qf = e4m3_decode(q_idx)                      # [64,128]
+    qf = e4m3_decode(q_idx)                      # [HI,128]
     kf = e4m3_decode(keys)                       # [n,128]
-    dots = kf @ qf.T                             # [n,64]  per-head q.k
+    dots = kf @ qf.T                             # [n,HI]  per-head q.k
     relu = np.maximum(dots, 0.0)
     return relu @ np.asarray(w, dtype=np.float64)
 
@@ -136,19 +139,19 @@ def latent_rows(pool: np.ndarray, page_table_row: np.ndarray, positions: np.ndar
 
 
 def sparse_mla(q: np.ndarray, rows: np.ndarray, scale: float) -> Tuple[np.ndarray, np.ndarray]:
-    """Attention of 128 heads over n selected latent rows (one shared row per
-    token serves every head).
+    """Attention of H heads (128, or GLM-5.2's 64) over n selected latent
+    rows (one shared row per token serves every head).
 
-    q:    float64 [128,576]
+    q:    float64 [H,576]
     rows: float64 [n,576]
-    returns O float64 [128,512] = softmax_j(scale * q.c_j) @ c_j[:512]
-            LSE float64 [128]   = ln sum_j exp(scale * q.c_j)
+    returns O float64 [H,512] = softmax_j(scale * q.c_j) @ c_j[:512]
+            LSE float64 [H]   = ln sum_j exp(scale * q.c_j)
     With n = 0: O = 0 and LSE = -inf.
     """
     nh = q.shape[0]
     if rows.shape[0] == 0:
         return np.zeros((nh, DV)), np.full(nh, -np.inf)
-    s = scale * (q @ rows.T)                     # [128,n]
+    s = scale * (q @ rows.T)                     # [H,n]
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
@@ -204,8 +207,9 @@ def decode_step(inp: Dict, queries: Optional[Sequence[int]] = None,
 
     inp keys (numpy arrays): B, T, topk, scale, num_splits, index_share,
       mtp_index_share, n_layers, seq_offsets[B+1], q_vis[Q], page_table[B,P],
-      indexer: list per group of {q_idx[Q,64,128] u8, w[Q,64] f32, k_idx[N,128] u8},
-      layers: list per layer of {q[Q,128,576] u16 bits, pool[P,64,576] u16 bits}.
+      indexer: list per group of {q_idx[Q,HI,128] u8, w[Q,HI] f32, k_idx[N,128] u8},
+      layers: list per layer of {q[Q,H,576] u16 bits, pool[P,64,576] u16 bits},
+      with (H, HI) = (128, 64) for DeepSeek-V3.2 and (64, 32) for GLM-5.2.
     Layer l takes its indices from the indexer of group l // index_share
     (IndexShare); with mtp_index_share the first position of each sequence
     supplies the indices of all its positions (IndexShare on MTP).

@@ -15,10 +15,12 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 PAGE_SIZE = 64
-HEADS = 128
+HEADS = 128          # MLA heads, DeepSeek-V3.2
+HEADS_GLM = 64       # MLA heads, GLM-5.2
 DIM = 576
 DIM_V = 512
-IDX_HEADS = 64
+IDX_HEADS = 64       # indexer heads, DeepSeek-V3.2
+IDX_HEADS_GLM = 32   # indexer heads, GLM-5.2
 IDX_DIM = 128
 MAX_TOPK = 2048
 MAX_Q_PER_SEQ = 8
@@ -34,16 +36,18 @@ SIGNATURES = {
     "dsa_version": (_I, []),
     "dsa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "dsa_choose_splits": (_I, [_I, _I, _I]),
-    "dsa_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _SZ, _P]),
+    "dsa_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _SZ,
+                                _P]),
     "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
-    "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
-    "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P,
-                                   _SZ, _P]),
-    "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _F, _I, _P,
-                                           _P, _P]),
-    "dsa_lse_combine": (_I, [_P, _P, _I, _I, _P, _P, _P]),
-    "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _PP, _PP,
-                             _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
+    "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
+                              _P]),
+    "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P,
+                                   _P, _SZ, _P]),
+    "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I,
+                                           _P, _P, _P]),
+    "dsa_lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
+    "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                             _PP, _PP, _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
     "dsa_check_error": (_I, [_P, _P]),
 }
 
@@ -128,8 +132,8 @@ def dsa_indexer_scores(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_le
                        first_only=False, stream=None):
     _check(lib().dsa_indexer_scores(
         _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
-        _ptr(q_vis), B, q_idx.shape[0], max_len, int(first_only), _ptr(scores), scores.shape[1],
-        _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_scores")
+        _ptr(q_vis), B, q_idx.shape[0], q_idx.shape[1], max_len, int(first_only), _ptr(scores),
+        scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_scores")
 
 
 def dsa_topk_select(scores, q_offsets, q_vis, B, max_len, topk, out_idx, ws, out_scores=None,
@@ -144,16 +148,16 @@ def dsa_indexer_topk(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len,
                      ws, out_scores=None, first_only=False, stream=None):
     _check(lib().dsa_indexer_topk(
         _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
-        _ptr(q_vis), B, q_idx.shape[0], max_len, topk, int(first_only), _ptr(out_idx),
-        _ptr(out_scores), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
+        _ptr(q_vis), B, q_idx.shape[0], q_idx.shape[1], max_len, topk, int(first_only),
+        _ptr(out_idx), _ptr(out_scores), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
 
 
 def dsa_sparse_mla_decode(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scale, out, lse, ws,
                           num_splits=0, stream=None):
     _check(lib().dsa_sparse_mla_decode(
         _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
-        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], idx.shape[1], float(scale),
-        num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1],
+        float(scale), num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
         "dsa_sparse_mla_decode")
 
 
@@ -163,13 +167,14 @@ def dsa_sparse_mla_decode_noalloc(q, kv_pool, page_table, q_offsets, q_vis, idx,
     library's own fixed device array; see include/dsa.h)."""
     _check(lib().dsa_sparse_mla_decode_noalloc(
         _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
-        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], idx.shape[1], float(scale),
-        num_splits, _ptr(out), _ptr(lse), _stream(stream)), "dsa_sparse_mla_decode_noalloc")
+        _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1],
+        float(scale), num_splits, _ptr(out), _ptr(lse), _stream(stream)),
+        "dsa_sparse_mla_decode_noalloc")
 
 
 def dsa_lse_combine(o_parts, lse_parts, out, lse, stream=None):
-    Q, S = lse_parts.shape[0], lse_parts.shape[1]
-    _check(lib().dsa_lse_combine(_ptr(o_parts), _ptr(lse_parts), Q, S, _ptr(out), _ptr(lse),
+    Q, S, H = lse_parts.shape[0], lse_parts.shape[1], lse_parts.shape[2]
+    _check(lib().dsa_lse_combine(_ptr(o_parts), _ptr(lse_parts), Q, S, H, _ptr(out), _ptr(lse),
                                  _stream(stream)), "dsa_lse_combine")
 
 
@@ -180,10 +185,12 @@ def dsa_decode_step(q_idx_layers, w_layers, k_idx_layers, seq_offsets, q_offsets
     """Per-layer lists; entries of the indexer lists for non-indexer layers may be None."""
     n = len(q_layers)
     lead = next(t for t in k_idx_layers if t is not None)
+    lead_q = next(t for t in q_idx_layers if t is not None)
     _check(lib().dsa_decode_step(
         n, index_share, int(mtp_index_share), _ptr_array(q_idx_layers), _ptr_array(w_layers),
         _ptr_array(k_idx_layers), lead.shape[0], _ptr(seq_offsets), _ptr(q_offsets), _ptr(q_vis),
-        B, q_layers[0].shape[0], max_len, topk, _ptr_array(q_layers), _ptr_array(pool_layers),
+        B, q_layers[0].shape[0], q_layers[0].shape[1], lead_q.shape[1], max_len, topk,
+        _ptr_array(q_layers), _ptr_array(pool_layers),
         pool_layers[0].shape[0], _ptr_array(page_table_layers), page_table_layers[0].shape[1],
         float(scale), num_splits, _ptr_array(out_layers), _ptr_array(lse_layers), _ptr(idx_out),
         _ptr(ws), ws.numel(), _stream(stream)), "dsa_decode_step")

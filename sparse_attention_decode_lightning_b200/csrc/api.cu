@@ -11,9 +11,9 @@ namespace dsa {
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                                    int num_pages, const int32_t* page_table, int max_pages,
                                    const int32_t* q_offsets, const int32_t* q_vis,
-                                   const int32_t* idx, int B, int Q, int topk, float scale,
-                                   int S, float* out, float* lse, float* o_part, float* l_part,
-                                   uint32_t* err, cudaStream_t st, bool pdl);
+                                   const int32_t* idx, int B, int Q, int H, int topk,
+                                   float scale, int S, float* out, float* lse, float* o_part,
+                                   float* l_part, uint32_t* err, cudaStream_t st, bool pdl);
 
 namespace {
 
@@ -97,9 +97,15 @@ dsa_status check_common(const int64_t* seq_offsets, const int32_t* q_offsets,
   return DSA_OK;
 }
 
+// head counts of the two model shapes: DeepSeek-V3.2 (128 MLA heads, 64
+// indexer heads) and GLM-5.2 (64 and 32)
+bool heads_ok(int heads) { return heads == DSA_HEADS || heads == DSA_HEADS_GLM; }
+bool idx_heads_ok(int idx_heads) { return idx_heads == DSA_IDX_HEADS || idx_heads == DSA_IDX_HEADS_GLM; }
+
 dsa_status indexer_checks(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
-                          int64_t total_keys) {
+                          int64_t total_keys, int idx_heads) {
   if (!q_idx || !w || !k_idx) return DSA_ERR_INVALID_ARG;
+  if (!idx_heads_ok(idx_heads)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
   if (total_keys <= 0) return DSA_ERR_INVALID_ARG;
   if (total_keys >= (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
@@ -111,12 +117,12 @@ dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_E
 dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                           int max_len, int topk, int first_only, int32_t* out_idx,
+                           int idx_heads, int max_len, int topk, int first_only, int32_t* out_idx,
                            float* out_scores, void* ws, const WsLayout& L, cudaStream_t st) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* scores = ws_ptr<float>(ws, L.scores);
   cudaError_t e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B,
-                                 Q, first_only, scores, L.ld, err, st);
+                                 Q, idx_heads, first_only, scores, L.ld, err, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   // the selector starts while the indexer drains (its scores are waited for)
   e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
@@ -131,19 +137,19 @@ dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* 
 
 dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
                          const int32_t* page_table, int max_pages, const int32_t* q_offsets,
-                         const int32_t* q_vis, const int32_t* idx, int B, int Q, int topk,
-                         float scale, int S, float* out, float* lse, void* ws,
+                         const int32_t* q_vis, const int32_t* idx, int B, int Q, int H,
+                         int topk, float scale, int S, float* out, float* lse, void* ws,
                          const WsLayout& L, cudaStream_t st, bool pdl) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* o_part = ws_ptr<float>(ws, L.o_part);
   float* l_part = ws_ptr<float>(ws, L.l_part);
   cudaError_t e = launch_sparse_mla(static_cast<const __nv_bfloat16*>(q),
                                     static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
-                                    page_table, max_pages, q_offsets, q_vis, idx, B, Q, topk,
+                                    page_table, max_pages, q_offsets, q_vis, idx, B, Q, H, topk,
                                     scale, S, out, lse, o_part, l_part, err, st, pdl);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (S > 1) {
-    e = launch_combine(o_part, l_part, Q, S, out, lse, st, true);
+    e = launch_combine(o_part, l_part, Q, S, H, out, lse, st, true);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
   }
   return DSA_OK;
@@ -151,8 +157,9 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
 
 dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages,
                       const int32_t* page_table, int max_pages, const int32_t* idx, float* out,
-                      float* lse, float scale) {
+                      float* lse, float scale, int heads) {
   if (!q || !kv_pool || !page_table || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+  if (!heads_ok(heads)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kv_pool) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
   if (num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale != scale) return DSA_ERR_INVALID_ARG;
@@ -164,11 +171,11 @@ dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages,
 cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
                               const int32_t* page_table, int max_pages,
                               const int32_t* q_offsets, const int32_t* q_vis,
-                              const int32_t* idx, int B, int Q, int topk, float scale, int S,
+                              const int32_t* idx, int B, int Q, int H, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st, bool pdl) {
   return launch_sparse_mla_tc(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B,
-                              Q, topk, scale, S, out, lse, o_part, l_part, err, st, pdl);
+                              Q, H, topk, scale, S, out, lse, o_part, l_part, err, st, pdl);
 }
 
 }  // namespace dsa
@@ -190,7 +197,7 @@ const char* dsa_status_string(int s) {
   }
 }
 
-int dsa_version(void) { return 100; }
+int dsa_version(void) { return 200; }
 
 int dsa_choose_splits(int Q, int topk, int num_splits) {
   if (Q <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || num_splits < 0 || num_splits > DSA_MAX_SPLITS)
@@ -207,16 +214,16 @@ size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits) {
 dsa_status dsa_indexer_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                               int64_t total_keys, const int64_t* seq_offsets,
                               const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                              int max_len, int first_only, float* scores, int ld_scores,
-                              void* ws, size_t ws_bytes, void* stream) {
+                              int idx_heads, int max_len, int first_only, float* scores,
+                              int ld_scores, void* ws, size_t ws_bytes, void* stream) {
   dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, 1);
   if (s != DSA_OK) return s;
-  if ((s = indexer_checks(q_idx, w, k_idx, total_keys)) != DSA_OK) return s;
+  if ((s = indexer_checks(q_idx, w, k_idx, total_keys, idx_heads)) != DSA_OK) return s;
   if (!scores || !ws || ld_scores < max_len || (ld_scores & 3) || !aligned16(scores))
     return DSA_ERR_INVALID_ARG;
   if (ws_bytes < 256) return DSA_ERR_WORKSPACE;
   return cuda_status(launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis,
-                                    B, Q, first_only, scores, ld_scores,
+                                    B, Q, idx_heads, first_only, scores, ld_scores,
                                     static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
@@ -240,46 +247,50 @@ dsa_status dsa_topk_select(const float* scores, int ld_scores, const int32_t* q_
 dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                             int64_t total_keys, const int64_t* seq_offsets,
                             const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                            int max_len, int topk, int first_only, int32_t* out_idx,
-                            float* out_scores, void* ws, size_t ws_bytes, void* stream) {
+                            int idx_heads, int max_len, int topk, int first_only,
+                            int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
+                            void* stream) {
   dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, topk);
   if (s != DSA_OK) return s;
-  if ((s = indexer_checks(q_idx, w, k_idx, total_keys)) != DSA_OK) return s;
+  if ((s = indexer_checks(q_idx, w, k_idx, total_keys, idx_heads)) != DSA_OK) return s;
   if (!out_idx || !ws) return DSA_ERR_INVALID_ARG;
   WsLayout L;
   if (!ws_layout(Q, max_len, topk, 1, &L)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   return do_indexer_topk(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
-                         max_len, topk, first_only, out_idx, out_scores, ws, L,
+                         idx_heads, max_len, topk, first_only, out_idx, out_scores, ws, L,
                          static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int topk, float scale,
-                                 int num_splits, float* out, float* lse, void* ws,
+                                 const int32_t* idx, int B, int Q, int heads, int topk,
+                                 float scale, int num_splits, float* out, float* lse, void* ws,
                                  size_t ws_bytes, void* stream) {
   if (!q_offsets || !q_vis || !ws) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Q <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
   if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
   if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
-  dsa_status s = mla_checks(q, kv_pool, num_pages, page_table, max_pages, idx, out, lse, scale);
+  dsa_status s = mla_checks(q, kv_pool, num_pages, page_table, max_pages, idx, out, lse, scale,
+                            heads);
   if (s != DSA_OK) return s;
   WsLayout L;
   if (!ws_layout(Q, 1, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   return do_sparse_mla(q, kv_pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
-                       topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream), false);
+                       heads, topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream),
+                       false);
 }
 
-dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, float* out,
-                           float* lse, void* stream) {
+dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, int heads,
+                           float* out, float* lse, void* stream) {
   if (!o_parts || !lse_parts || !out || !lse) return DSA_ERR_INVALID_ARG;
   if (Q <= 0 || S <= 0) return DSA_ERR_INVALID_ARG;
+  if (!heads_ok(heads)) return DSA_ERR_UNSUPPORTED;
   if (Q > 65535 * 8 || S > 1024) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(o_parts) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
-  return cuda_status(launch_combine(o_parts, lse_parts, Q, S, out, lse,
+  return cuda_status(launch_combine(o_parts, lse_parts, Q, S, heads, out, lse,
                                     static_cast<cudaStream_t>(stream), false));
 }
 
@@ -287,7 +298,8 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                            const uint8_t* const* q_idx_layers, const float* const* w_layers,
                            const uint8_t* const* k_idx_layers, int64_t total_keys,
                            const int64_t* seq_offsets, const int32_t* q_offsets,
-                           const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                           const int32_t* q_vis, int B, int Q, int heads, int idx_heads,
+                           int max_len, int topk,
                            const void* const* q_layers, const void* const* pool_layers,
                            int num_pages, const int32_t* const* page_table_layers,
                            int max_pages, float scale, int num_splits,
@@ -302,10 +314,11 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
   if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
   for (int l = 0; l < n_layers; ++l) {
     if (l % index_share == 0 &&
-        (s = indexer_checks(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys)) != DSA_OK)
+        (s = indexer_checks(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys,
+                            idx_heads)) != DSA_OK)
       return s;
     if ((s = mla_checks(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
-                        idx_out, out_layers[l], lse_layers[l], scale)) != DSA_OK)
+                        idx_out, out_layers[l], lse_layers[l], scale, heads)) != DSA_OK)
       return s;
   }
   WsLayout L;
@@ -317,12 +330,12 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
     int32_t* idx_g = idx_out + static_cast<size_t>(g) * Q * topk;
     if (l % index_share == 0) {
       s = do_indexer_topk(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys, seq_offsets,
-                          q_offsets, q_vis, B, Q, max_len, topk, mtp_index_share, idx_g, nullptr,
-                          ws, L, st);
+                          q_offsets, q_vis, B, Q, idx_heads, max_len, topk, mtp_index_share, idx_g,
+                          nullptr, ws, L, st);
       if (s != DSA_OK) return s;
     }
     s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
-                      q_offsets, q_vis, idx_g, B, Q, topk, scale, L.S, out_layers[l],
+                      q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S, out_layers[l],
                       lse_layers[l], ws, L, st, true);
     if (s != DSA_OK) return s;
   }

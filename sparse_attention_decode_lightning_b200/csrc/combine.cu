@@ -1,7 +1,8 @@
 // Split-K merge of partial attentions by log-sum-exp:
 //   LSE = ln sum_c exp(LSE_c),  O = sum_c exp(LSE_c - LSE) O_c,
 // parts with LSE_c = -inf (no selected token) get weight 0; if every part is
-// empty O = 0 and LSE = -inf.  One CTA of 256 threads per (query, 8 heads): a
+// empty O = 0 and LSE = -inf.  H heads per query (128, or GLM-5.2's 64).
+// One CTA of 256 threads per (query, 8 heads): a
 // warp per head, 16 outputs per thread; the split weights are recomputed by
 // every thread from the S partial LSEs (L1-resident).  One CTA per head (4096
 // CTAs of 128 threads for 32 queries) spent its time in CTA scheduling.
@@ -16,19 +17,20 @@ constexpr int CTHREADS = HEADS_PER_CTA * DSA_DIM_V / 16;
 
 __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __restrict__ o_part,
                                                                const float* __restrict__ l_part,
-                                                               int S, float* __restrict__ out,
+                                                               int S, int H,
+                                                               float* __restrict__ out,
                                                                float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();                                   // the partials come from the previous kernel
   // CTA: query q, heads [h0, h0 + 8); thread: head h0 + tid / 32, outputs
   // [16 * (tid % 32), +16) as four float4 spread 128 floats apart
-  const int q = blockIdx.x / (DSA_HEADS / HEADS_PER_CTA);
-  const int h = (blockIdx.x % (DSA_HEADS / HEADS_PER_CTA)) * HEADS_PER_CTA + (threadIdx.x >> 5);
+  const int q = blockIdx.x / (H / HEADS_PER_CTA);
+  const int h = (blockIdx.x % (H / HEADS_PER_CTA)) * HEADS_PER_CTA + (threadIdx.x >> 5);
   const int c4 = threadIdx.x & 31;              // float4 column within each 128-float quarter
-  const size_t qh = static_cast<size_t>(q) * DSA_HEADS + h;
-  const float* lp = l_part + static_cast<size_t>(q) * S * DSA_HEADS + h;
+  const size_t qh = static_cast<size_t>(q) * H + h;
+  const float* lp = l_part + static_cast<size_t>(q) * S * H + h;
   float m = -INFINITY;
-  for (int c = 0; c < S; ++c) m = fmaxf(m, lp[static_cast<size_t>(c) * DSA_HEADS]);
+  for (int c = 0; c < S; ++c) m = fmaxf(m, lp[static_cast<size_t>(c) * H]);
   float4* o = reinterpret_cast<float4*>(out + qh * DSA_DIM_V) + c4;
   if (m == -INFINITY) {
 #pragma unroll
@@ -41,12 +43,12 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int c = 0; c < S; ++c) {
-    const float lc = lp[static_cast<size_t>(c) * DSA_HEADS];
+    const float lc = lp[static_cast<size_t>(c) * H];
     if (lc == -INFINITY) continue;
     const float wc = expf(lc - m);
     tot += wc;
     const float4* v = reinterpret_cast<const float4*>(
-                          o_part + ((static_cast<size_t>(q) * S + c) * DSA_HEADS + h) * DSA_DIM_V) + c4;
+                          o_part + ((static_cast<size_t>(q) * S + c) * H + h) * DSA_DIM_V) + c4;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float4 x = v[32 * k];
@@ -65,11 +67,12 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
 
 }  // namespace
 
-cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, float* out,
-                           float* lse, cudaStream_t st, bool pdl) {
+cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
+                           float* out, float* lse, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
+  if (H <= 0 || H % HEADS_PER_CTA) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(Q) * (DSA_HEADS / HEADS_PER_CTA), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(Q) * (H / HEADS_PER_CTA), 1, 1);
   cfg.blockDim = dim3(CTHREADS, 1, 1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -77,7 +80,7 @@ cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int 
   add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, lse_combine_kernel, o_part, l_part, S, out, lse);
+  return cudaLaunchKernelEx(&cfg, lse_combine_kernel, o_part, l_part, S, H, out, lse);
 }
 
 }  // namespace dsa

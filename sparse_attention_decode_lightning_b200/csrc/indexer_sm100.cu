@@ -3,7 +3,9 @@
 // Source: "大语言模型结构总览", section 2.2 DeepSeek-V3.2 -- the indexer is a
 // light FP8 scorer (64 heads x 128 dims) that gives every prior token of a
 // query one relevance scalar; it streams the whole key cache, which makes it
-// the HBM-bound part of the decode step.
+// the HBM-bound part of the decode step.  Section 7.2 GLM-5.2 gives the same
+// scorer with 32 heads; the kernel is instantiated for HI = 64 and HI = 32
+// heads (the per-query MMA has N = HI).
 //
 // Design (persistent, one CTA per SM, two independent sub-pipelines):
 // the CTA's contiguous range of (sequence, 128-key tile) items is cut in two
@@ -11,10 +13,10 @@
 //   a producer warp   TMA loads of 128-key x 128-byte e4m3 tiles (16 KB,
 //                     128-byte swizzle, L2 evict-first) into its own ring,
 //                     and the queries of its current sequence (8 KB each);
-//   an issuer warp    for every query of the tile's sequence, D[128 keys, 64
+//   an issuer warp    for every query of the tile's sequence, D[128 keys, HI
 //                     heads] = K_tile . q^T as 4 MMAs of kind::f8f6f4 (M=128,
-//                     N=64, K=32) into one of its 4 TMEM slots;
-//   an epilogue warpgroup   each thread reads its key row (64 fp32 head
+//                     N=HI, K=32) into one of its 4 TMEM slots;
+//   an epilogue warpgroup   each thread reads its key row (HI fp32 head
 //                     dots) with tcgen05.ld and reduces sum_h w_h max(d_h, 0)
 //                     in registers; scores are written coalesced.
 // A single issuer thread spends ~1500 cycles per tile on mbarrier waits, MMA
@@ -34,11 +36,11 @@ namespace {
 constexpr int KT = 128;                                // keys per tile (MMA M)
 constexpr int PIPES = 2;                               // independent sub-pipelines per CTA
 constexpr int SLOTS = 4;                               // TMEM accumulator slots per pipeline
-constexpr int ACC_COLS = DSA_IDX_HEADS;                // 64 fp32 columns per slot
+constexpr int ACC_COLS = DSA_IDX_HEADS;                // TMEM columns per slot (64 heads at most)
 constexpr int WARPS_PER_PIPE = 6;                      // producer, MMA issuer, 4 epilogue warps
 constexpr int THREADS = 32 * WARPS_PER_PIPE * PIPES;
 constexpr int KEY_TILE = KT * DSA_IDX_DIM;             // 16384 B
-constexpr int Q_TILE = DSA_IDX_HEADS * DSA_IDX_DIM;    // 8192 B
+constexpr int Q_TILE = DSA_IDX_HEADS * DSA_IDX_DIM;    // 8192 B: one query's tile at 64 heads
 constexpr int MAX_STAGES = 6;                          // per pipeline
 constexpr int OFF_PREFIX = 0;
 constexpr int OFF_SCAN = OFF_PREFIX + ((DSA_MAX_BATCH + 1) * 4 + 15) / 16 * 16;
@@ -133,6 +135,7 @@ __device__ __forceinline__ int seq_of_tile(const int* prefix, int B, int t) {
   return lo;
 }
 
+template <int HI>
 __global__ void __launch_bounds__(THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_q, IdxArgs a) {
@@ -166,16 +169,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   block_exclusive_scan(prefix, B, scan_tmp);
   const int maxq = *s_maxq;
   // Sequences with several queries (MTP verify) take their queries two at a
-  // time: one MMA with N = 128 (two 64-head query tiles side by side) into one
-  // of 2 accumulator slots of 128 columns, instead of one N = 64 MMA per query
-  // into 4 slots of 64.  Halves the MMAs and commits per tile.
+  // time: one MMA with N = 2 HI (two query tiles side by side) into one of 2
+  // accumulator slots, instead of one N = HI MMA per query into 4 slots.
+  // Halves the MMAs and commits per tile.
+  constexpr int QT = HI * DSA_IDX_DIM;             // one query's e4m3 tile (bytes)
   const int G = maxq >= 2 ? 2 : 1;
   const int nslots = SLOTS / G;
-  const uint32_t slot_cols = ACC_COLS * G;
+  const uint32_t slot_cols = HI * G;
   const int qtiles = (maxq + G - 1) / G * G;      // the last pair may read one tile past nq
   // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of qtiles tiles]
   const int pipe_bytes = (DATA_BYTES / PIPES) / 1024 * 1024;
-  const int stages = min(MAX_STAGES, (pipe_bytes - qtiles * Q_TILE) / KEY_TILE);
+  const int stages = min(MAX_STAGES, (pipe_bytes - qtiles * QT) / KEY_TILE);
 
   const int pipe = warp / WARPS_PER_PIPE;          // 0 / 1
   const int pw = warp % WARPS_PER_PIPE;            // role within the pipeline
@@ -243,9 +247,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             qphase ^= 1;
           }
           const int nq = seq_queries(a, b);
-          mbar_arrive_expect_tx(q_full, nq * Q_TILE);
+          mbar_arrive_expect_tx(q_full, nq * QT);
           for (int j = 0; j < nq; ++j)
-            tma_load_2d(qbuf + j * Q_TILE, &tmap_q, 0, (a.q_offsets[b] + j) * DSA_IDX_HEADS, q_full);
+            tma_load_2d(qbuf + j * QT, &tmap_q, 0, (a.q_offsets[b] + j) * HI, q_full);
           ++q_issued;
           cur_b = b;
         }
@@ -290,9 +294,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t slot = n % nslots;
           if (!mbar_wait(&acc_empty[slot], ((n / nslots) & 1) ^ 1, a.err)) { ok = false; break; }
           tc_fence_after();
-          // G consecutive 64-row query tiles form one 64G-row B operand (the
+          // G consecutive HI-row query tiles form one HI*G-row B operand (the
           // 128-byte swizzle atoms continue every 1024 bytes across tiles)
-          const uint32_t b_base = smem_u32(qbuf + j0 * Q_TILE);
+          const uint32_t b_base = smem_u32(qbuf + j0 * QT);
 #pragma unroll
           for (int kk = 0; kk < DSA_IDX_DIM / 32; ++kk) {
             mma_f8f6f4(tmem + slot * slot_cols, umma_desc_sw128(a_base + kk * 32, 1024, 16),
@@ -329,8 +333,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           q0 = a.q_offsets[b];
           const int64_t len = a.seq_offsets[b + 1] - a.seq_offsets[b];
           const int e = pw - 2;                  // 0..3
-          for (int x = e * 32 + lane; x < nq * DSA_IDX_HEADS; x += 128)
-            w_s[x] = __ldg(a.w + static_cast<size_t>(q0) * DSA_IDX_HEADS + x);
+          for (int x = e * 32 + lane; x < nq * HI; x += 128)
+            w_s[x] = __ldg(a.w + static_cast<size_t>(q0) * HI + x);
           if (e == 0 && lane < nq) {
             bool bad = false;
             vis_s[lane] = query_vis(a, q0 + lane, len, &bad);
@@ -342,7 +346,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           cur_b = b;
         }
         const int t = i - prefix[b];
-        // query pairs: both queries' 128 columns are read with a single wait
+        // query pairs: both queries' 2 HI columns are read with a single wait
         // (the wait covers every outstanding TMEM load, so reading the second
         // query later would cost a second full load latency)
         if (G == 2) {
@@ -351,12 +355,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool two = j0 + 1 < nq;
             if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
             tc_fence_after();
-            float v[2 * ACC_COLS];
+            float v[2 * HI];
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols;
-            tmem_ld32(taddr + 0, v + 0);
-            tmem_ld32(taddr + 32, v + 32);
-            tmem_ld32(taddr + 64, v + 64);      // past nq for an odd last query: not used
-            tmem_ld32(taddr + 96, v + 96);
+            // the second query's columns are past nq for an odd last query: not used
+#pragma unroll
+            for (int c = 0; c < 2 * HI / 32; ++c) tmem_ld32(taddr + 32 * c, v + 32 * c);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
@@ -364,21 +367,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int s = t * KT + row;
             float r0 = 0.f, r1 = 0.f;
             {
-              const float4* w0 = reinterpret_cast<const float4*>(w_s + j0 * DSA_IDX_HEADS);
-              const float4* w1 = reinterpret_cast<const float4*>(w_s + (two ? j0 + 1 : j0) * DSA_IDX_HEADS);
+              const float4* w0 = reinterpret_cast<const float4*>(w_s + j0 * HI);
+              const float4* w1 = reinterpret_cast<const float4*>(w_s + (two ? j0 + 1 : j0) * HI);
               float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
-              for (int h4 = 0; h4 < DSA_IDX_HEADS / 4; ++h4) {
+              for (int h4 = 0; h4 < HI / 4; ++h4) {
                 const float4 x = w0[h4];
                 const float4 y = w1[h4];
                 a0 = fmaf(x.x, fmaxf(v[4 * h4 + 0], 0.f), a0);
                 a1 = fmaf(x.y, fmaxf(v[4 * h4 + 1], 0.f), a1);
                 a0 = fmaf(x.z, fmaxf(v[4 * h4 + 2], 0.f), a0);
                 a1 = fmaf(x.w, fmaxf(v[4 * h4 + 3], 0.f), a1);
-                b0 = fmaf(y.x, fmaxf(v[64 + 4 * h4 + 0], 0.f), b0);
-                b1 = fmaf(y.y, fmaxf(v[64 + 4 * h4 + 1], 0.f), b1);
-                b0 = fmaf(y.z, fmaxf(v[64 + 4 * h4 + 2], 0.f), b0);
-                b1 = fmaf(y.w, fmaxf(v[64 + 4 * h4 + 3], 0.f), b1);
+                b0 = fmaf(y.x, fmaxf(v[HI + 4 * h4 + 0], 0.f), b0);
+                b1 = fmaf(y.y, fmaxf(v[HI + 4 * h4 + 1], 0.f), b1);
+                b0 = fmaf(y.z, fmaxf(v[HI + 4 * h4 + 2], 0.f), b0);
+                b1 = fmaf(y.w, fmaxf(v[HI + 4 * h4 + 3], 0.f), b1);
               }
               r0 = a0 + a1;
               r1 = b0 + b1;
@@ -395,13 +398,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
             tc_fence_after();
           }
-          float v[ACC_COLS];
+          float v[HI];
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols +
-                                 static_cast<uint32_t>(jj * ACC_COLS);
-          tmem_ld16(taddr + 0, v + 0);
-          tmem_ld16(taddr + 16, v + 16);
-          tmem_ld16(taddr + 32, v + 32);
-          tmem_ld16(taddr + 48, v + 48);
+                                 static_cast<uint32_t>(jj * HI);
+#pragma unroll
+          for (int c = 0; c < HI / 16; ++c) tmem_ld16(taddr + 16 * c, v + 16 * c);
           tmem_ld_wait();
           if (jj == G - 1 || j == nq - 1) {        // last query of the slot: release it
             tc_fence_before();
@@ -413,10 +414,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int vis = vis_s[j];
           const int s = t * KT + row;
           if (s < vis) {
-            const float4* wp = reinterpret_cast<const float4*>(w_s + j * DSA_IDX_HEADS);
+            const float4* wp = reinterpret_cast<const float4*>(w_s + j * HI);
             float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-            for (int h4 = 0; h4 < DSA_IDX_HEADS / 4; ++h4) {
+            for (int h4 = 0; h4 < HI / 4; ++h4) {
               const float4 ww = wp[h4];
               s0 = fmaf(ww.x, fmaxf(v[4 * h4 + 0], 0.f), s0);
               s1 = fmaf(ww.y, fmaxf(v[4 * h4 + 1], 0.f), s1);
@@ -440,32 +441,44 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace
 
+namespace {
+
+template <int HI>
+cudaError_t launch_indexer_h(const CUtensorMap& tk, const CUtensorMap& tq, const IdxArgs& args,
+                             cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<HI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  indexer_kernel<HI><<<device_sm_count(), THREADS, SMEM_BYTES, st>>>(tk, tq, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                           int first_only, float* scores, int ld, uint32_t* err,
+                           int idx_heads, int first_only, float* scores, int ld, uint32_t* err,
                            cudaStream_t st) {
   if (B <= 0 || Q <= 0 || total_keys <= 0) return cudaSuccess;
+  if (idx_heads != 64 && idx_heads != 32) return cudaErrorInvalidValue;
   CUtensorMap tk, tq;
   if (!encode_tiled_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, DSA_IDX_DIM,
                        static_cast<uint64_t>(total_keys), DSA_IDX_DIM, DSA_IDX_DIM, KT))
     return cudaErrorInvalidValue;
   if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_idx, DSA_IDX_DIM,
-                       static_cast<uint64_t>(Q) * DSA_IDX_HEADS, DSA_IDX_DIM, DSA_IDX_DIM,
-                       DSA_IDX_HEADS))
+                       static_cast<uint64_t>(Q) * idx_heads, DSA_IDX_DIM, DSA_IDX_DIM,
+                       static_cast<uint32_t>(idx_heads)))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
   IdxArgs args{w, seq_offsets, q_offsets, q_vis, scores, ld, B, first_only, err};
-  const int grid = device_sm_count();
-  indexer_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tk, tq, args);
-  return cudaGetLastError();
+  return idx_heads == 64 ? launch_indexer_h<64>(tk, tq, args, st)
+                         : launch_indexer_h<32>(tk, tq, args, st);
 }
 
 }  // namespace dsa

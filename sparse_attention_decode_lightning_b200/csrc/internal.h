@@ -36,7 +36,7 @@ int choose_splits(int Q, int topk, int requested);
 cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
-                           int first_only, float* scores, int ld, uint32_t* err,
+                           int idx_heads, int first_only, float* scores, int ld, uint32_t* err,
                            cudaStream_t st);
 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
@@ -50,12 +50,12 @@ cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,
 cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
                               const int32_t* page_table, int max_pages,
                               const int32_t* q_offsets, const int32_t* q_vis,
-                              const int32_t* idx, int B, int Q, int topk, float scale, int S,
+                              const int32_t* idx, int B, int Q, int H, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st, bool pdl);
 
-cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, float* out,
-                           float* lse, cudaStream_t st, bool pdl);
+cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
+                           float* out, float* lse, cudaStream_t st, bool pdl);
 
 // pdl = true: the kernel may start before the previous kernel on the stream
 // ends (programmatic dependent launch); it waits for it in pdl_wait().  Only

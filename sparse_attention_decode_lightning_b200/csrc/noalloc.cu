@@ -23,15 +23,15 @@ namespace dsa {
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int topk, float scale, int S,
-                                 float* out, float* lse, float* o_part, float* l_part,
+                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
+                                 int S, float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st, bool pdl);
 
 namespace {
 
 constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;   // 16 MiB per device
-constexpr size_t PART_O_BYTES = size_t(DSA_HEADS) * DSA_DIM_V * 4;   // one (query, split) output
-constexpr size_t PART_L_BYTES = size_t(DSA_HEADS) * 4;
+constexpr size_t PART_O_BYTES = size_t(DSA_DIM_V) * 4;   // one head of one (query, split) output
+constexpr size_t PART_L_BYTES = 4;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
@@ -67,7 +67,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
                                                     int num_pages, const int32_t* page_table,
                                                     int max_pages, const int32_t* q_offsets,
                                                     const int32_t* q_vis, const int32_t* idx,
-                                                    int B, int Q, int topk, float scale,
+                                                    int B, int Q, int heads, int topk, float scale,
                                                     int num_splits, float* out, float* lse,
                                                     void* stream) {
   if (!q || !kv_pool || !page_table || !q_offsets || !q_vis || !idx || !out || !lse)
@@ -76,24 +76,26 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
   if (B <= 0 || Q <= 0 || topk <= 0 || num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
   if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (heads != DSA_HEADS && heads != DSA_HEADS_GLM) return DSA_ERR_UNSUPPORTED;
   if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
   const int S = choose_splits(Q, topk, num_splits);
-  const size_t need = S > 1 ? static_cast<size_t>(Q) * S * (PART_O_BYTES + PART_L_BYTES) : 0;
+  const size_t parts = static_cast<size_t>(Q) * S * heads;      // (query, split, head) partials
+  const size_t need = S > 1 ? parts * (PART_O_BYTES + PART_L_BYTES) : 0;
   if (need > NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;   // beyond the fixed array
   dsa_status st = DSA_OK;
   uint8_t* scratch = static_cast<uint8_t*>(scratch_ptr(&st));
   if (!scratch) return st;
   float* o_part = reinterpret_cast<float*>(scratch);
-  float* l_part = reinterpret_cast<float*>(scratch + static_cast<size_t>(Q) * S * PART_O_BYTES);
+  float* l_part = reinterpret_cast<float*>(scratch + parts * PART_O_BYTES);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // every partial is written by the kernel before the merge reads it, so the
   // array needs no clearing; range violations are skipped but not reported
   if (launch_sparse_mla_tc(static_cast<const __nv_bfloat16*>(q),
                            static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_table,
-                           max_pages, q_offsets, q_vis, idx, B, Q, topk, scale, S, out, lse, o_part,
-                           l_part, nullptr, s, false) != cudaSuccess)
+                           max_pages, q_offsets, q_vis, idx, B, Q, heads, topk, scale, S, out, lse,
+                           o_part, l_part, nullptr, s, false) != cudaSuccess)
     return DSA_ERR_CUDA;
-  if (S > 1 && launch_combine(o_part, l_part, Q, S, out, lse, s, true) != cudaSuccess)
+  if (S > 1 && launch_combine(o_part, l_part, Q, S, heads, out, lse, s, true) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }

@@ -1,9 +1,16 @@
 // Sparse MLA decode on sm_100a tensor cores (absorbed MQA over the selected
 // latents).  Source: "大语言模型结构总览", section 2.2 (MLA in MQA mode over the
 // k = 2048 selected tokens; paged and non-paged kernels) and section 2.1 (one
-// 576-d latent per token = 512 kv rank + 64 RoPE; 128 heads).  Per head h:
+// 576-d latent per token = 512 kv rank + 64 RoPE; 128 heads; section 7.2
+// gives GLM-5.2's 64 heads over the same absorbed latent).  Per head h:
 //   z_j = scale * q[h,:] . C[j,:],  O[h] = sum_j softmax(z)_j C[j,:512],
 //   LSE[h] = ln sum_j exp(z_j).
+//
+// H = 128 or 64 heads.  The MMAs always have M = 128 (the tensor core's full
+// rate shape); with H = 64 the upper 64 TMEM lanes carry no head, and the
+// warps that own them (lane quarters 2 and 3) skip the exchange, the
+// softmax and the output, keeping only their barrier arrivals, so the
+// partial-score exchange moves half the bytes.
 //
 // Work unit: (query, split) on a cluster of two CTAs that divide the
 // contraction dims and the output:
@@ -137,6 +144,7 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+template <int NH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_o, MlaTcArgs a) {
@@ -196,8 +204,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_holder;
   if (tid == 0) {
     tma_prefetch_desc(&tmap_q);
-    mbar_arrive_expect_tx(q_ready, QROPE_BYTES);
-    tma_load_2d(qrope, &tmap_q, 8 * 64, q * DSA_HEADS, q_ready);
+    mbar_arrive_expect_tx(q_ready, NH * 128);
+    tma_load_2d(qrope, &tmap_q, 8 * 64, q * NH, q_ready);
   }
   // the selected indices (and the error word) come from the kernel before
   pdl_wait();
@@ -320,15 +328,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool live = quarter * 32 < NH;         // this warp's lanes carry heads
     const uint32_t peer = rank ^ 1u;
     const uint32_t peer_x = map_to_rank(smem_u32(xb), peer);
     const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
     // partial scores are exchanged by push: each CTA stores its partial into
     // the peer's shared memory with st.async and reads the peer's from its own
-    if (g == 0) {
+    if (g == 0 && live) {
       // this CTA's 256 latent query dims of head h -> tensor memory (bf16 pairs)
       const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + (static_cast<size_t>(q) * DSA_HEADS + h) * DSA_DIM + (rank ? 256 : 0));
+          a.q + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float w[32];
@@ -344,6 +353,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       tmem_st_wait();
       tc_fence_before();
+    }
+    if (g == 0) {
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
@@ -352,6 +363,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int t = 0; t < ntiles && ok; ++t) {
       const int sb = t & 1;
       const uint32_t ph = (t >> 1) & 1;
+      if (!live) {
+        // no heads in these lanes: only the tile-max barrier and the P arrival
+        named_barrier(1, 32 * SMX_WARPS);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
+        continue;
+      }
       const int j = t * NR + 32 * g + lane;
       const uint32_t vm = __ballot_sync(0xffffffffu, j < nrows && crd[j] >= 0);
       if (!(ok = warp_wait(&s_full[sb], ph, a.err))) break;
@@ -367,7 +385,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // three words, a quarter fewer bytes over the ~16 B/cycle DSMEM link.
       // Slot layout [16-byte chunk k][warpgroup][head]: a warp's chunk k is
       // 512 contiguous bytes, bank-conflict free; the peer fills mine alike.
-      if (gt == 0) mbar_arrive_expect_tx(&x_full[sb], X_BYTES);
+      if (g == 0 && quarter == 0 && lane == 0)
+        mbar_arrive_expect_tx(&x_full[sb], static_cast<uint32_t>(NH) * (NR * 3));
       uint32_t u[32];
 #pragma unroll
       for (int r = 0; r < 32; ++r) u[r] = round_to_24bit(z[r]);
@@ -503,18 +522,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     lsum[g * DSA_HEADS + h] = l;
     named_barrier(1, 32 * SMX_WARPS);
     const float lt = lsum[h] + lsum[DSA_HEADS + h];
-    const bool have = ok && ntiles > 0 && warp_wait(o_final, 0, a.err);
+    const bool have = ok && live && ntiles > 0 && warp_wait(o_final, 0, a.err);
     if (have) tc_fence_after();
     const float inv = lt > 0.f ? 1.f / lt : 0.f;
     // O / l leaves through shared memory: warpgroup g fills four boxes of
     // [128 heads x 32 fp32] (its columns [128g, 128g+128) of this CTA's 256)
     // in the 128-byte swizzle, then one thread stores them with TMA.  The
     // stage ring and the exchange slots are idle once the last PV is done.
-    float* lrow = a.S == 1 ? a.lse + static_cast<size_t>(q) * DSA_HEADS + h
-                           : a.l_part + (static_cast<size_t>(q) * a.S + split) * DSA_HEADS + h;
-    const int orow0 = (a.S == 1 ? q : q * a.S + split) * DSA_HEADS;
+    float* lrow = a.S == 1 ? a.lse + static_cast<size_t>(q) * NH + h
+                           : a.l_part + (static_cast<size_t>(q) * a.S + split) * NH + h;
+    const int orow0 = (a.S == 1 ? q : q * a.S + split) * NH;
     uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
-    for (int c = 0; c < 128 / 32; ++c) {
+    for (int c = 0; c < 128 / 32 && live; ++c) {
       float o[32];
       if (have) {
         tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
@@ -538,7 +557,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       bulk_commit_group();
       bulk_wait_all_read();   // the shared-memory boxes may be released; the grid's end publishes O
     }
-    if (rank == 0 && g == 0) *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
+    if (rank == 0 && g == 0 && live)
+      *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
     (void)gt;
   }
 
@@ -556,29 +576,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int topk, float scale, int S,
-                                 float* out, float* lse, float* o_part, float* l_part,
+                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
+                                 int S, float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
+  if (H != 128 && H != 64) return cudaErrorInvalidValue;
+  // RoPE query dims: boxes of H heads x 64 bf16 (rows past H in shared memory
+  // are never read into a head's result)
   CUtensorMap tq;
   if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, DSA_DIM,
-                       static_cast<uint64_t>(Q) * DSA_HEADS, DSA_DIM * 2, 64, DSA_HEADS))
+                       static_cast<uint64_t>(Q) * H, DSA_DIM * 2, 64, static_cast<uint32_t>(H)))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
+  static bool attr_set[2][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_mla_tc_kernel,
+  const int hi = H == 128 ? 0 : 1;
+  if (dev >= 0 && dev < 64 && !attr_set[hi][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(H == 128 ? sparse_mla_tc_kernel<128> : sparse_mla_tc_kernel<64>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[hi][dev] = true;
   }
-  // output boxes of 128 heads x 32 fp32 into O [Q, 128, 512] (S = 1) or the
-  // split partials [Q, S, 128, 512]
+  // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
+  // split partials [Q, S, H, 512]
   CUtensorMap to;
   if (!encode_tiled_2d(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S == 1 ? out : o_part, DSA_DIM_V,
-                       static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * DSA_HEADS, DSA_DIM_V * 4, 32,
-                       DSA_HEADS))
+                       static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4, 32,
+                       static_cast<uint32_t>(H)))
     return cudaErrorInvalidValue;
   MlaTcArgs a{q, pool, page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
@@ -592,7 +616,8 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel, tq, to, a);
+  return H == 128 ? cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<128>, tq, to, a)
+                  : cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<64>, tq, to, a);
 }
 
 }  // namespace dsa

@@ -27,11 +27,10 @@ import torch
 from .workloads import Workload
 
 PAGE = 64          # latent-cache page size (tokens)
-H = 128            # MLA heads
 D = 576            # latent row: 512 latent + 64 rope
 DV = 512           # value dims
-HI = 64            # indexer heads
 DI = 128           # indexer head dim
+# head counts come from the workload (128 / 64 DeepSeek-V3.2, 64 / 32 GLM-5.2)
 FP8_MAX = 448.0
 
 
@@ -76,6 +75,8 @@ class DSAInputs:
     topk: int
     scale: float
     num_splits: int
+    heads: int                      # MLA heads
+    idx_heads: int                  # indexer heads
     n_layers: int
     index_share: int
     mtp_index_share: bool
@@ -150,8 +151,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", layers_to_make: Option
     indexer = []
     for gi in range(n_groups):
         indexer.append({
-            "q_idx": _randn_e4m3((Q, HI, DI), _gen(seed, f"q_idx{gi}", dev), dev),
-            "w": torch.randn((Q, HI), generator=_gen(seed, f"w{gi}", dev), device=dev,
+            "q_idx": _randn_e4m3((Q, w.idx_heads, DI), _gen(seed, f"q_idx{gi}", dev), dev),
+            "w": torch.randn((Q, w.idx_heads), generator=_gen(seed, f"w{gi}", dev), device=dev,
                              dtype=torch.float32) / 8.0,
             "k_idx": _randn_e4m3((total_keys, DI), _gen(seed, f"k_idx{gi}", dev), dev),
         })
@@ -159,12 +160,13 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", layers_to_make: Option
     layers = []
     for li in range(n_make):
         layers.append({
-            "q": _randn_bf16((Q, H, D), _gen(seed, f"q{li}", dev), dev),
+            "q": _randn_bf16((Q, w.heads, D), _gen(seed, f"q{li}", dev), dev),
             "pool": _randn_bf16((num_pages, PAGE, D), _gen(seed, f"pool{li}", dev), dev),
         })
     return DSAInputs(
         workload=w, seed=seed, device=str(dev), B=B, T=T, Q=Q, topk=w.topk,
-        scale=1.0 / math.sqrt(192.0), num_splits=w.num_splits, n_layers=w.n_layers,
+        scale=1.0 / math.sqrt(float(w.qk_head_dim)), num_splits=w.num_splits,
+        heads=w.heads, idx_heads=w.idx_heads, n_layers=w.n_layers,
         index_share=w.index_share, mtp_index_share=w.mtp_index_share,
         seq_lens=seq_lens, seq_offsets=torch.from_numpy(seq_offsets).to(dev),
         q_offsets=torch.from_numpy(q_offsets).to(dev), q_vis=torch.from_numpy(q_vis).to(dev),

@@ -1,11 +1,13 @@
-"""The five DSA decode workloads, named by what they are and their sizes.
+"""The DSA decode workloads, named by what they are and their sizes.
 
 Shapes follow the DeepSeek-V3.2 DSA description (DeepSeek-V3.2 section of the
 2026 architecture survey page: lightning indexer with 64 heads of dim 128 in
 FP8, top-k = 2048 over prior tokens, MLA in MQA mode with a 512-d latent plus a
 64-d RoPE part, 128 heads) and the GLM-5.2 IndexShare / MTP descriptions
 (GLM-5.2 section of the same survey; MTP section of the GLM-5.2 inference
-page).
+page).  The glm52_* workloads take GLM-5.2's shapes from the same survey's
+GLM-5.2 section: 64 MLA heads with qk head dim 192 + 64 RoPE (softmax scale
+1/sqrt(256)) over the same 512 + 64 latent, and a 32-head FP8 indexer.
 """
 from dataclasses import dataclass, field
 from typing import Optional, Tuple
@@ -25,6 +27,9 @@ class Workload:
     num_splits: int = 0         # 0 = let the library choose; >0 = split-K partitions
     paged_permuted: bool = True  # pages of 64 randomly permuted in the pool
     topk: int = 2048
+    heads: int = 128            # MLA heads (GLM-5.2: 64)
+    idx_heads: int = 64         # indexer heads (GLM-5.2: 32)
+    qk_head_dim: int = 192      # softmax scale 1/sqrt(qk_head_dim) (GLM-5.2: 192 + 64 = 256)
     note: str = ""
 
     @property
@@ -49,6 +54,16 @@ WORKLOADS = {
                  note="MTP verify with position 0's top-k reused by the drafts"),
         Workload("decode_b4_ctx1m_split16", B=4, T=1, L=1048576, num_splits=16,
                  note="1M-context decode, 16-way split-K plus LSE combine"),
+        Workload("glm52_decode_b32_ctx128k", B=32, T=1, L=131072,
+                 heads=64, idx_heads=32, qk_head_dim=256,
+                 note="GLM-5.2 shapes: batch-32 decode at 128K"),
+        Workload("glm52_indexshare4_b64_ctx16k_128k", B=64, T=1, L=131072,
+                 L_range=(16384, 131072), n_layers=4, index_share=4,
+                 heads=64, idx_heads=32, qk_head_dim=256,
+                 note="GLM-5.2 shapes with its IndexShare: one indexer per 4 layers"),
+        Workload("glm52_decode_b4_ctx1m_split16", B=4, T=1, L=1048576, num_splits=16,
+                 heads=64, idx_heads=32, qk_head_dim=256,
+                 note="GLM-5.2 shapes at its 1M context, 16-way split-K"),
     ]
 }
 

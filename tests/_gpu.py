@@ -11,8 +11,8 @@ def run_decode_step(inp, num_splits=None, ws=None):
     qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
     wl = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
     kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
-    outs = [torch.empty(Q, 128, 512, dtype=torch.float32, device=DEV) for _ in range(n)]
-    lses = [torch.empty(Q, 128, dtype=torch.float32, device=DEV) for _ in range(n)]
+    outs = [torch.empty(Q, inp.heads, 512, dtype=torch.float32, device=DEV) for _ in range(n)]
+    lses = [torch.empty(Q, inp.heads, dtype=torch.float32, device=DEV) for _ in range(n)]
     ng = (n + G - 1) // G
     idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=DEV)
     S = inp.num_splits if num_splits is None else num_splits

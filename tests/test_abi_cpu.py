@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_library_loads_and_reports_version_and_status_names():
     L = dsa.lib()
-    assert L.dsa_version() == 100
+    assert L.dsa_version() == 200
     for code, name in dsa.STATUS.items():
         assert dsa.dsa_status_string(code) == name
     assert dsa.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
@@ -80,36 +80,46 @@ def test_host_checks_reject_bad_arguments_without_a_device():
     fake = P(1 << 20)          # never dereferenced: checks fail first
     null = P(0)
     # null pointers
-    assert L.dsa_indexer_topk(null, fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048, 0, fake,
+    assert L.dsa_indexer_topk(null, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
                               null, fake, 1 << 30, null) == 1
     # top-k above the supported maximum
-    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 100, 4096, 0, fake,
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 4096, 0, fake,
                               null, fake, 1 << 30, null) == 2
     # more queries than sequences allow
-    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 9, 100, 2048, 0, fake,
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 9, 64, 100, 2048, 0, fake,
                               null, fake, 1 << 30, null) == 2
     # misaligned pointer
-    assert L.dsa_indexer_topk(P((1 << 20) + 4), fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048,
-                              0, fake, null, fake, 1 << 30, null) == 1
+    assert L.dsa_indexer_topk(P((1 << 20) + 4), fake, fake, 100, fake, fake, fake, 1, 1, 64, 100,
+                              2048, 0, fake, null, fake, 1 << 30, null) == 1
+    # indexer head counts other than 64 (DeepSeek-V3.2) and 32 (GLM-5.2)
+    for hi, want in ((48, 2), (128, 2), (0, 2)):
+        assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, hi, 100, 2048, 0,
+                                  fake, null, fake, 1 << 30, null) == want
     # workspace too small
-    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 100, 2048, 0, fake,
+    assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
                               null, fake, 16, null) == 6
     # sparse MLA: bad scale, bad split count, null page table
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.0), 0, fake, fake, fake, 1 << 30, null) == 1
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.07), 33, fake, fake, fake, 1 << 30, null) == 2
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, null, 4, fake, fake, fake, 1, 1, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, null, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30, null) == 1
+    # MLA head counts other than 128 (DeepSeek-V3.2) and 64 (GLM-5.2)
+    for h in (32, 96, 256):
+        assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, h, 2048,
+                                       ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30,
+                                       null) == 2
+        assert L.dsa_lse_combine(fake, fake, 1, 2, h, fake, fake, null) == 2
     # decode step: no layers, zero share group
     PP = ctypes.POINTER(ctypes.c_void_p)
     arr = (ctypes.c_void_p * 1)(1 << 20)
-    assert L.dsa_decode_step(0, 1, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 100, 2048, arr,
-                             arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake, fake,
-                             1 << 30, null) == 1
-    assert L.dsa_decode_step(1, 0, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 100, 2048, arr,
-                             arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake, fake,
-                             1 << 30, null) == 1
+    assert L.dsa_decode_step(0, 1, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 128, 64, 100,
+                             2048, arr, arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
+                             fake, 1 << 30, null) == 1
+    assert L.dsa_decode_step(1, 0, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 128, 64, 100,
+                             2048, arr, arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
+                             fake, 1 << 30, null) == 1
     # check_error without a workspace
     assert L.dsa_check_error(null, null) == 1
 

@@ -47,15 +47,17 @@ def _same(a_outs, a_lses, a_idx, b_outs, b_lses, b_idx):
 
 
 @pytest.mark.parametrize("name,over", [("decode_b32_ctx128k", dict(B=4, L=9000)),
-                                       ("indexshare4_b64_ctx16k_128k", dict(B=3, L_range=(1500, 7000)))])
+                                       ("indexshare4_b64_ctx16k_128k", dict(B=3, L_range=(1500, 7000))),
+                                       ("glm52_indexshare4_b64_ctx16k_128k",
+                                        dict(B=3, L_range=(1500, 7000)))])
 def test_captured_step_matches_eager_and_reads_inputs_at_replay(name, over):
     inp = make_inputs(get_workload(name, **over), seed=3, device=DEV)
     Q, n = inp.Q, inp.n_layers
     ng = (n + inp.index_share - 1) // inp.index_share
 
     def buffers():
-        return ([torch.empty(Q, 128, 512, device=DEV) for _ in range(n)],
-                [torch.empty(Q, 128, device=DEV) for _ in range(n)],
+        return ([torch.empty(Q, inp.heads, 512, device=DEV) for _ in range(n)],
+                [torch.empty(Q, inp.heads, device=DEV) for _ in range(n)],
                 torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=DEV))
 
     ws = dsa.workspace(Q, inp.max_len, inp.topk, inp.num_splits, device=DEV)

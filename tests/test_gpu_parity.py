@@ -23,8 +23,10 @@ def _e4m3(x: torch.Tensor) -> torch.Tensor:
 
 
 # ------------------------------------------------------------------ indexer
-@pytest.mark.parametrize("T,first_only", [(1, False), (8, False), (8, True)])
-def test_indexer_scores_match_oracle(T, first_only):
+# indexer heads: 64 (DeepSeek-V3.2) and 32 (GLM-5.2)
+@pytest.mark.parametrize("T,first_only,hi", [(1, False, 64), (8, False, 64), (8, True, 64),
+                                             (1, False, 32), (8, False, 32), (8, True, 32)])
+def test_indexer_scores_match_oracle(T, first_only, hi):
     torch.manual_seed(0)
     lens = [1000, 300, 129, 4096 + 77]
     B = len(lens)
@@ -34,8 +36,8 @@ def test_indexer_scores_match_oracle(T, first_only):
     vis = torch.tensor([lens[b] - (T - 1 - t) for b in range(B) for t in range(T)],
                        dtype=torch.int32, device=DEV)
     k = _e4m3(torch.randn(int(sum(lens)), 128, device=DEV))
-    qi = _e4m3(torch.randn(Q, 64, 128, device=DEV))
-    w = torch.randn(Q, 64, device=DEV) / 8
+    qi = _e4m3(torch.randn(Q, hi, 128, device=DEV))
+    w = torch.randn(Q, hi, device=DEV) / 8
     ld = max(lens) + 60
     ld += (-ld) % 4
     scores = torch.full((Q, ld), float("nan"), device=DEV)
@@ -54,10 +56,10 @@ def test_indexer_scores_match_oracle(T, first_only):
             continue
         keys = kb[so[b]:so[b] + vv[q]]
         ref = O.indexer_scores(qb[q], wb[q], keys)
-        # fp32 summation bound for the 64-head reduction (products are exact)
+        # fp32 summation bound for the hi-head reduction (products are exact)
         d = O.e4m3_decode(keys) @ O.e4m3_decode(qb[q]).T
         mag = np.abs(np.maximum(d, 0) * wb[q].astype(np.float64)).sum(1)
-        tol = 64 * 2.0 ** -24 * mag + 1e-30
+        tol = hi * 2.0 ** -24 * mag + 1e-30
         got = sc[q, :vv[q]].astype(np.float64)
         bad = np.abs(got - ref) > tol
         assert not bad.any(), (q, np.flatnonzero(bad)[:5], got[bad][:5], ref[bad][:5])
@@ -122,9 +124,11 @@ def test_topk_select_exact_on_fixed_scores(case):
 
 
 # ------------------------------------------------------------------ sparse MLA
-@pytest.mark.parametrize("S", [1, 3, 16])
-def test_sparse_mla_matches_oracle(S):
-    w = get_workload("decode_b32_ctx128k", B=3, L=1500, topk=2048)
+@pytest.mark.parametrize("S,name", [(1, "decode_b32_ctx128k"), (3, "decode_b32_ctx128k"),
+                                    (16, "decode_b32_ctx128k"), (1, "glm52_decode_b32_ctx128k"),
+                                    (3, "glm52_decode_b32_ctx128k")])
+def test_sparse_mla_matches_oracle(S, name):
+    w = get_workload(name, B=3, L=1500, topk=2048)
     inp = make_inputs(w, seed=11, device=DEV)
     Q = inp.Q
     g = torch.Generator(device="cpu").manual_seed(5)
@@ -133,8 +137,8 @@ def test_sparse_mla_matches_oracle(S):
         n = [1500, 700, 1][q]
         idx[q, :n] = torch.randperm(1500, generator=g)[:n].to(torch.int32)
     idx = idx.to(DEV)
-    out = torch.empty(Q, 128, 512, device=DEV)
-    lse = torch.empty(Q, 128, device=DEV)
+    out = torch.empty(Q, inp.heads, 512, device=DEV)
+    lse = torch.empty(Q, inp.heads, device=DEV)
     ws = dsa.workspace(Q, 1, 2048, S)
     dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], inp.page_table,
                               inp.q_offsets, inp.q_vis, idx, inp.B, inp.scale, out, lse, ws,
@@ -147,11 +151,13 @@ def test_sparse_mla_matches_oracle(S):
         check_attention(out[q].cpu().numpy(), lse[q].cpu().numpy(), o_ref, l_ref)
 
 
-def test_sparse_mla_all_padding_gives_zero_and_neg_inf():
-    inp = make_inputs(get_workload("decode_b1_ctx8k", L=256), seed=2, device=DEV)
+@pytest.mark.parametrize("heads,idx_heads,qk", [(128, 64, 192), (64, 32, 256)])
+def test_sparse_mla_all_padding_gives_zero_and_neg_inf(heads, idx_heads, qk):
+    inp = make_inputs(get_workload("decode_b1_ctx8k", L=256, heads=heads, idx_heads=idx_heads,
+                                   qk_head_dim=qk), seed=2, device=DEV)
     idx = torch.full((1, 2048), -1, dtype=torch.int32, device=DEV)
-    out = torch.full((1, 128, 512), 7.0, device=DEV)
-    lse = torch.zeros(1, 128, device=DEV)
+    out = torch.full((1, heads, 512), 7.0, device=DEV)
+    lse = torch.zeros(1, heads, device=DEV)
     for S in (1, 4):
         ws = dsa.workspace(1, 1, 2048, S)
         dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], inp.layers[0]["pool"], inp.page_table,
@@ -161,15 +167,16 @@ def test_sparse_mla_all_padding_gives_zero_and_neg_inf():
         assert (out == 0).all() and torch.isneginf(lse).all()
 
 
-def test_lse_combine_matches_oracle():
+@pytest.mark.parametrize("H", [128, 64])
+def test_lse_combine_matches_oracle(H):
     rng = np.random.default_rng(3)
     Q, S = 3, 5
-    o = rng.standard_normal((Q, S, 128, 512)).astype(np.float32)
-    l = (rng.standard_normal((Q, S, 128)) * 4).astype(np.float32)
+    o = rng.standard_normal((Q, S, H, 512)).astype(np.float32)
+    l = (rng.standard_normal((Q, S, H)) * 4).astype(np.float32)
     l[0, 2] = -np.inf
     l[1, :, :7] = -np.inf
-    out = torch.empty(Q, 128, 512, device=DEV)
-    lse = torch.empty(Q, 128, device=DEV)
+    out = torch.empty(Q, H, 512, device=DEV)
+    lse = torch.empty(Q, H, device=DEV)
     dsa.dsa_lse_combine(torch.from_numpy(o).to(DEV), torch.from_numpy(l).to(DEV), out, lse)
     torch.cuda.synchronize()
     for q in range(Q):
@@ -188,6 +195,9 @@ SMALL = {
     "mtp_verify_b16_t8_ctx128k": dict(B=2, L=5000),
     "mtp_verify_reuse_b16_t8_ctx128k": dict(B=2, L=5000),
     "decode_b4_ctx1m_split16": dict(B=2, L=40000),
+    "glm52_decode_b32_ctx128k": dict(B=4, L=9000),
+    "glm52_indexshare4_b64_ctx16k_128k": dict(B=5, L_range=(1500, 7000)),
+    "glm52_decode_b4_ctx1m_split16": dict(B=2, L=40000),
 }
 
 

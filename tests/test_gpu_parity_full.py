@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 FULL = ["decode_b32_ctx128k", "indexshare4_b64_ctx16k_128k", "mtp_verify_b16_t8_ctx128k",
-        "mtp_verify_reuse_b16_t8_ctx128k", "decode_b4_ctx1m_split16"]
+        "mtp_verify_reuse_b16_t8_ctx128k", "decode_b4_ctx1m_split16", "glm52_decode_b32_ctx128k",
+        "glm52_indexshare4_b64_ctx16k_128k", "glm52_decode_b4_ctx1m_split16"]
 
 
 def _check_index_properties(idx: torch.Tensor, vis: torch.Tensor, topk: int):

@@ -59,26 +59,35 @@ def test_bf16_decode_matches_torch():
     assert np.array_equal(O.bf16_decode(bits), ref)
 
 
+# Model shapes: DeepSeek-V3.2 (128 MLA heads, 64 indexer heads, qk head dim
+# 192) and GLM-5.2 (64 MLA heads, 32 indexer heads, qk head dim 256; "大语言
+# 模型结构总览" section 7.2).
+IDX_HEADS = [64, 32]
+MLA_SHAPES = [(128, 1 / math.sqrt(192)), (64, 1 / math.sqrt(256))]
+
+
 # ---------------------------------------------------------------- indexer
-def test_indexer_brute_force_loops():
-    q = _e4m3_bytes(RNG.standard_normal((64, 128)))
+@pytest.mark.parametrize("hi", IDX_HEADS)
+def test_indexer_brute_force_loops(hi):
+    q = _e4m3_bytes(RNG.standard_normal((hi, 128)))
     k = _e4m3_bytes(RNG.standard_normal((5, 128)))
-    w = (RNG.standard_normal(64) / 8).astype(np.float32)
+    w = (RNG.standard_normal(hi) / 8).astype(np.float32)
     got = O.indexer_scores(q, w, k)
     tab = O.e4m3_table()
     for s in range(5):
         acc = 0.0
-        for h in range(64):
+        for h in range(hi):
             d = sum(float(tab[q[h, i]]) * float(tab[k[s, i]]) for i in range(128))
             acc += float(w[h]) * (d if d > 0 else 0.0)
         assert abs(got[s] - acc) <= 1e-12 * max(1.0, abs(acc))
 
 
-def test_indexer_one_hot_keys_closed_form():
+@pytest.mark.parametrize("hi", IDX_HEADS)
+def test_indexer_one_hot_keys_closed_form(hi):
     # K[s] = e_s (a single 1.0 at dim s): q_h . K[s] = q_h[s], so
     # I[s] = sum_h w_h * max(0, q_h[s]).
-    q = _e4m3_bytes(RNG.standard_normal((64, 128)))
-    w = (RNG.standard_normal(64) / 8).astype(np.float32)
+    q = _e4m3_bytes(RNG.standard_normal((hi, 128)))
+    w = (RNG.standard_normal(hi) / 8).astype(np.float32)
     keys = np.zeros((128, 128), dtype=np.uint8)
     keys[np.arange(128), np.arange(128)] = 0x38          # e4m3 1.0
     qf = O.e4m3_decode(q)
@@ -86,11 +95,12 @@ def test_indexer_one_hot_keys_closed_form():
     assert np.allclose(O.indexer_scores(q, w, keys), want, rtol=0, atol=1e-12)
 
 
-def test_indexer_relu_sign_identity():
+@pytest.mark.parametrize("hi", IDX_HEADS)
+def test_indexer_relu_sign_identity(hi):
     # I(q,K) - I(q,-K) = sum_h w_h (q_h . K): catches a dropped or mirrored ReLU.
-    q = _e4m3_bytes(RNG.standard_normal((64, 128)))
+    q = _e4m3_bytes(RNG.standard_normal((hi, 128)))
     k = _e4m3_bytes(RNG.standard_normal((33, 128)))
-    w = (RNG.standard_normal(64) / 8).astype(np.float32)
+    w = (RNG.standard_normal(hi) / 8).astype(np.float32)
     k_neg = k ^ 0x80
     lhs = O.indexer_scores(q, w, k) - O.indexer_scores(q, w, k_neg)
     qw = O.e4m3_decode(q).T @ w.astype(np.float64)              # [128]
@@ -138,12 +148,12 @@ def _rows(n, dtype_bits=True):
     return O.bf16_decode(_bf16_bits(RNG.standard_normal((n, 576))))
 
 
-def test_mla_k_ge_L_equals_library_dense_attention():
+@pytest.mark.parametrize("nh,scale", MLA_SHAPES)
+def test_mla_k_ge_L_equals_library_dense_attention(nh, scale):
     # with k >= L the selector keeps every token, so DSA is dense MLA; compare
     # with torch's scaled_dot_product_attention in float64 (value = first 512).
     rows = _rows(37)
-    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((128, 576))))
-    scale = 1 / math.sqrt(192)
+    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((nh, 576))))
     sc = RNG.standard_normal(37)
     idx = O.topk_select(sc, 2048)
     sel = idx[idx >= 0]
@@ -158,26 +168,28 @@ def test_mla_k_ge_L_equals_library_dense_attention():
     assert np.allclose(lse, ref_lse, rtol=1e-13, atol=1e-12)
 
 
-def test_mla_softmax_weights_sum_to_one():
+@pytest.mark.parametrize("nh,scale", MLA_SHAPES)
+def test_mla_softmax_weights_sum_to_one(nh, scale):
     # value dims all equal to 1 -> O = sum_j p_j = 1 for every head and dim
     rows = _rows(50)
     rows[:, :512] = 1.0
-    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((128, 576)) * 3))
-    o, _ = O.sparse_mla(q, rows, 1 / math.sqrt(192))
+    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((nh, 576)) * 3))
+    o, _ = O.sparse_mla(q, rows, scale)
+    assert o.shape == (nh, 512)
     assert np.allclose(o, 1.0, rtol=0, atol=1e-12)
 
 
-def test_mla_closed_forms():
-    scale = 1 / math.sqrt(192)
-    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((128, 576))))
+@pytest.mark.parametrize("nh,scale", MLA_SHAPES)
+def test_mla_closed_forms(nh, scale):
+    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((nh, 576))))
     r = _rows(1)
     # one row: O = its latent, LSE = its score
     o, lse = O.sparse_mla(q, r, scale)
-    assert np.allclose(o, np.broadcast_to(r[0, :512], (128, 512)), atol=1e-12)
+    assert np.allclose(o, np.broadcast_to(r[0, :512], (nh, 512)), atol=1e-12)
     assert np.allclose(lse, scale * (q @ r[0]), atol=1e-12)
     # n identical rows: O = the row, LSE = s + ln n
     o, lse = O.sparse_mla(q, np.repeat(r, 9, axis=0), scale)
-    assert np.allclose(o, np.broadcast_to(r[0, :512], (128, 512)), atol=1e-12)
+    assert np.allclose(o, np.broadcast_to(r[0, :512], (nh, 512)), atol=1e-12)
     assert np.allclose(lse, scale * (q @ r[0]) + math.log(9), atol=1e-12)
     # two rows: O = sigmoid(s1 - s2) c1 + sigmoid(s2 - s1) c2
     r2 = _rows(2)
@@ -339,10 +351,12 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     caught = []
     for name, fn, attr, pins in [
-        ("relu", no_relu, "indexer_scores", [test_indexer_relu_sign_identity, test_indexer_one_hot_keys_closed_form]),
+        ("relu", no_relu, "indexer_scores", [lambda: test_indexer_relu_sign_identity(32),
+                                             lambda: test_indexer_one_hot_keys_closed_form(64)]),
         ("ties", ties_high, "topk_select", [lambda: test_topk_equals_full_sort_with_ties(7)]),
-        ("scale", no_scale, "sparse_mla", [test_mla_k_ge_L_equals_library_dense_attention]),
-        ("value", value_from_rope_end, "sparse_mla", [test_mla_closed_forms]),
+        ("scale", no_scale, "sparse_mla", [lambda: test_mla_k_ge_L_equals_library_dense_attention(
+            *MLA_SHAPES[1])]),
+        ("value", value_from_rope_end, "sparse_mla", [lambda: test_mla_closed_forms(*MLA_SHAPES[0])]),
     ]:
         monkeypatch.setattr(O, attr, fn)
         failed = False

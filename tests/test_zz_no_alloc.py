@@ -24,7 +24,8 @@ def _call_noalloc(inp, layer, idx, out, lse, num_splits):
         ctypes.c_void_p(inp.layers[layer]["pool"].data_ptr()), inp.num_pages,
         ctypes.c_void_p(inp.page_table.data_ptr()), inp.max_pages,
         ctypes.c_void_p(inp.q_offsets.data_ptr()), ctypes.c_void_p(inp.q_vis.data_ptr()),
-        ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, idx.shape[1], ctypes.c_float(inp.scale),
+        ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, inp.layers[layer]["q"].shape[1], idx.shape[1],
+        ctypes.c_float(inp.scale),
         num_splits, ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, dsa.dsa_status_string(st)
@@ -70,6 +71,6 @@ def test_noalloc_rejects_requests_beyond_its_array():
         ctypes.c_void_p(inp.layers[0]["q"].data_ptr()), ctypes.c_void_p(inp.layers[0]["pool"].data_ptr()),
         inp.num_pages, ctypes.c_void_p(inp.page_table.data_ptr()), inp.max_pages,
         ctypes.c_void_p(inp.q_offsets.data_ptr()), ctypes.c_void_p(inp.q_vis.data_ptr()),
-        ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, 2048, ctypes.c_float(inp.scale), 2,
+        ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, 128, 2048, ctypes.c_float(inp.scale), 2,
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), None)
     assert st == 2          # 32 queries x 2 splits > 63 partials: DSA_ERR_UNSUPPORTED
