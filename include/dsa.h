@@ -68,7 +68,8 @@
 extern "C" {
 #endif
 
-#define DSA_PAGE_SIZE 64        /* latent-cache page (tokens) */
+#define DSA_PAGE_SIZE 64        /* latent-cache page (tokens) of the built-in workloads */
+#define DSA_TIER_PAGE 16        /* tokens per slot of the two-tier (HiSparse) cache */
 #define DSA_HEADS 128           /* MLA query heads (DeepSeek-V3.2) */
 #define DSA_HEADS_GLM 64        /* MLA query heads (GLM-5.2) */
 #define DSA_DIM 576             /* latent row: 512 kv-rank + 64 RoPE */
@@ -175,10 +176,13 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
  *   q          bf16 [Q,heads,576]  absorbed queries (512 latent + 64 RoPE)
  *   heads      128 (DeepSeek-V3.2) or 64 (GLM-5.2); 64 heads run on the same
  *              128-row tensor-core tiles with the upper rows unused
- *   kv_pool    bf16 [num_pages,64,576]  paged latent cache shared by all heads
+ *   kv_pool    bf16 [num_pages,page_size,576]  paged latent cache shared by all heads
+ *   page_size  tokens per page: a power of two from 1 to 1024 with
+ *              num_pages*page_size < 2^31 (64 for the built-in workloads; 16,
+ *              DSA_TIER_PAGE, for a device buffer of the two-tier cache below)
  *   page_table int32 [B,max_pages]: page of token s of sequence b is
- *              page_table[b*max_pages + s/64], row s%64 in that page.  A
- *              non-paged cache is the identity table.
+ *              page_table[b*max_pages + s/page_size], row s%page_size in that
+ *              page.  A non-paged cache is the identity table.
  *   idx        int32 [Q,topk]: token positions (any order), -1 = skip.
  *   scale      softmax scale applied to the 576-d dot product.
  *   num_splits split-K parts (1..DSA_MAX_SPLITS, 0 = library's choice); the
@@ -193,7 +197,7 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
  * enters the value product as a bf16 high + low pair (~16 significant bits).
  * ws: at least dsa_workspace_bytes(Q, 1, topk, num_splits) bytes.
  */
-dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
+dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages, int page_size,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int heads, int topk,
@@ -223,7 +227,7 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
  *   dsa_sparse_mla_decode but are not reported (there is no error word).
  */
 dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool, int num_pages,
-                                         const int32_t* page_table, int max_pages,
+                                         int page_size, const int32_t* page_table, int max_pages,
                                          const int32_t* q_offsets, const int32_t* q_vis,
                                          const int32_t* idx, int B, int Q, int heads, int topk,
                                          float scale, int num_splits, float* out, float* lse,
@@ -266,10 +270,76 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                            const int32_t* q_vis, int B, int Q, int heads, int idx_heads,
                            int max_len, int topk,
                            const void* const* q_layers, const void* const* pool_layers,
-                           int num_pages, const int32_t* const* page_table_layers,
+                           int num_pages, int page_size, const int32_t* const* page_table_layers,
                            int max_pages, float scale, int num_splits,
                            float* const* out_layers, float* const* lse_layers,
                            int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Two-tier latent cache (HiSparse)  ("GLM-5.2 推理部署", section "HiSparse 的
+ * 通信路径：GPU↔CPU KV swap": the full cache in pinned host memory, a buffer
+ * of hot 16-token slots in HBM; per step, top-K miss detection, LRU
+ * eviction, page-table update and an H2D fetch of the missing entries).
+ *
+ * Layouts.  The host tier of sequence b is pages b*max_pages .. of a pinned
+ * host array bf16 [B*max_pages, 16, 576]; its device buffer is slots
+ * b*dev_slots .. of a device pool bf16 [B*dev_slots, 16, 576], which
+ * dsa_sparse_mla_decode reads with page_size = DSA_TIER_PAGE through the page
+ * table the plan produces.  Token s of sequence b is row s%16 of its logical
+ * page s/16.
+ *
+ * Rules (readings of the page): every page a step selects counts as used at
+ * that step; the misses of a sequence are placed, in ascending page order,
+ * into the slots not selected at this step with the oldest last use (never
+ * used first, ties to the lower slot), evicting their pages; a step that
+ * selects more distinct pages of one sequence than dev_slots is refused.
+ *
+ * The state is caller-owned HOST memory of dsa_tier_state_bytes bytes
+ * (8-byte aligned); dsa_tier_init resets it (every slot empty).  The plan and
+ * the state live on the host: no device work, no synchronisation.
+ */
+size_t dsa_tier_state_bytes(int B, int dev_slots, int max_pages);   /* 0 = invalid sizes */
+dsa_status dsa_tier_init(void* state, size_t state_bytes, int B, int dev_slots, int max_pages);
+
+/*
+ * One step's plan, on the host.
+ *   idx        HOST int32 [Q,topk]: the step's selected positions (-1 = none),
+ *              rows of sequence b at q_offsets[b] .. q_offsets[b+1]-1
+ *   q_offsets  HOST int32 [B+1] (q_offsets[B] = Q)
+ *   page_table NULL or HOST int32 [B,max_pages] out: device pool page of every
+ *              resident logical page, -1 elsewhere (a full table; the fetch
+ *              below patches a device table incrementally instead)
+ *   copies     HOST int32 [cap_copies,3] out: (host page to fetch, device page
+ *              it goes to, host page evicted from that slot or -1)
+ *   n_copies   out: copies written;  stats: NULL or int64 [3] out: this
+ *              step's hits, misses, evictions (distinct pages)
+ * Returns DSA_ERR_UNSUPPORTED if a sequence needs more slots than it has,
+ * DSA_ERR_DEVICE_BOUNDS for a position beyond max_pages*16, DSA_ERR_WORKSPACE
+ * if the misses exceed cap_copies; a refused step leaves the state unchanged.
+ */
+dsa_status dsa_tier_plan(void* state, const int32_t* idx, int Q, int topk,
+                         const int32_t* q_offsets, int32_t* page_table, int32_t* copies,
+                         int cap_copies, int* n_copies, int64_t* stats);
+
+/*
+ * Fetch of the planned pages: one kernel reads each planned host page of
+ * `copies` (DEVICE int32 [n,3], as the plan wrote them) from the pinned host
+ * cache and writes the 18,432-byte page into its device slot, on `stream`.
+ *   page_table  NULL or DEVICE int32 [B,max_pages]: patched in the same kernel
+ *               (the evicted page's entry becomes -1, the fetched page's
+ *               entry its device page), so a table that started as all -1 and
+ *               went through every step's fetch equals the plan's table
+ *   host_cache  PINNED host memory (cudaHostAlloc / pinned torch tensor) of
+ *               host_pages pages; anything else (pageable or device memory)
+ *               is refused with DSA_ERR_INVALID_ARG before any launch
+ *   dev_pool    device memory of dev_pages pages
+ *   ws          workspace (its error word flags copies outside either cache,
+ *               which are skipped)
+ * Call it once per layer's cache with the same copies.
+ */
+dsa_status dsa_tier_fetch(const void* host_cache, int64_t host_pages, void* dev_pool,
+                          int64_t dev_pages, const int32_t* copies, int n, int32_t* page_table,
+                          void* ws, void* stream);
 
 /*
  * Synchronises `stream`, reads and clears the workspace's device error flag.

@@ -15,6 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdsa.so")
 
 PAGE_SIZE = 64
+TIER_PAGE = 16       # tokens per slot of the two-tier (HiSparse) cache
 HEADS = 128          # MLA heads, DeepSeek-V3.2
 HEADS_GLM = 64       # MLA heads, GLM-5.2
 DIM = 576
@@ -41,13 +42,17 @@ SIGNATURES = {
     "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
                               _P]),
-    "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _P,
-                                   _P, _SZ, _P]),
-    "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I,
-                                           _P, _P, _P]),
+    "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P,
+                                   _P, _P, _SZ, _P]),
+    "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F,
+                                           _I, _P, _P, _P]),
     "dsa_lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                             _PP, _PP, _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
+                             _PP, _PP, _I, _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
+    "dsa_tier_state_bytes": (_SZ, [_I, _I, _I]),
+    "dsa_tier_init": (_I, [_P, _SZ, _I, _I, _I]),
+    "dsa_tier_plan": (_I, [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P]),
+    "dsa_tier_fetch": (_I, [_P, _I64, _P, _I64, _P, _I, _P, _P, _P]),
     "dsa_check_error": (_I, [_P, _P]),
 }
 
@@ -81,6 +86,14 @@ def _ptr(t: Optional[torch.Tensor]):
         return None
     if not t.is_cuda:
         raise ValueError("libdsa takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libdsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("this argument is host memory")
     if not t.is_contiguous():
         raise ValueError("libdsa takes contiguous tensors")
     return ctypes.c_void_p(t.data_ptr())
@@ -155,7 +168,8 @@ def dsa_indexer_topk(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len,
 def dsa_sparse_mla_decode(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scale, out, lse, ws,
                           num_splits=0, stream=None):
     _check(lib().dsa_sparse_mla_decode(
-        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
+        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], kv_pool.shape[1], _ptr(page_table),
+        page_table.shape[1],
         _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1],
         float(scale), num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
         "dsa_sparse_mla_decode")
@@ -166,7 +180,8 @@ def dsa_sparse_mla_decode_noalloc(q, kv_pool, page_table, q_offsets, q_vis, idx,
     """dsa_sparse_mla_decode without a workspace (split-K partials in the
     library's own fixed device array; see include/dsa.h)."""
     _check(lib().dsa_sparse_mla_decode_noalloc(
-        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(page_table), page_table.shape[1],
+        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], kv_pool.shape[1], _ptr(page_table),
+        page_table.shape[1],
         _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1],
         float(scale), num_splits, _ptr(out), _ptr(lse), _stream(stream)),
         "dsa_sparse_mla_decode_noalloc")
@@ -191,9 +206,54 @@ def dsa_decode_step(q_idx_layers, w_layers, k_idx_layers, seq_offsets, q_offsets
         _ptr_array(k_idx_layers), lead.shape[0], _ptr(seq_offsets), _ptr(q_offsets), _ptr(q_vis),
         B, q_layers[0].shape[0], q_layers[0].shape[1], lead_q.shape[1], max_len, topk,
         _ptr_array(q_layers), _ptr_array(pool_layers),
-        pool_layers[0].shape[0], _ptr_array(page_table_layers), page_table_layers[0].shape[1],
+        pool_layers[0].shape[0], pool_layers[0].shape[1], _ptr_array(page_table_layers),
+        page_table_layers[0].shape[1],
         float(scale), num_splits, _ptr_array(out_layers), _ptr_array(lse_layers), _ptr(idx_out),
         _ptr(ws), ws.numel(), _stream(stream)), "dsa_decode_step")
+
+
+def dsa_tier_state_bytes(B: int, dev_slots: int, max_pages: int) -> int:
+    return lib().dsa_tier_state_bytes(B, dev_slots, max_pages)
+
+
+def tier_state(B: int, dev_slots: int, max_pages: int) -> torch.Tensor:
+    """Host memory for a two-tier cache's state, initialised (every slot empty)."""
+    n = dsa_tier_state_bytes(B, dev_slots, max_pages)
+    if n == 0:
+        raise DSAError(1, "dsa_tier_state_bytes")
+    st = torch.empty((n + 7) // 8, dtype=torch.int64)      # 8-byte aligned host bytes
+    dsa_tier_init(st, B, dev_slots, max_pages)
+    return st
+
+
+def dsa_tier_init(state: torch.Tensor, B: int, dev_slots: int, max_pages: int):
+    _check(lib().dsa_tier_init(_host_ptr(state), state.numel() * state.element_size(), B,
+                               dev_slots, max_pages), "dsa_tier_init")
+
+
+def dsa_tier_plan(state, idx, q_offsets, copies, page_table=None):
+    """Host tensors: idx int32 [Q,topk], q_offsets int32 [B+1], copies int32
+    [cap,3] (out), page_table None or int32 [B,max_pages] (out).  Returns
+    (n_copies, (hits, misses, evictions))."""
+    n = ctypes.c_int(0)
+    stats = (ctypes.c_int64 * 3)()
+    _check(lib().dsa_tier_plan(_host_ptr(state), _host_ptr(idx), idx.shape[0], idx.shape[1],
+                               _host_ptr(q_offsets),
+                               None if page_table is None else _host_ptr(page_table),
+                               _host_ptr(copies), copies.shape[0], ctypes.byref(n), stats),
+           "dsa_tier_plan")
+    return n.value, (stats[0], stats[1], stats[2])
+
+
+def dsa_tier_fetch(host_cache, dev_pool, copies, n, ws, page_table=None, stream=None):
+    """host_cache: pinned host tensor [host_pages,16,576] bf16; dev_pool: device
+    tensor [dev_pages,16,576] bf16; copies: device int32 [>=n,3]; page_table:
+    None or the device int32 [B,max_pages] table to patch."""
+    if not host_cache.is_pinned():
+        raise ValueError("host_cache must be pinned host memory")
+    _check(lib().dsa_tier_fetch(_host_ptr(host_cache), host_cache.shape[0], _ptr(dev_pool),
+                                dev_pool.shape[0], _ptr(copies), n, _ptr(page_table), _ptr(ws),
+                                _stream(stream)), "dsa_tier_fetch")
 
 
 def dsa_check_error(ws, stream=None):

@@ -9,7 +9,8 @@
 namespace dsa {
 
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool,
-                                   int num_pages, const int32_t* page_table, int max_pages,
+                                   int num_pages, int page_size, const int32_t* page_table,
+                                   int max_pages,
                                    const int32_t* q_offsets, const int32_t* q_vis,
                                    const int32_t* idx, int B, int Q, int H, int topk,
                                    float scale, int S, float* out, float* lse, float* o_part,
@@ -66,6 +67,11 @@ bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* L) {
   w.total = off;
   *L = w;
   return true;
+}
+
+bool page_size_ok(int page_size, int num_pages) {
+  if (page_size < 1 || page_size > 1024 || (page_size & (page_size - 1))) return false;
+  return static_cast<int64_t>(num_pages) * page_size < (int64_t(1) << 31);
 }
 
 int device_sm_count() {
@@ -135,7 +141,7 @@ dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* 
   return DSA_OK;
 }
 
-dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
+dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages, int page_size,
                          const int32_t* page_table, int max_pages, const int32_t* q_offsets,
                          const int32_t* q_vis, const int32_t* idx, int B, int Q, int H,
                          int topk, float scale, int S, float* out, float* lse, void* ws,
@@ -145,7 +151,7 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
   float* l_part = ws_ptr<float>(ws, L.l_part);
   cudaError_t e = launch_sparse_mla(static_cast<const __nv_bfloat16*>(q),
                                     static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
-                                    page_table, max_pages, q_offsets, q_vis, idx, B, Q, H, topk,
+                                    page_size, page_table, max_pages, q_offsets, q_vis, idx, B, Q, H, topk,
                                     scale, S, out, lse, o_part, l_part, err, st, pdl);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (S > 1) {
@@ -155,11 +161,12 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages,
   return DSA_OK;
 }
 
-dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages,
+dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages, int page_size,
                       const int32_t* page_table, int max_pages, const int32_t* idx, float* out,
                       float* lse, float scale, int heads) {
   if (!q || !kv_pool || !page_table || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
   if (!heads_ok(heads)) return DSA_ERR_UNSUPPORTED;
+  if (!page_size_ok(page_size, num_pages > 0 ? num_pages : 1)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kv_pool) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
   if (num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale != scale) return DSA_ERR_INVALID_ARG;
@@ -169,13 +176,14 @@ dsa_status mla_checks(const void* q, const void* kv_pool, int num_pages,
 }  // namespace
 
 cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                              const int32_t* page_table, int max_pages,
+                              int page_size, const int32_t* page_table, int max_pages,
                               const int32_t* q_offsets, const int32_t* q_vis,
                               const int32_t* idx, int B, int Q, int H, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st, bool pdl) {
-  return launch_sparse_mla_tc(q, pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B,
-                              Q, H, topk, scale, S, out, lse, o_part, l_part, err, st, pdl);
+  return launch_sparse_mla_tc(q, pool, num_pages, page_size, page_table, max_pages, q_offsets,
+                              q_vis, idx, B, Q, H, topk, scale, S, out, lse, o_part, l_part, err,
+                              st, pdl);
 }
 
 }  // namespace dsa
@@ -262,7 +270,7 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
                          static_cast<cudaStream_t>(stream));
 }
 
-dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages,
+dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages, int page_size,
                                  const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int heads, int topk,
@@ -272,15 +280,15 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
   if (B <= 0 || Q <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
   if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
   if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
-  dsa_status s = mla_checks(q, kv_pool, num_pages, page_table, max_pages, idx, out, lse, scale,
-                            heads);
+  dsa_status s = mla_checks(q, kv_pool, num_pages, page_size, page_table, max_pages, idx, out, lse,
+                            scale, heads);
   if (s != DSA_OK) return s;
   WsLayout L;
   if (!ws_layout(Q, 1, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
-  return do_sparse_mla(q, kv_pool, num_pages, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
-                       heads, topk, scale, L.S, out, lse, ws, L, static_cast<cudaStream_t>(stream),
-                       false);
+  return do_sparse_mla(q, kv_pool, num_pages, page_size, page_table, max_pages, q_offsets, q_vis,
+                       idx, B, Q, heads, topk, scale, L.S, out, lse, ws, L,
+                       static_cast<cudaStream_t>(stream), false);
 }
 
 dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, int heads,
@@ -301,7 +309,7 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                            const int32_t* q_vis, int B, int Q, int heads, int idx_heads,
                            int max_len, int topk,
                            const void* const* q_layers, const void* const* pool_layers,
-                           int num_pages, const int32_t* const* page_table_layers,
+                           int num_pages, int page_size, const int32_t* const* page_table_layers,
                            int max_pages, float scale, int num_splits,
                            float* const* out_layers, float* const* lse_layers,
                            int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
@@ -317,8 +325,8 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
         (s = indexer_checks(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys,
                             idx_heads)) != DSA_OK)
       return s;
-    if ((s = mla_checks(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
-                        idx_out, out_layers[l], lse_layers[l], scale, heads)) != DSA_OK)
+    if ((s = mla_checks(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
+                        max_pages, idx_out, out_layers[l], lse_layers[l], scale, heads)) != DSA_OK)
       return s;
   }
   WsLayout L;
@@ -334,8 +342,9 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
                           nullptr, ws, L, st);
       if (s != DSA_OK) return s;
     }
-    s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_table_layers[l], max_pages,
-                      q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S, out_layers[l],
+    s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
+                      max_pages, q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S,
+                      out_layers[l],
                       lse_layers[l], ws, L, st, true);
     if (s != DSA_OK) return s;
   }

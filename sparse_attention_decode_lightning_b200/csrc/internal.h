@@ -29,6 +29,9 @@ bool encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ba
                      uint32_t box_inner, uint32_t box_rows);
 
 bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* out);
+// a latent-cache page of page_size tokens: a power of two from 1 to 1024, and
+// every pool row index (num_pages * page_size) fits in int32
+bool page_size_ok(int page_size, int num_pages);
 int device_sm_count();
 int choose_splits(int Q, int topk, int requested);
 
@@ -48,7 +51,7 @@ cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,
                               int32_t* out_idx, float* out_scores, cudaStream_t st);
 
 cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                              const int32_t* page_table, int max_pages,
+                              int page_size, const int32_t* page_table, int max_pages,
                               const int32_t* q_offsets, const int32_t* q_vis,
                               const int32_t* idx, int B, int Q, int H, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,

@@ -21,7 +21,7 @@
 namespace dsa {
 
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                                 const int32_t* page_table, int max_pages,
+                                 int page_size, const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int H, int topk, float scale,
                                  int S, float* out, float* lse, float* o_part, float* l_part,
@@ -64,7 +64,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 using namespace dsa;
 
 extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool,
-                                                    int num_pages, const int32_t* page_table,
+                                                    int num_pages, int page_size,
+                                                    const int32_t* page_table,
                                                     int max_pages, const int32_t* q_offsets,
                                                     const int32_t* q_vis, const int32_t* idx,
                                                     int B, int Q, int heads, int topk, float scale,
@@ -75,6 +76,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
   if (!aligned16(q) || !aligned16(kv_pool) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
   if (B <= 0 || Q <= 0 || topk <= 0 || num_pages <= 0 || max_pages <= 0) return DSA_ERR_INVALID_ARG;
   if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!page_size_ok(page_size, num_pages)) return DSA_ERR_UNSUPPORTED;
   if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
   if (heads != DSA_HEADS && heads != DSA_HEADS_GLM) return DSA_ERR_UNSUPPORTED;
   if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
@@ -91,7 +93,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
   // every partial is written by the kernel before the merge reads it, so the
   // array needs no clearing; range violations are skipped but not reported
   if (launch_sparse_mla_tc(static_cast<const __nv_bfloat16*>(q),
-                           static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_table,
+                           static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_size, page_table,
                            max_pages, q_offsets, q_vis, idx, B, Q, heads, topk, scale, S, out, lse,
                            o_part, l_part, nullptr, s, false) != cudaSuccess)
     return DSA_ERR_CUDA;

@@ -89,6 +89,7 @@ struct MlaTcArgs {
   const int32_t* page_table;
   int max_pages;
   int num_pages;
+  int page_shift;                              // log2 of the tokens per cache page
   const int32_t* q_offsets;
   const int32_t* q_vis;
   const int32_t* idx;
@@ -223,8 +224,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int sx = sv[k];
-      const bool ok = sx >= 0 && sx < vis && (sx >> 6) < a.max_pages;
-      pg[k] = ok ? a.page_table[static_cast<size_t>(b) * a.max_pages + (sx >> 6)] : -1;
+      const bool ok = sx >= 0 && sx < vis && (sx >> a.page_shift) < a.max_pages;
+      pg[k] = ok ? a.page_table[static_cast<size_t>(b) * a.max_pages + (sx >> a.page_shift)] : -1;
     }
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
@@ -233,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int sx = sv[k];
         const bool ok = pg[k] >= 0 && pg[k] < a.num_pages;
         if (!ok && sx != -1 && rank == 0) raise_error(a.err, DEVERR_BOUNDS);
-        crd[jj] = ok ? pg[k] * DSA_PAGE_SIZE + (sx & (DSA_PAGE_SIZE - 1)) : -1;
+        crd[jj] = ok ? (pg[k] << a.page_shift) + (sx & ((1 << a.page_shift) - 1)) : -1;
       }
     }
   }
@@ -574,13 +575,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }  // namespace
 
 cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                                 const int32_t* page_table, int max_pages,
+                                 int page_size, const int32_t* page_table, int max_pages,
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int H, int topk, float scale,
                                  int S, float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
   if (H != 128 && H != 64) return cudaErrorInvalidValue;
+  int page_shift = 0;
+  while ((1 << page_shift) < page_size) ++page_shift;
+  if (page_size <= 0 || (1 << page_shift) != page_size) return cudaErrorInvalidValue;
   // RoPE query dims: boxes of H heads x 64 bf16 (rows past H in shared memory
   // are never read into a head's result)
   CUtensorMap tq;
@@ -604,7 +608,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                        static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4, 32,
                        static_cast<uint32_t>(H)))
     return cudaErrorInvalidValue;
-  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, q_offsets, q_vis, idx, B, Q, topk, S,
+  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, page_shift, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * Q * S), 1, 1);

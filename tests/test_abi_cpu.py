@@ -99,15 +99,15 @@ def test_host_checks_reject_bad_arguments_without_a_device():
     assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
                               null, fake, 16, null) == 6
     # sparse MLA: bad scale, bad split count, null page table
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, 64, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.0), 0, fake, fake, fake, 1 << 30, null) == 1
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, 64, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.07), 33, fake, fake, fake, 1 << 30, null) == 2
-    assert L.dsa_sparse_mla_decode(fake, fake, 10, null, 4, fake, fake, fake, 1, 1, 128, 2048,
+    assert L.dsa_sparse_mla_decode(fake, fake, 10, 64, null, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30, null) == 1
     # MLA head counts other than 128 (DeepSeek-V3.2) and 64 (GLM-5.2)
     for h in (32, 96, 256):
-        assert L.dsa_sparse_mla_decode(fake, fake, 10, fake, 4, fake, fake, fake, 1, 1, h, 2048,
+        assert L.dsa_sparse_mla_decode(fake, fake, 10, 64, fake, 4, fake, fake, fake, 1, 1, h, 2048,
                                        ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30,
                                        null) == 2
         assert L.dsa_lse_combine(fake, fake, 1, 2, h, fake, fake, null) == 2
@@ -115,10 +115,10 @@ def test_host_checks_reject_bad_arguments_without_a_device():
     PP = ctypes.POINTER(ctypes.c_void_p)
     arr = (ctypes.c_void_p * 1)(1 << 20)
     assert L.dsa_decode_step(0, 1, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 128, 64, 100,
-                             2048, arr, arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
+                             2048, arr, arr, 10, 64, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
                              fake, 1 << 30, null) == 1
     assert L.dsa_decode_step(1, 0, 0, arr, arr, arr, 100, fake, fake, fake, 1, 1, 128, 64, 100,
-                             2048, arr, arr, 10, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
+                             2048, arr, arr, 10, 64, arr, 4, ctypes.c_float(0.07), 0, arr, arr, fake,
                              fake, 1 << 30, null) == 1
     # check_error without a workspace
     assert L.dsa_check_error(null, null) == 1

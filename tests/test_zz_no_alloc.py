@@ -21,7 +21,7 @@ def _call_noalloc(inp, layer, idx, out, lse, num_splits):
     L = dsa.lib()
     st = L.dsa_sparse_mla_decode_noalloc(
         ctypes.c_void_p(inp.layers[layer]["q"].data_ptr()),
-        ctypes.c_void_p(inp.layers[layer]["pool"].data_ptr()), inp.num_pages,
+        ctypes.c_void_p(inp.layers[layer]["pool"].data_ptr()), inp.num_pages, 64,
         ctypes.c_void_p(inp.page_table.data_ptr()), inp.max_pages,
         ctypes.c_void_p(inp.q_offsets.data_ptr()), ctypes.c_void_p(inp.q_vis.data_ptr()),
         ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, inp.layers[layer]["q"].shape[1], idx.shape[1],
@@ -69,7 +69,7 @@ def test_noalloc_rejects_requests_beyond_its_array():
     L = dsa.lib()
     st = L.dsa_sparse_mla_decode_noalloc(
         ctypes.c_void_p(inp.layers[0]["q"].data_ptr()), ctypes.c_void_p(inp.layers[0]["pool"].data_ptr()),
-        inp.num_pages, ctypes.c_void_p(inp.page_table.data_ptr()), inp.max_pages,
+        inp.num_pages, 64, ctypes.c_void_p(inp.page_table.data_ptr()), inp.max_pages,
         ctypes.c_void_p(inp.q_offsets.data_ptr()), ctypes.c_void_p(inp.q_vis.data_ptr()),
         ctypes.c_void_p(idx.data_ptr()), inp.B, inp.Q, 128, 2048, ctypes.c_float(inp.scale), 2,
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), None)
