@@ -488,10 +488,12 @@ def run_reference(args):
 def run_tier(args):
     """Two-tier (HiSparse) decode at GLM-5.2 shapes and 1M context, one GPU.
 
-    Per step: the host plan (miss detection, LRU eviction), the upload of the
-    copy list and the index rows, one kernel that fetches the missing 16-token
-    pages from pinned host memory and patches the device page table, and the
-    sparse MLA over the device buffer (page size 16).  The full latent cache (4 x 1M tokens, 4.8 GB)
+    Per step (the line's value): the upload of the index rows, the device
+    planner (miss detection, LRU eviction, page-table update) and the fetch
+    kernel that pulls the missing 16-token pages from pinned host memory, then
+    the sparse MLA over the device buffer (page size 16).  The same steps are
+    then run with the plan on the host (host_plan_path), whose fetch kernel
+    time gives the roofline line.  The full latent cache (4 x 1M tokens, 4.8 GB)
     lives in pinned host memory; each sequence has 8192 device slots (host :
     device = 8).  The selected tokens come from a hot set of 1024 pages per
     sequence of which 64 are replaced every step (a synthetic locality model:
@@ -543,6 +545,33 @@ def run_tier(args):
         idx_steps.append(torch.from_numpy(np.stack(rows)).pin_memory())
     stream = torch.cuda.current_stream(dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    scale = 1 / qk ** 0.5
+    # device path: the planner and the fetch run on the GPU, no host round trip
+    pt_dev = torch.empty(B, P, dtype=torch.int32, device=dev)
+    dst = dsa.tier_dev_state(B, D, P, pt_dev)
+    # steps are enqueued back to back (no host wait inside the loop), so the
+    # host-side argument checks overlap the GPU and the events time the GPU
+    drec = {"upload": [], "swap_in": [], "mla": []}
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in idx_steps]
+    for i, idx_h in enumerate(idx_steps):
+        e = evs[i]
+        e[0].record(stream)
+        idx_d.copy_(idx_h, non_blocking=True)
+        e[1].record(stream)
+        dsa.dsa_tier_swap_in(dst, B, D, P, idx_d, q_off, pt_dev, host, pool, ws, stream=stream)
+        e[2].record(stream)
+        dsa.dsa_sparse_mla_decode(q, pool, pt_dev, q_off, vis, idx_d, B, scale, out, lse, ws,
+                                  stream=stream)
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    for e in evs[n_steps - args.steps:]:
+        drec["upload"].append(e[0].elapsed_time(e[1]) * 1e3)
+        drec["swap_in"].append(e[1].elapsed_time(e[2]) * 1e3)
+        drec["mla"].append(e[2].elapsed_time(e[3]) * 1e3)
+    dev_step_span_us = evs[n_steps - args.steps][0].elapsed_time(evs[-1][3]) * 1e3 / args.steps
+    dsa.dsa_check_error(ws)
+    # host path: the same steps with the plan on the host (fresh tier state)
+    pool.zero_()
     rec = {"plan": [], "upload": [], "fetch": [], "mla": [], "misses": [], "bytes": []}
     for i, idx_h in enumerate(idx_steps):
         t0 = time.perf_counter()
@@ -554,7 +583,7 @@ def run_tier(args):
         ev[1].record(stream)
         dsa.dsa_tier_fetch(host, pool, cp_d, n, ws, page_table=pt_d, stream=stream)
         ev[2].record(stream)
-        dsa.dsa_sparse_mla_decode(q, pool, pt_d, q_off, vis, idx_d, B, 1 / qk ** 0.5, out, lse, ws,
+        dsa.dsa_sparse_mla_decode(q, pool, pt_d, q_off, vis, idx_d, B, scale, out, lse, ws,
                                   stream=stream)
         ev[3].record(stream)
         torch.cuda.synchronize(dev)
@@ -577,19 +606,25 @@ def run_tier(args):
     torch.cuda.synchronize(dev)
     copy_gbs = 3 * (256 << 20) / (ev[3].elapsed_time(ev[4]) / 1e3) / 1e9
     m = {k: float(np.mean(v)) for k, v in rec.items()}
-    step_us = m["plan"] + m["upload"] + m["fetch"] + m["mla"]
+    dm = {k: float(np.mean(v)) for k, v in drec.items()}
+    host_step_us = m["plan"] + m["upload"] + m["fetch"] + m["mla"]
+    step_us = dev_step_span_us          # first timed step's start to the last one's end
     fetch_gbs = m["bytes"] / (m["fetch"] / 1e6) / 1e9 if m["fetch"] > 0 else 0.0
     return {
-        "metric": "HiSparse two-tier decode step, GLM-5.2 shapes, 1M ctx (plan + upload + fetch + MLA)",
+        "metric": "HiSparse two-tier decode step, GLM-5.2 shapes, 1M ctx (device plan + fetch + MLA)",
         "value": B / (step_us / 1e6), "unit": "query-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": step_us / 1e3, "higher_is_better": True,
         "dtype": "bf16 attention, f32 accumulate", "data": "synthetic",
         "config": {"workload": "glm52_tier_b4_ctx1m", "B": B, "L": L, "heads": heads, "topk": topk,
                    "dev_slots_per_seq": D, "host_pages_per_seq": P, "page_tokens": PT,
                    "hot_pages": HOT, "hot_pages_replaced_per_step": CHURN},
-        "stages_us": {"plan_host": m["plan"], "upload": m["upload"], "fetch": m["fetch"],
-                      "mla": m["mla"]},
+        "stages_us": {"upload_idx": dm["upload"], "swap_in": dm["swap_in"], "mla": dm["mla"]},
         "misses_per_step": m["misses"],
+        "misses_note": "from the host-plan pass over the same steps (the two plans are equal)",
+        "host_plan_path": {"ms_per_step": host_step_us / 1e3,
+                           "stages_us": {"plan_host": m["plan"], "upload": m["upload"],
+                                         "fetch": m["fetch"], "mla": m["mla"]},
+                           "misses_per_step": m["misses"]},
         "roofline": {"bound": "host link", "kernel": "tier_fetch_kernel", "achieved": fetch_gbs,
                      "peak": copy_gbs, "peak_source": "pinned cudaMemcpyAsync H2D in this run",
                      "unit": "GB/s", "frac": fetch_gbs / copy_gbs if copy_gbs else None},

@@ -342,8 +342,43 @@ dsa_status dsa_tier_fetch(const void* host_cache, int64_t host_pages, void* dev_
                           void* ws, void* stream);
 
 /*
+ * The same plan computed on the device, followed by the fetch: one call per
+ * step that needs no host round trip (and can be captured in a CUDA graph).
+ *   dev_state   DEVICE memory of dsa_tier_dev_state_bytes bytes, reset by
+ *               dsa_tier_dev_init (which also sets every page_table entry to
+ *               -1); dev_slots <= 8192 (the planner sorts a sequence's slots
+ *               in shared memory)
+ *   idx         DEVICE int32 [Q,topk]   q_offsets DEVICE int32 [B+1]
+ *   page_table  DEVICE int32 [B,max_pages]: the page -> device pool page map,
+ *               updated in place (dsa_sparse_mla_decode reads it with
+ *               page_size = DSA_TIER_PAGE)
+ *   host_cache  PINNED host bf16 [B*max_pages,16,576]   dev_pool DEVICE bf16
+ *               [B*dev_slots,16,576]
+ *   ws          workspace whose error word takes DSA_ERR_DEVICE_BOUNDS for a
+ *               position beyond max_pages*16 (skipped) and DSA_ERR_UNSUPPORTED
+ *               (through dsa_check_error) for a sequence that selected more
+ *               distinct pages than dev_slots (its step is skipped)
+ * The rules are those of dsa_tier_plan; the copy list holds the same triples
+ * (sequences may appear in any order).  dsa_tier_dev_stats synchronises the
+ * stream and returns the last step's n_copies, hits, misses, evictions and
+ * the number of steps so far; dsa_tier_dev_copies is the device address of
+ * the copy list (int32 [n_copies,3]) inside dev_state.
+ */
+size_t dsa_tier_dev_state_bytes(int B, int dev_slots, int max_pages);   /* 0 = invalid sizes */
+dsa_status dsa_tier_dev_init(void* dev_state, size_t state_bytes, int B, int dev_slots,
+                             int max_pages, int32_t* page_table, void* stream);
+dsa_status dsa_tier_swap_in(void* dev_state, size_t state_bytes, int B, int dev_slots,
+                            int max_pages, const int32_t* idx, int Q, int topk,
+                            const int32_t* q_offsets, int32_t* page_table,
+                            const void* host_cache, void* dev_pool, void* ws, void* stream);
+dsa_status dsa_tier_dev_stats(const void* dev_state, int64_t* stats /* host int64 [5] */,
+                              void* stream);
+const int32_t* dsa_tier_dev_copies(const void* dev_state, int B, int dev_slots, int max_pages);
+
+/*
  * Synchronises `stream`, reads and clears the workspace's device error flag.
- * Returns DSA_OK, DSA_ERR_DEVICE_BOUNDS, DSA_ERR_TIMEOUT or DSA_ERR_CUDA.
+ * Returns DSA_OK, DSA_ERR_DEVICE_BOUNDS, DSA_ERR_TIMEOUT, DSA_ERR_UNSUPPORTED (a device
+ * tier step that needed more slots than a sequence has) or DSA_ERR_CUDA.
  */
 dsa_status dsa_check_error(void* ws, void* stream);
 

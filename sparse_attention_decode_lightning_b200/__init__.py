@@ -53,6 +53,11 @@ SIGNATURES = {
     "dsa_tier_init": (_I, [_P, _SZ, _I, _I, _I]),
     "dsa_tier_plan": (_I, [_P, _P, _I, _I, _P, _P, _P, _I, _P, _P]),
     "dsa_tier_fetch": (_I, [_P, _I64, _P, _I64, _P, _I, _P, _P, _P]),
+    "dsa_tier_dev_state_bytes": (_SZ, [_I, _I, _I]),
+    "dsa_tier_dev_init": (_I, [_P, _SZ, _I, _I, _I, _P, _P]),
+    "dsa_tier_swap_in": (_I, [_P, _SZ, _I, _I, _I, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "dsa_tier_dev_stats": (_I, [_P, _P, _P]),
+    "dsa_tier_dev_copies": (_P, [_P, _I, _I, _I]),
     "dsa_check_error": (_I, [_P, _P]),
 }
 
@@ -254,6 +259,45 @@ def dsa_tier_fetch(host_cache, dev_pool, copies, n, ws, page_table=None, stream=
     _check(lib().dsa_tier_fetch(_host_ptr(host_cache), host_cache.shape[0], _ptr(dev_pool),
                                 dev_pool.shape[0], _ptr(copies), n, _ptr(page_table), _ptr(ws),
                                 _stream(stream)), "dsa_tier_fetch")
+
+
+def tier_dev_state(B: int, dev_slots: int, max_pages: int, page_table, stream=None) -> torch.Tensor:
+    """Device memory for the on-device planner's state, initialised; page_table
+    (device int32 [B,max_pages]) is set to all -1."""
+    n = lib().dsa_tier_dev_state_bytes(B, dev_slots, max_pages)
+    if n == 0:
+        raise DSAError(2, "dsa_tier_dev_state_bytes")
+    st = torch.empty(n, dtype=torch.uint8, device=page_table.device)
+    _check(lib().dsa_tier_dev_init(_ptr(st), n, B, dev_slots, max_pages, _ptr(page_table),
+                                   _stream(stream)), "dsa_tier_dev_init")
+    return st
+
+
+def dsa_tier_swap_in(dev_state, B, dev_slots, max_pages, idx, q_offsets, page_table, host_cache,
+                     dev_pool, ws, stream=None):
+    """Plan on the device and fetch: idx device int32 [Q,topk], q_offsets device
+    int32 [B+1], page_table device int32 [B,max_pages] (updated), host_cache
+    pinned host bf16 [B*max_pages,16,576], dev_pool device bf16 [B*dev_slots,16,576]."""
+    if not host_cache.is_pinned():
+        raise ValueError("host_cache must be pinned host memory")
+    _check(lib().dsa_tier_swap_in(_ptr(dev_state), dev_state.numel(), B, dev_slots, max_pages,
+                                  _ptr(idx), idx.shape[0], idx.shape[1], _ptr(q_offsets),
+                                  _ptr(page_table), _host_ptr(host_cache), _ptr(dev_pool), _ptr(ws),
+                                  _stream(stream)), "dsa_tier_swap_in")
+
+
+def dsa_tier_dev_stats(dev_state, stream=None):
+    """(n_copies, hits, misses, evictions) of the last device step, and the step count."""
+    out = (ctypes.c_int64 * 5)()
+    _check(lib().dsa_tier_dev_stats(_ptr(dev_state), out, _stream(stream)), "dsa_tier_dev_stats")
+    return tuple(out[:4]), out[4]
+
+
+def dsa_tier_dev_copies(dev_state, B, dev_slots, max_pages, n):
+    """The device planner's copy list (int32 [n,3]) as a tensor view of dev_state."""
+    p = lib().dsa_tier_dev_copies(_ptr(dev_state), B, dev_slots, max_pages)
+    off = p - dev_state.data_ptr()
+    return dev_state[off:off + 12 * n].view(torch.int32).view(n, 3)
 
 
 def dsa_check_error(ws, stream=None):

@@ -362,6 +362,7 @@ dsa_status dsa_check_error(void* ws, void* stream) {
     if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
   }
   if (flag & DEVERR_TIMEOUT) return DSA_ERR_TIMEOUT;
+  if (flag & DEVERR_CAPACITY) return DSA_ERR_UNSUPPORTED;   // the cause of any bounds flag after it
   if (flag & DEVERR_BOUNDS) return DSA_ERR_DEVICE_BOUNDS;
   return DSA_OK;
 }

@@ -15,6 +15,7 @@ namespace dsa {
 // device error flag bits (first word of the workspace)
 constexpr uint32_t DEVERR_BOUNDS = 1u;
 constexpr uint32_t DEVERR_TIMEOUT = 2u;
+constexpr uint32_t DEVERR_CAPACITY = 4u;   // a step needed more device slots than exist
 
 // a bounded wait gives up after this many nanoseconds of %globaltimer
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;

@@ -117,11 +117,13 @@ bool tier_sizes_ok(int B, int dev_slots, int max_pages) {
 __global__ void __launch_bounds__(256) tier_fetch_kernel(const uint4* __restrict__ host,
                                                          uint4* __restrict__ dev,
                                                          const int32_t* __restrict__ copies, int n,
+                                                         const int32_t* n_dev,
                                                          int64_t host_pages, int64_t dev_pages,
                                                          int32_t* __restrict__ page_table,
                                                          uint32_t* err) {
   constexpr int V = TIER_PAGE_BYTES / 16;      // 1152 uint4 per page
   constexpr int PER = (V + 255) / 256;         // 5 per thread
+  if (n_dev) n = min(n, *n_dev);               // the count the device planner wrote
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int64_t src = copies[3 * i], dst = copies[3 * i + 1], gone = copies[3 * i + 2];
     if (src < 0 || src >= host_pages || dst < 0 || dst >= dev_pages || gone >= host_pages) {
@@ -146,6 +148,307 @@ __global__ void __launch_bounds__(256) tier_fetch_kernel(const uint4* __restrict
       page_table[src] = static_cast<int32_t>(dst);
     }
   }
+}
+
+// ---------------------------------------------------------------- device planner
+// The same plan as dsa_tier_plan, computed on the device so that a tiered
+// step needs no host round trip (and can be captured in a graph).  Device
+// state, each region 256-byte aligned:
+//   hdr   int32 [16]: n_copies, hits, misses, evictions of the last step; step; done
+//   stamp int32 [B,P], page_of_slot int32 [B,D], last_use int32 [B,D], copies int32 [B*D,3]
+// The device page table (int32 [B,P], pool page b*D + slot or -1) is the
+// page -> slot map itself.
+constexpr int DEV_MAX_SLOTS = 8192;            // slots per sequence the planner sorts on chip
+constexpr int PLAN_THREADS = 1024;
+
+struct DevLayout {
+  size_t hdr, stamp, page_of_slot, last_use, copies, total;
+};
+
+DevLayout dev_layout(int B, int D, int P) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  DevLayout L;
+  size_t off = 0;
+  L.hdr = off;          off = up(off + 64);
+  L.stamp = off;        off = up(off + static_cast<size_t>(B) * P * 4);
+  L.page_of_slot = off; off = up(off + static_cast<size_t>(B) * D * 4);
+  L.last_use = off;     off = up(off + static_cast<size_t>(B) * D * 4);
+  L.copies = off;       off = up(off + static_cast<size_t>(B) * D * 12);
+  L.total = off;
+  return L;
+}
+
+int pow2_at_least(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+__device__ __forceinline__ int pow2_dev(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+// ascending bitonic sort of a[0..N) in shared memory, N a power of two; every
+// thread of the block calls it
+template <typename T>
+__device__ void block_bitonic_sort(T* a, int N) {
+  for (int k = 2; k <= N; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const T x = a[i], y = a[ixj];
+          if ((x > y) == ((i & k) == 0)) {
+            a[i] = y;
+            a[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// One CTA per sequence.  1. the distinct selected pages (a page's stamp is
+// swapped to this step; the thread that changed it lists the page);
+// 2. hits refresh their slot's last use, misses are listed; 3. every slot
+// gets the key (last use + 1, slot), or the largest key if its page is
+// selected now; the nmiss oldest are found by a radix select on the age
+// (ties to the lower slot) and only they, and the misses, are sorted on
+// chip; 4. miss i goes to the slot of victim i, evicting its page, and the
+// page table and copy list are written.  The last CTA to finish advances the step.
+__global__ void __launch_bounds__(PLAN_THREADS) tier_plan_kernel(
+    int32_t* __restrict__ hdr, int32_t* __restrict__ stamp, int32_t* __restrict__ page_of_slot,
+    int32_t* __restrict__ last_use, int32_t* __restrict__ copies, const int32_t* __restrict__ idx,
+    int Q, int topk, const int32_t* __restrict__ q_offsets, int D, int P,
+    int32_t* __restrict__ page_table, uint32_t* err) {
+  extern __shared__ __align__(16) uint8_t tsm[];
+  const int N = pow2_dev(D);
+  uint64_t* keys = reinterpret_cast<uint64_t*>(tsm);               // [N]
+  uint32_t* need = reinterpret_cast<uint32_t*>(keys + N);          // [D]
+  uint32_t* miss = need + D;                                       // [N]
+  __shared__ int s_nneed, s_nmiss, s_hits, s_base, s_digit, s_below, s_nvict;
+  __shared__ int s_hist[256], s_wsum[32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int t = hdr[4];
+  if (tid == 0) { s_nneed = 0; s_nmiss = 0; s_hits = 0; }
+  __syncthreads();
+  int32_t* stamp_b = stamp + static_cast<size_t>(b) * P;
+  int32_t* table_b = page_table + static_cast<size_t>(b) * P;
+  int q0 = q_offsets[b], q1 = q_offsets[b + 1];
+  if (q0 < 0 || q1 > Q || q1 < q0) {            // rows outside idx: none of them is read
+    if (tid == 0) raise_error(err, DEVERR_BOUNDS);
+    q0 = q1 = 0;
+  }
+  for (int q = q0; q < q1; ++q) {
+    const int32_t* row = idx + static_cast<size_t>(q) * topk;
+    for (int j = tid; j < topk; j += PLAN_THREADS) {
+      const int32_t pos = row[j];
+      if (pos < 0) continue;
+      const int pg = pos / DSA_TIER_PAGE;
+      if (pg >= P) {
+        raise_error(err, DEVERR_BOUNDS);
+        continue;
+      }
+      if (atomicExch(&stamp_b[pg], t) != t) {
+        const int k = atomicAdd(&s_nneed, 1);
+        if (k < D) need[k] = static_cast<uint32_t>(pg);
+      }
+    }
+  }
+  __syncthreads();
+  const int nneed = s_nneed;
+  if (nneed > D) {
+    // more distinct pages than slots: this sequence's step cannot be served
+    if (tid == 0) raise_error(err, DEVERR_CAPACITY);
+  } else {
+    for (int i = tid; i < nneed; i += PLAN_THREADS) {
+      const int pg = static_cast<int>(need[i]);
+      const int e = table_b[pg];
+      if (e >= 0) {
+        last_use[e] = t;
+        atomicAdd(&s_hits, 1);
+      } else {
+        miss[atomicAdd(&s_nmiss, 1)] = static_cast<uint32_t>(pg);
+      }
+    }
+    __syncthreads();
+    const int nmiss = s_nmiss;
+    if (nmiss > 0) {
+      uint32_t* age = need;      // the page list is spent once hits and misses are known
+      // 3. every slot's age: last use + 1 (0 = never used), or the largest
+      // value for the slots whose page this step selected (never victims)
+      {
+        constexpr int SPT = DEV_MAX_SLOTS / PLAN_THREADS;
+        int own[SPT], stp[SPT], lu[SPT];
+#pragma unroll
+        for (int k = 0; k < SPT; ++k) {
+          const int x = tid + k * PLAN_THREADS;
+          own[k] = x < D ? page_of_slot[static_cast<size_t>(b) * D + x] : -1;
+          lu[k] = x < D ? last_use[static_cast<size_t>(b) * D + x] : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < SPT; ++k) stp[k] = own[k] >= 0 ? stamp_b[own[k]] : -1;
+#pragma unroll
+        for (int k = 0; k < SPT; ++k) {
+          const int x = tid + k * PLAN_THREADS;
+          if (x < D)
+            age[x] = (own[k] >= 0 && stp[k] == t) ? 0xFFFFFFFFu : static_cast<uint32_t>(lu[k] + 1);
+        }
+      }
+      // 4. the nmiss-th smallest age T, 8 bits at a time from the top: every
+      // slot whose age is below T is a victim, and so are the `remaining`
+      // lowest-indexed slots whose age equals T
+      uint32_t prefix = 0, mask = 0;
+      int remaining = nmiss;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += PLAN_THREADS) s_hist[i] = 0;
+        __syncthreads();
+        for (int x = tid; x < D; x += PLAN_THREADS) {
+          const uint32_t a = age[x];
+          if ((a & mask) == prefix) atomicAdd(&s_hist[(a >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+          int c[8], sum = 0;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            c[k] = s_hist[tid * 8 + k];
+            sum += c[k];
+          }
+          int incl = sum;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (tid >= off) incl += y;
+          }
+          const int excl = incl - sum;
+          if (excl < remaining && remaining <= incl) {
+            int acc = excl;
+            for (int k = 0; k < 8; ++k) {
+              if (acc + c[k] >= remaining) {
+                s_digit = tid * 8 + k;
+                s_below = acc;
+                break;
+              }
+              acc += c[k];
+            }
+          }
+        }
+        __syncthreads();
+        remaining -= s_below;
+        prefix |= static_cast<uint32_t>(s_digit) << shift;
+        mask |= 0xFFu << shift;
+        __syncthreads();                       // s_digit and s_below are rewritten next pass
+      }
+      // 5. the victims' keys (age, slot): ties at T ranked in slot order by a
+      // block scan over contiguous slot ranges
+      {
+        const int chunk = (D + PLAN_THREADS - 1) / PLAN_THREADS;
+        const int x0 = min(D, tid * chunk), x1 = min(D, x0 + chunk);
+        int eq = 0;
+        for (int x = x0; x < x1; ++x) eq += age[x] == prefix;
+        const int lane = tid & 31, warp = tid >> 5;
+        int v = eq;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, v, off);
+          if (lane >= off) v += y;
+        }
+        if (lane == 31) s_wsum[warp] = v;
+        if (tid == 0) s_nvict = 0;
+        __syncthreads();
+        if (warp == 0) {
+          const int w0 = s_wsum[lane];
+          int w = w0;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += y;
+          }
+          s_wsum[lane] = w - w0;
+        }
+        __syncthreads();
+        int rank = s_wsum[warp] + v - eq;
+        for (int x = x0; x < x1; ++x) {
+          const uint32_t a = age[x];
+          bool take = a < prefix;
+          if (a == prefix) take = rank++ < remaining;
+          if (take) keys[atomicAdd(&s_nvict, 1)] = (static_cast<uint64_t>(a) << 32) | static_cast<uint32_t>(x);
+        }
+      }
+      const int Nv = pow2_dev(nmiss);
+      __syncthreads();
+      for (int i = nmiss + tid; i < Nv; i += PLAN_THREADS) {
+        keys[i] = ~0ull;
+        miss[i] = 0xFFFFFFFFu;
+      }
+      __syncthreads();
+      block_bitonic_sort(keys, Nv);
+      block_bitonic_sort(miss, Nv);
+      if (tid == 0) s_base = atomicAdd(&hdr[0], nmiss);
+      __syncthreads();
+      for (int i = tid; i < nmiss; i += PLAN_THREADS) {
+        const int x = static_cast<int>(keys[i] & 0xFFFFFFFFu);
+        const int pg = static_cast<int>(miss[i]);
+        const int gs = b * D + x;
+        const int old = page_of_slot[gs];
+        if (old >= 0) {
+          table_b[old] = -1;
+          atomicAdd(&hdr[3], 1);
+        }
+        page_of_slot[gs] = pg;
+        table_b[pg] = gs;
+        last_use[gs] = t;
+        const int c = s_base + i;
+        copies[3 * c] = b * P + pg;
+        copies[3 * c + 1] = gs;
+        copies[3 * c + 2] = old >= 0 ? b * P + old : -1;
+      }
+    }
+    if (tid == 0) {
+      atomicAdd(&hdr[1], s_hits);
+      atomicAdd(&hdr[2], nmiss);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(&hdr[5], 1) == static_cast<int>(gridDim.x) - 1) {
+      hdr[4] = t + 1;
+      hdr[5] = 0;
+    }
+  }
+}
+
+// pinned host memory the device can address over [p, p + pages * page bytes)
+bool host_cache_device_ptr(const void* p, int64_t pages, const void** dptr) {
+  cudaPointerAttributes a0, a1;
+  const uint8_t* first = static_cast<const uint8_t*>(p);
+  const uint8_t* last = first + pages * static_cast<int64_t>(TIER_PAGE_BYTES) - 1;
+  if (cudaPointerGetAttributes(&a0, first) != cudaSuccess ||
+      cudaPointerGetAttributes(&a1, last) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer ||
+      !a1.devicePointer ||
+      static_cast<const uint8_t*>(a1.devicePointer) - static_cast<const uint8_t*>(a0.devicePointer) !=
+          last - first)
+    return false;
+  *dptr = a0.devicePointer;
+  return true;
+}
+
+bool is_device_memory(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice;
 }
 
 }  // namespace
@@ -310,29 +613,98 @@ dsa_status dsa_tier_fetch(const void* host_cache, int64_t host_pages, void* dev_
   if (n == 0) return DSA_OK;
   // the host cache must be pinned host memory the device can address, over
   // its whole extent (a pageable pointer would fault the kernel)
-  cudaPointerAttributes a0, a1;
-  const uint8_t* first = static_cast<const uint8_t*>(host_cache);
-  const uint8_t* last = first + host_pages * static_cast<int64_t>(TIER_PAGE_BYTES) - 1;
-  if (cudaPointerGetAttributes(&a0, first) != cudaSuccess ||
-      cudaPointerGetAttributes(&a1, last) != cudaSuccess) {
-    cudaGetLastError();
+  const void* hdev = nullptr;
+  if (!host_cache_device_ptr(host_cache, host_pages, &hdev) || !is_device_memory(dev_pool))
     return DSA_ERR_INVALID_ARG;
-  }
-  if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer ||
-      !a1.devicePointer ||
-      static_cast<const uint8_t*>(a1.devicePointer) - static_cast<const uint8_t*>(a0.devicePointer) !=
-          last - first)
-    return DSA_ERR_INVALID_ARG;
-  cudaPointerAttributes ad;
-  if (cudaPointerGetAttributes(&ad, dev_pool) != cudaSuccess || ad.type != cudaMemoryTypeDevice) {
-    cudaGetLastError();
-    return DSA_ERR_INVALID_ARG;
-  }
   const int grid = std::min(n, 8 * device_sm_count());
   tier_fetch_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(a0.devicePointer), static_cast<uint4*>(dev_pool), copies, n,
+      static_cast<const uint4*>(hdev), static_cast<uint4*>(dev_pool), copies, n, nullptr,
       host_pages, dev_pages, page_table, static_cast<uint32_t*>(ws));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+size_t dsa_tier_dev_state_bytes(int B, int dev_slots, int max_pages) {
+  if (!tier_sizes_ok(B, dev_slots, max_pages) || dev_slots > DEV_MAX_SLOTS) return 0;
+  return dev_layout(B, dev_slots, max_pages).total;
+}
+
+dsa_status dsa_tier_dev_init(void* dev_state, size_t state_bytes, int B, int dev_slots,
+                             int max_pages, int32_t* page_table, void* stream) {
+  if (!dev_state || !page_table) return DSA_ERR_INVALID_ARG;
+  if (!tier_sizes_ok(B, dev_slots, max_pages) || dev_slots > DEV_MAX_SLOTS)
+    return DSA_ERR_UNSUPPORTED;
+  const DevLayout L = dev_layout(B, dev_slots, max_pages);
+  if (state_bytes < L.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(dev_state);
+  // counters and step 0; every stamp, slot owner and last use -1; every page absent
+  if (cudaMemsetAsync(base + L.hdr, 0, 64, st) != cudaSuccess ||
+      cudaMemsetAsync(base + L.stamp, 0xFF, L.copies - L.stamp, st) != cudaSuccess ||
+      cudaMemsetAsync(page_table, 0xFF, static_cast<size_t>(B) * max_pages * 4, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status dsa_tier_swap_in(void* dev_state, size_t state_bytes, int B, int dev_slots,
+                            int max_pages, const int32_t* idx, int Q, int topk,
+                            const int32_t* q_offsets, int32_t* page_table,
+                            const void* host_cache, void* dev_pool, void* ws, void* stream) {
+  if (!dev_state || !idx || !q_offsets || !page_table || !host_cache || !dev_pool || !ws)
+    return DSA_ERR_INVALID_ARG;
+  if (!tier_sizes_ok(B, dev_slots, max_pages) || dev_slots > DEV_MAX_SLOTS)
+    return DSA_ERR_UNSUPPORTED;
+  if (Q <= 0 || topk <= 0 || topk > DSA_MAX_TOPK) return DSA_ERR_INVALID_ARG;
+  const DevLayout L = dev_layout(B, dev_slots, max_pages);
+  if (state_bytes < L.total) return DSA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(host_cache) & 15u) || (reinterpret_cast<uintptr_t>(dev_pool) & 15u))
+    return DSA_ERR_INVALID_ARG;
+  const int64_t host_pages = static_cast<int64_t>(B) * max_pages;
+  const int64_t dev_pages = static_cast<int64_t>(B) * dev_slots;
+  const void* hdev = nullptr;
+  if (!host_cache_device_ptr(host_cache, host_pages, &hdev) || !is_device_memory(dev_pool) ||
+      !is_device_memory(dev_state))
+    return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(dev_state);
+  int32_t* hdr = reinterpret_cast<int32_t*>(base + L.hdr);
+  int32_t* copies = reinterpret_cast<int32_t*>(base + L.copies);
+  const int N = pow2_at_least(dev_slots);
+  const size_t smem = static_cast<size_t>(N) * 8 + static_cast<size_t>(dev_slots) * 4 + static_cast<size_t>(N) * 4;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(tier_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(DEV_MAX_SLOTS) * 16) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  if (cudaMemsetAsync(hdr, 0, 16, st) != cudaSuccess) return DSA_ERR_CUDA;   // this step's counters
+  tier_plan_kernel<<<B, PLAN_THREADS, smem, st>>>(
+      hdr, reinterpret_cast<int32_t*>(base + L.stamp), reinterpret_cast<int32_t*>(base + L.page_of_slot),
+      reinterpret_cast<int32_t*>(base + L.last_use), copies, idx, Q, topk, q_offsets, dev_slots,
+      max_pages, page_table, static_cast<uint32_t*>(ws));
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  tier_fetch_kernel<<<8 * device_sm_count(), 256, 0, st>>>(
+      static_cast<const uint4*>(hdev), static_cast<uint4*>(dev_pool), copies,
+      static_cast<int>(dev_pages), hdr, host_pages, dev_pages, nullptr, static_cast<uint32_t*>(ws));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_tier_dev_stats(const void* dev_state, int64_t* stats, void* stream) {
+  if (!dev_state || !stats) return DSA_ERR_INVALID_ARG;
+  int32_t h[5];
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemcpy(h, dev_state, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  for (int i = 0; i < 5; ++i) stats[i] = h[i];
+  return DSA_OK;
+}
+
+const int32_t* dsa_tier_dev_copies(const void* dev_state, int B, int dev_slots, int max_pages) {
+  if (!dev_state || !tier_sizes_ok(B, dev_slots, max_pages)) return nullptr;
+  return reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(dev_state) +
+                                          dev_layout(B, dev_slots, max_pages).copies);
 }
 
 }  // extern "C"

@@ -118,3 +118,72 @@ def test_fetch_skips_and_flags_copies_outside_the_caches():
         dsa.dsa_check_error(ws)
     assert e.value.status == 4
     assert torch.equal(pool[1].cpu(), host[2]) and bool((pool[0] == 0).all())
+
+
+# ------------------------------------------------------------------ device planner
+def _trace(rng, B, P, steps, hot, churn, rows_per_seq, topk):
+    hot_sets = [list(rng.choice(P, hot, replace=False)) for _ in range(B)]
+    out = []
+    for _ in range(steps):
+        rows = []
+        for b in range(B):
+            for _ in range(churn):
+                hot_sets[b][int(rng.integers(hot))] = int(rng.integers(P))
+            for _ in range(rows_per_seq):
+                rows.append(_local_rows(rng, np.array(hot_sets[b]), P * PT, topk))
+        out.append(np.stack(rows))
+    return out
+
+
+@pytest.mark.parametrize("B,D,P,hot,churn,rows", [(3, 64, 400, 50, 6, 2), (2, 1024, 4000, 700, 60, 1)])
+def test_device_planner_matches_oracle(B, D, P, hot, churn, rows):
+    rng = np.random.default_rng(D)
+    topk = 256 if D == 64 else 2048
+    host = torch.randn(B * P, PT, 576).to(torch.bfloat16).pin_memory()
+    pool = torch.full((B * D, PT, 576), float("nan"), dtype=torch.bfloat16, device=DEV)
+    pt = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    st = dsa.tier_dev_state(B, D, P, pt)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    q_off_h = torch.arange(B + 1, dtype=torch.int32) * rows
+    q_off = q_off_h.to(DEV)
+    tier = O.TierOracle(B, D, P)
+    host_bits = np_bits(host)
+    for step, idx_np in enumerate(_trace(rng, B, P, 12, hot, churn, rows, topk)):
+        idx = torch.from_numpy(idx_np).to(DEV)
+        dsa.dsa_tier_swap_in(st, B, D, P, idx, q_off, pt, host, pool, ws)
+        (n, hits, misses, ev), steps = dsa.dsa_tier_dev_stats(st)
+        dsa.dsa_check_error(ws)
+        per_seq = [[list(r) for r in idx_np[b * rows:(b + 1) * rows]] for b in range(B)]
+        table, copies, h_o, m_o, e_o = tier.step(per_seq)
+        assert steps == step + 1
+        assert (n, hits, misses, ev) == (len(copies), h_o, m_o, e_o)
+        assert pt.cpu().tolist() == table
+        got = sorted(tuple(x) for x in dsa.dsa_tier_dev_copies(st, B, D, P, n).cpu().tolist())
+        assert got == sorted(copies)
+        ptn = pt.cpu().numpy()
+        pool_bits = np_bits(pool)
+        for b in range(B):
+            res = np.flatnonzero(ptn[b] >= 0)
+            assert np.array_equal(pool_bits[ptn[b, res]], host_bits[b * P + res])
+
+
+def test_device_planner_refuses_a_step_beyond_its_slots():
+    B, D, P = 2, 8, 100
+    host = torch.randn(B * P, PT, 576).to(torch.bfloat16).pin_memory()
+    pool = torch.zeros(B * D, PT, 576, dtype=torch.bfloat16, device=DEV)
+    pt = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    st = dsa.tier_dev_state(B, D, P, pt)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    q_off = torch.arange(B + 1, dtype=torch.int32, device=DEV)
+    ok = torch.full((B, 16), -1, dtype=torch.int32)
+    ok[:, :3] = torch.tensor([0, 16, 32])
+    dsa.dsa_tier_swap_in(st, B, D, P, ok.to(DEV), q_off, pt, host, pool, ws)
+    dsa.dsa_check_error(ws)
+    before = pt.clone()
+    bad = ok.clone()
+    bad[0] = torch.arange(16, dtype=torch.int32) * 16          # 16 distinct pages for 8 slots
+    dsa.dsa_tier_swap_in(st, B, D, P, bad.to(DEV), q_off, pt, host, pool, ws)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.dsa_check_error(ws)
+    assert e.value.status == 2
+    assert torch.equal(pt[0], before[0])                         # sequence 0 was left as it was
