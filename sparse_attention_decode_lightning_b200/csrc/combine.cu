@@ -2,10 +2,13 @@
 //   LSE = ln sum_c exp(LSE_c),  O = sum_c exp(LSE_c - LSE) O_c,
 // parts with LSE_c = -inf (no selected token) get weight 0; if every part is
 // empty O = 0 and LSE = -inf.  H heads per query (128, or GLM-5.2's 64).
-// One CTA of 256 threads per (query, 8 heads): a
-// warp per head, 16 outputs per thread; the split weights are recomputed by
-// every thread from the S partial LSEs (L1-resident).  One CTA per head (4096
-// CTAs of 128 threads for 32 queries) spent its time in CTA scheduling.
+// One CTA of 256 threads per (query, 8 heads, part of the 512 outputs): a
+// warp per head; the split weights are recomputed by every thread from the S
+// partial LSEs (L1-resident).  With few queries the outputs are cut into 2 or
+// 4 parts (grid.y) so that the grid still covers the SMs: 4 queries x 64
+// heads were 32 CTAs, each reading 16 partials of 8 x 512 floats.  One CTA per
+// head (4096 CTAs of 128 threads for 32 queries) spent its time in CTA
+// scheduling.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,8 +25,9 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
                                                                float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();                                   // the partials come from the previous kernel
-  // CTA: query q, heads [h0, h0 + 8); thread: head h0 + tid / 32, outputs
-  // [16 * (tid % 32), +16) as four float4 spread 128 floats apart
+  // CTA: query q, heads [h0, h0 + 8), 128-float quarters [k0, k1) of the 512
+  // outputs; thread: head h0 + tid / 32, float4 column tid % 32 of each quarter
+  const int k0 = blockIdx.y * 4 / gridDim.y, k1 = (blockIdx.y + 1) * 4 / gridDim.y;
   const int q = blockIdx.x / (H / HEADS_PER_CTA);
   const int h = (blockIdx.x % (H / HEADS_PER_CTA)) * HEADS_PER_CTA + (threadIdx.x >> 5);
   const int c4 = threadIdx.x & 31;              // float4 column within each 128-float quarter
@@ -34,14 +38,16 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
   float4* o = reinterpret_cast<float4*>(out + qh * DSA_DIM_V) + c4;
   if (m == -INFINITY) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) o[32 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (c4 == 0) lse[qh] = -INFINITY;
+    for (int k = 0; k < 4; ++k)
+      if (k >= k0 && k < k1) o[32 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c4 == 0 && blockIdx.y == 0) lse[qh] = -INFINITY;
     return;
   }
   float tot = 0.f;
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int c = 0; c < S; ++c) {
     const float lc = lp[static_cast<size_t>(c) * H];
     if (lc == -INFINITY) continue;
@@ -51,6 +57,7 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
                           o_part + ((static_cast<size_t>(q) * S + c) * H + h) * DSA_DIM_V) + c4;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+      if (k < k0 || k >= k1) continue;
       const float4 x = v[32 * k];
       acc[k].x = fmaf(wc, x.x, acc[k].x);
       acc[k].y = fmaf(wc, x.y, acc[k].y);
@@ -61,8 +68,9 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
   const float inv = 1.f / tot;
 #pragma unroll
   for (int k = 0; k < 4; ++k)
-    o[32 * k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
-  if (c4 == 0) lse[qh] = m + logf(tot);
+    if (k >= k0 && k < k1)
+      o[32 * k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+  if (c4 == 0 && blockIdx.y == 0) lse[qh] = m + logf(tot);
 }
 
 }  // namespace
@@ -71,8 +79,12 @@ cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int 
                            float* out, float* lse, cudaStream_t st, bool pdl) {
   if (Q <= 0) return cudaSuccess;
   if (H <= 0 || H % HEADS_PER_CTA) return cudaErrorInvalidValue;
+  // cut the 512 outputs into parts until the grid covers twice the SMs
+  const int ctas = Q * (H / HEADS_PER_CTA);
+  const int sms = device_sm_count();
+  const int parts = ctas >= 2 * sms ? 1 : (2 * ctas >= 2 * sms ? 2 : 4);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(Q) * (H / HEADS_PER_CTA), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), static_cast<unsigned>(parts), 1);
   cfg.blockDim = dim3(CTHREADS, 1, 1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
