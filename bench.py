@@ -47,6 +47,8 @@ def parse():
                     help="override the workload's sequence count (small profiling cases)")
     ap.add_argument("--tier", action="store_true",
                     help="time the two-tier (HiSparse) decode path instead (one GPU)")
+    ap.add_argument("--csa", action="store_true",
+                    help="time the compressed-sparse (DeepSeek-V4 CSA) decode step instead (one GPU)")
     return ap.parse_args()
 
 
@@ -631,6 +633,94 @@ def run_tier(args):
     }
 
 
+def run_csa(args):
+    """DeepSeek-V4 CSA decode step, V4-Flash selection at 1M raw context: the
+    lightning indexer scores the 4x-compressed keys (256K per sequence), the
+    selector keeps top-512, and sparse MLA attends to the 512 compressed rows
+    plus the 128 most recent raw tokens.  32 sequences, DeepSeek-V3.2 head
+    counts (the pages give none for V4).  Only the raw pages under the window
+    are allocated: nothing else of the raw cache is read.  L2 is flushed
+    before every step."""
+    import statistics
+
+    import torch
+
+    import sparse_attention_decode_lightning_b200 as dsa
+
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    B, L_raw, ratio, topk, window = 32, 1 << 20, 4, 512, 128
+    Lc = L_raw // ratio
+    g = torch.Generator(device=dev).manual_seed(args.seed)
+    pc = Lc // 64                                   # compressed pages per sequence
+    pr_used = (window + 63) // 64 + 1               # raw pages under the window
+    num_pages = B * (pc + pr_used)
+    perm = torch.randperm(num_pages, generator=g, device=dev).to(torch.int32)
+    ct = perm[:B * pc].view(B, pc).contiguous()
+    rt = torch.full((B, L_raw // 64), -1, dtype=torch.int32, device=dev)
+    rt[:, -pr_used:] = perm[B * pc:].view(B, pr_used)
+    pool = torch.empty(num_pages, 64, 576, dtype=torch.bfloat16, device=dev)
+    for i in range(0, num_pages, 4096):
+        pool[i:i + 4096] = torch.randn(pool[i:i + 4096].shape, generator=g, device=dev)
+    q = torch.randn(B, 128, 576, generator=g, device=dev).to(torch.bfloat16)
+    keys = torch.randn(B * Lc, 128, generator=g, device=dev).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    qi = torch.randn(B, 64, 128, generator=g, device=dev).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    w = torch.randn(B, 64, generator=g, device=dev) / 8
+    so = torch.arange(B + 1, dtype=torch.int64, device=dev) * Lc
+    qo = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    vis = torch.full((B,), Lc, dtype=torch.int32, device=dev)
+    wvis = torch.full((B,), L_raw, dtype=torch.int32, device=dev)
+    idx = torch.empty(B, topk, dtype=torch.int32, device=dev)
+    out = torch.empty(B, 128, 512, device=dev)
+    lse = torch.empty(B, 128, device=dev)
+    ws = dsa.workspace(B, Lc, topk + window, 0, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1 / 192 ** 0.5
+
+    def step():
+        dsa.dsa_indexer_topk(qi, w, keys, so, qo, vis, B, Lc, topk, idx, ws, stream=stream)
+        dsa.dsa_sparse_mla_decode_window(q, pool, ct, rt, qo, vis, wvis, idx, B, window, scale,
+                                         out, lse, ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    times = {"step": [], "indexer_topk": [], "mla_window": []}
+    for _ in range(args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        dsa.dsa_indexer_topk(qi, w, keys, so, qo, vis, B, Lc, topk, idx, ws, stream=stream)
+        e[1].record(stream)
+        dsa.dsa_sparse_mla_decode_window(q, pool, ct, rt, qo, vis, wvis, idx, B, window, scale,
+                                         out, lse, ws, stream=stream)
+        e[2].record(stream)
+        torch.cuda.synchronize(dev)
+        times["indexer_topk"].append(e[0].elapsed_time(e[1]))
+        times["mla_window"].append(e[1].elapsed_time(e[2]))
+        times["step"].append(e[0].elapsed_time(e[2]))
+    dsa.dsa_check_error(ws)
+    m = {k: statistics.mean(v) for k, v in times.items()}
+    key_b = B * Lc * 128
+    gat_b = B * (topk + window) * 576 * 2
+    hbm, hbm_kind = peaks()
+    return {
+        "metric": "DeepSeek-V4 CSA decode query-tokens/s (top-512 of 4x-compressed 1M ctx + 128 window)",
+        "value": B / (m["step"] / 1e3), "unit": "query-tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": m["step"], "higher_is_better": True,
+        "dtype": "e4m3 indexer, bf16 attention, f32 accumulate", "data": "synthetic",
+        "config": {"workload": "v4flash_csa_b32_ctx1m", "B": B, "L_raw": L_raw, "ratio": ratio,
+                   "compressed_entries": Lc, "topk": topk, "window": window, "heads": 128,
+                   "l2": "256 MiB flush before every step"},
+        "stages_ms": {"indexer_topk": m["indexer_topk"], "mla_window": m["mla_window"]},
+        "step_roofline": {"bytes_per_step": key_b + gat_b, "achieved_gbs": (key_b + gat_b) / (m["step"] / 1e3) / 1e9,
+                          "peak": hbm, "peak_source": hbm_kind,
+                          "frac": (key_b + gat_b) / (m["step"] / 1e3) / 1e9 / hbm},
+    }
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -643,6 +733,10 @@ def main():
     if args.tier:
         if rank == 0:
             print(json.dumps(run_tier(args)), flush=True)
+        return
+    if args.csa:
+        if rank == 0:
+            print(json.dumps(run_csa(args)), flush=True)
         return
     if world > 1:
         import datetime

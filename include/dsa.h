@@ -205,6 +205,33 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
                                  void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Sparse MLA decode with a sliding window, DeepSeek-V4's CSA  ("大语言模型结构
+ * 总览", section 2.3 DeepSeek-V4: the KV cache is compressed 4x along the
+ * sequence, DSA keeps the top-1024 (Pro) or top-512 (Flash) compressed
+ * entries, and a 128-token sliding window of raw tokens is attended as well).
+ * Each query attends, in one softmax, to
+ *   the topk selected entries of idx: positions in the compressed cache,
+ *     mapped through page_table and checked against q_vis as above, and
+ *   the `window` most recent raw tokens: positions win_vis[q]-window ..
+ *     win_vis[q]-1 (those below 0 are skipped), mapped through win_page_table
+ *     [B,win_max_pages] into the same kv_pool.
+ *   win_vis  DEVICE int32 [Q]: raw tokens visible to each query
+ *   topk + window <= DSA_MAX_TOPK; window = 0 is dsa_sparse_mla_decode.
+ * How the compressed entries are formed is the model's (learned) business;
+ * the call takes them as latent rows.  Other arguments, layouts, precision
+ * and errors as in dsa_sparse_mla_decode; ws: at least
+ * dsa_workspace_bytes(Q, 1, topk + window, num_splits) bytes.
+ */
+dsa_status dsa_sparse_mla_decode_window(const void* q, const void* kv_pool, int num_pages,
+                                        int page_size, const int32_t* page_table, int max_pages,
+                                        const int32_t* win_page_table, int win_max_pages,
+                                        const int32_t* q_offsets, const int32_t* q_vis,
+                                        const int32_t* win_vis, const int32_t* idx, int B, int Q,
+                                        int heads, int topk, int window, float scale,
+                                        int num_splits, float* out, float* lse, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/*
  * Sparse MLA decode that allocates nothing and takes no workspace.  The
  * pages have no counterpart of this call; it exists for callers that cannot
  * hand the library device memory: a serving engine whose allocator already

@@ -46,6 +46,8 @@ SIGNATURES = {
                                    _P, _P, _SZ, _P]),
     "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F,
                                            _I, _P, _P, _P]),
+    "dsa_sparse_mla_decode_window": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _I, _I,
+                                          _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "dsa_lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                              _PP, _PP, _I, _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
@@ -190,6 +192,19 @@ def dsa_sparse_mla_decode_noalloc(q, kv_pool, page_table, q_offsets, q_vis, idx,
         _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1],
         float(scale), num_splits, _ptr(out), _ptr(lse), _stream(stream)),
         "dsa_sparse_mla_decode_noalloc")
+
+
+def dsa_sparse_mla_decode_window(q, kv_pool, page_table, win_page_table, q_offsets, q_vis,
+                                 win_vis, idx, B, window, scale, out, lse, ws, num_splits=0,
+                                 stream=None):
+    """Sparse MLA over the selected compressed entries plus a sliding window of
+    raw tokens (DeepSeek-V4 CSA); see include/dsa.h."""
+    _check(lib().dsa_sparse_mla_decode_window(
+        _ptr(q), _ptr(kv_pool), kv_pool.shape[0], kv_pool.shape[1], _ptr(page_table),
+        page_table.shape[1], _ptr(win_page_table), win_page_table.shape[1], _ptr(q_offsets),
+        _ptr(q_vis), _ptr(win_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1], window,
+        float(scale), num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+        "dsa_sparse_mla_decode_window")
 
 
 def dsa_lse_combine(o_parts, lse_parts, out, lse, stream=None):

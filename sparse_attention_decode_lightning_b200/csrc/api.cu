@@ -14,7 +14,9 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                    const int32_t* q_offsets, const int32_t* q_vis,
                                    const int32_t* idx, int B, int Q, int H, int topk,
                                    float scale, int S, float* out, float* lse, float* o_part,
-                                   float* l_part, uint32_t* err, cudaStream_t st, bool pdl);
+                                   float* l_part, uint32_t* err, cudaStream_t st, bool pdl,
+                                   const int32_t* win_page_table, int win_max_pages,
+                                   const int32_t* win_vis, int window);
 
 namespace {
 
@@ -145,14 +147,17 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages, int 
                          const int32_t* page_table, int max_pages, const int32_t* q_offsets,
                          const int32_t* q_vis, const int32_t* idx, int B, int Q, int H,
                          int topk, float scale, int S, float* out, float* lse, void* ws,
-                         const WsLayout& L, cudaStream_t st, bool pdl) {
+                         const WsLayout& L, cudaStream_t st, bool pdl,
+                         const int32_t* win_page_table = nullptr, int win_max_pages = 0,
+                         const int32_t* win_vis = nullptr, int window = 0) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* o_part = ws_ptr<float>(ws, L.o_part);
   float* l_part = ws_ptr<float>(ws, L.l_part);
   cudaError_t e = launch_sparse_mla(static_cast<const __nv_bfloat16*>(q),
                                     static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
-                                    page_size, page_table, max_pages, q_offsets, q_vis, idx, B, Q, H, topk,
-                                    scale, S, out, lse, o_part, l_part, err, st, pdl);
+                                    page_size, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
+                                    H, topk, scale, S, out, lse, o_part, l_part, err, st, pdl,
+                                    win_page_table, win_max_pages, win_vis, window);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (S > 1) {
     e = launch_combine(o_part, l_part, Q, S, H, out, lse, st, true);
@@ -180,10 +185,12 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               const int32_t* q_offsets, const int32_t* q_vis,
                               const int32_t* idx, int B, int Q, int H, int topk, float scale, int S,
                               float* out, float* lse, float* o_part, float* l_part,
-                              uint32_t* err, cudaStream_t st, bool pdl) {
+                              uint32_t* err, cudaStream_t st, bool pdl,
+                              const int32_t* win_page_table, int win_max_pages,
+                              const int32_t* win_vis, int window) {
   return launch_sparse_mla_tc(q, pool, num_pages, page_size, page_table, max_pages, q_offsets,
                               q_vis, idx, B, Q, H, topk, scale, S, out, lse, o_part, l_part, err,
-                              st, pdl);
+                              st, pdl, win_page_table, win_max_pages, win_vis, window);
 }
 
 }  // namespace dsa
@@ -289,6 +296,31 @@ dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pag
   return do_sparse_mla(q, kv_pool, num_pages, page_size, page_table, max_pages, q_offsets, q_vis,
                        idx, B, Q, heads, topk, scale, L.S, out, lse, ws, L,
                        static_cast<cudaStream_t>(stream), false);
+}
+
+dsa_status dsa_sparse_mla_decode_window(const void* q, const void* kv_pool, int num_pages,
+                                        int page_size, const int32_t* page_table, int max_pages,
+                                        const int32_t* win_page_table, int win_max_pages,
+                                        const int32_t* q_offsets, const int32_t* q_vis,
+                                        const int32_t* win_vis, const int32_t* idx, int B, int Q,
+                                        int heads, int topk, int window, float scale,
+                                        int num_splits, float* out, float* lse, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  if (!q_offsets || !q_vis || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || topk <= 0 || window < 0) return DSA_ERR_INVALID_ARG;
+  if (window > 0 && (!win_page_table || !win_vis || win_max_pages <= 0)) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk + window > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
+  dsa_status s = mla_checks(q, kv_pool, num_pages, page_size, page_table, max_pages, idx, out, lse,
+                            scale, heads);
+  if (s != DSA_OK) return s;
+  WsLayout L;
+  if (!ws_layout(Q, 1, topk + window, num_splits, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  return do_sparse_mla(q, kv_pool, num_pages, page_size, page_table, max_pages, q_offsets, q_vis,
+                       idx, B, Q, heads, topk, scale, L.S, out, lse, ws, L,
+                       static_cast<cudaStream_t>(stream), false, win_page_table, win_max_pages,
+                       win_vis, window);
 }
 
 dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, int heads,

@@ -90,6 +90,13 @@ struct MlaTcArgs {
   int max_pages;
   int num_pages;
   int page_shift;                              // log2 of the tokens per cache page
+  // sliding window (DeepSeek-V4 CSA): the `window` most recent raw tokens of
+  // the query, from a second page table into the same pool, follow the topk
+  // selected entries (window = 0: none)
+  const int32_t* win_page_table;
+  int win_max_pages;
+  const int32_t* win_vis;
+  int window;
   const int32_t* q_offsets;
   const int32_t* q_vis;
   const int32_t* idx;
@@ -176,9 +183,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int b = seq_of_query(a.q_offsets, a.B, q);
   int vis = a.q_vis[q];
   if (vis < 0) vis = 0;
-  const int per = (a.topk + a.S - 1) / a.S;
+  const int total = a.topk + a.window;             // selected entries, then the window
+  const int per = (total + a.S - 1) / a.S;
   const int r0 = split * per;
-  const int r1 = min(a.topk, r0 + per);
+  const int r1 = min(total, r0 + per);
   const int nrows = r1 > r0 ? r1 - r0 : 0;
   const int ntiles = (nrows + NR - 1) / NR;
 
@@ -214,18 +222,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   // many independent loads in flight (-1 = padding or out of range)
   {
     constexpr int PER = (DSA_MAX_TOPK + THREADS - 1) / THREADS;
+    int wvis = a.window > 0 ? a.win_vis[q] : 0;
+    if (wvis < 0) wvis = 0;
     int sv[PER];
+    bool win[PER];
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int j = r0 + tid + k * THREADS;
-      sv[k] = j < r1 ? a.idx[static_cast<size_t>(q) * a.topk + j] : -1;
+      win[k] = j >= a.topk;
+      if (j >= r1) sv[k] = -1;
+      else if (!win[k]) sv[k] = a.idx[static_cast<size_t>(q) * a.topk + j];
+      else sv[k] = max(-1, wvis - a.window + (j - a.topk));   // before token 0: none
     }
     int pg[PER];
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int sx = sv[k];
-      const bool ok = sx >= 0 && sx < vis && (sx >> a.page_shift) < a.max_pages;
-      pg[k] = ok ? a.page_table[static_cast<size_t>(b) * a.max_pages + (sx >> a.page_shift)] : -1;
+      const int32_t* tab = win[k] ? a.win_page_table : a.page_table;
+      const int mp = win[k] ? a.win_max_pages : a.max_pages;
+      const bool ok = sx >= 0 && sx < (win[k] ? wvis : vis) && (sx >> a.page_shift) < mp;
+      pg[k] = ok ? tab[static_cast<size_t>(b) * mp + (sx >> a.page_shift)] : -1;
     }
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
@@ -579,7 +595,9 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  const int32_t* q_offsets, const int32_t* q_vis,
                                  const int32_t* idx, int B, int Q, int H, int topk, float scale,
                                  int S, float* out, float* lse, float* o_part, float* l_part,
-                                 uint32_t* err, cudaStream_t st, bool pdl) {
+                                 uint32_t* err, cudaStream_t st, bool pdl,
+                                 const int32_t* win_page_table, int win_max_pages,
+                                 const int32_t* win_vis, int window) {
   if (Q <= 0) return cudaSuccess;
   if (H != 128 && H != 64) return cudaErrorInvalidValue;
   int page_shift = 0;
@@ -608,7 +626,8 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                        static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4, 32,
                        static_cast<uint32_t>(H)))
     return cudaErrorInvalidValue;
-  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, page_shift, q_offsets, q_vis, idx, B, Q, topk, S,
+  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, page_shift, win_page_table, win_max_pages,
+              win_vis, window, q_offsets, q_vis, idx, B, Q, topk, S,
               scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * Q * S), 1, 1);

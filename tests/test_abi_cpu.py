@@ -111,6 +111,13 @@ def test_host_checks_reject_bad_arguments_without_a_device():
                                        ctypes.c_float(0.07), 0, fake, fake, fake, 1 << 30,
                                        null) == 2
         assert L.dsa_lse_combine(fake, fake, 1, 2, h, fake, fake, null) == 2
+    # window mode: window without its tables, and more rows than the selector's maximum
+    assert L.dsa_sparse_mla_decode_window(fake, fake, 10, 64, fake, 4, null, 4, fake, fake, fake,
+                                          fake, 1, 1, 128, 512, 128, ctypes.c_float(0.07), 0,
+                                          fake, fake, fake, 1 << 30, null) == 1
+    assert L.dsa_sparse_mla_decode_window(fake, fake, 10, 64, fake, 4, fake, 4, fake, fake, fake,
+                                          fake, 1, 1, 128, 2048, 128, ctypes.c_float(0.07), 0,
+                                          fake, fake, fake, 1 << 30, null) == 2
     # decode step: no layers, zero share group
     PP = ctypes.POINTER(ctypes.c_void_p)
     arr = (ctypes.c_void_p * 1)(1 << 20)
