@@ -47,6 +47,8 @@ def parse():
                     help="override the workload's sequence count (small profiling cases)")
     ap.add_argument("--tier", action="store_true",
                     help="time the two-tier (HiSparse) decode path instead (one GPU)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the sparse MLA over an e4m3 latent cache against bf16 (one GPU)")
     ap.add_argument("--csa", action="store_true",
                     help="time the compressed-sparse (DeepSeek-V4 CSA) decode step instead (one GPU)")
     return ap.parse_args()
@@ -721,6 +723,64 @@ def run_csa(args):
     }
 
 
+def run_fp8(args):
+    """Sparse MLA over the same selected rows of the batch-32 128K workload,
+    with the latent cache in bf16 (1152 B a row) and in e4m3 (576 B a row, one
+    per-tensor scale; the kernel widens rows to bf16 on chip).  Indices come
+    from the library's indexer and selector; L2 is flushed before each call."""
+    import statistics
+
+    import torch
+
+    import sparse_attention_decode_lightning_b200 as dsa
+    from synth import get_workload, make_inputs
+
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    inp = make_inputs(get_workload(DEFAULT_WORKLOAD), seed=args.seed, device=dev, layers_to_make=1)
+    Q, ix = inp.Q, inp.indexer[0]
+    idx = torch.empty(Q, inp.topk, dtype=torch.int32, device=dev)
+    ws = dsa.workspace(Q, inp.max_len, inp.topk, 0, device=dev)
+    dsa.dsa_indexer_topk(ix["q_idx"], ix["w"], ix["k_idx"], inp.seq_offsets, inp.q_offsets,
+                         inp.q_vis, inp.B, inp.max_len, inp.topk, idx, ws)
+    pool = inp.layers[0]["pool"]
+    codes = pool.to(torch.float8_e4m3fn).view(torch.uint8)
+    out = torch.empty(Q, inp.heads, 512, device=dev)
+    lse = torch.empty(Q, inp.heads, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    calls = {
+        "bf16": lambda: dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], pool, inp.page_table,
+                                                  inp.q_offsets, inp.q_vis, idx, inp.B, inp.scale,
+                                                  out, lse, ws, stream=stream),
+        "e4m3": lambda: dsa.dsa_sparse_mla_decode_fp8(inp.layers[0]["q"], codes, 1.0, inp.page_table,
+                                                      inp.q_offsets, inp.q_vis, idx, inp.B,
+                                                      inp.scale, out, lse, ws, stream=stream),
+    }
+    res = {}
+    for name, fn in calls.items():
+        ts = []
+        for i in range(max(3, args.warmup) + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= max(3, args.warmup):
+                ts.append(a.elapsed_time(b) * 1e3)
+        res[name] = statistics.mean(ts)
+    dsa.dsa_check_error(ws)
+    rows = Q * inp.topk
+    return {
+        "metric": "sparse MLA + merge time, batch-32 128K selected rows: bf16 vs e4m3 latent cache",
+        "value": res["e4m3"], "unit": "us", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup), "data": "synthetic",
+        "config": {"workload": DEFAULT_WORKLOAD, "rows": rows, "l2": "256 MiB flush before each call"},
+        "us": res, "gather_bytes": {"bf16": rows * 1152, "e4m3": rows * 576},
+    }
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -737,6 +797,10 @@ def main():
     if args.csa:
         if rank == 0:
             print(json.dumps(run_csa(args)), flush=True)
+        return
+    if args.fp8:
+        if rank == 0:
+            print(json.dumps(run_fp8(args)), flush=True)
         return
     if world > 1:
         import datetime

@@ -232,6 +232,25 @@ dsa_status dsa_sparse_mla_decode_window(const void* q, const void* kv_pool, int 
                                         size_t ws_bytes, void* stream);
 
 /*
+ * Sparse MLA decode over an FP8 latent cache  ("GLM-5.2 推理部署": MLA plus an
+ * FP8 KV cache, --kv-cache-dtype fp8_e4m3, to fit 1M context).
+ *   kv_pool   e4m3 [num_pages,page_size,576]: one byte per value; the latent
+ *             row is the code's value times kv_scale (one scale for the
+ *             whole cache, > 0)
+ * Everything else as in dsa_sparse_mla_decode.  The gather widens each e4m3
+ * row exactly to bf16 on chip (every e4m3 value is a bf16 value) for the
+ * same bf16 tensor-core products; kv_scale multiplies the scores (with
+ * `scale`) and the output, so nothing is rounded that the bf16 call would
+ * not round.  A row is 576 bytes instead of 1152.
+ */
+dsa_status dsa_sparse_mla_decode_fp8(const void* q, const void* kv_pool, float kv_scale,
+                                     int num_pages, int page_size, const int32_t* page_table,
+                                     int max_pages, const int32_t* q_offsets, const int32_t* q_vis,
+                                     const int32_t* idx, int B, int Q, int heads, int topk,
+                                     float scale, int num_splits, float* out, float* lse, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/*
  * Sparse MLA decode that allocates nothing and takes no workspace.  The
  * pages have no counterpart of this call; it exists for callers that cannot
  * hand the library device memory: a serving engine whose allocator already

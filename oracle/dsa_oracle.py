@@ -50,7 +50,7 @@ DI = 128
 
 __all__ = [
     "e4m3_table", "e4m3_decode", "bf16_decode",
-    "indexer_scores", "topk_select", "latent_rows",
+    "indexer_scores", "topk_select", "latent_rows", "latent_rows_e4m3",
     "sparse_mla", "sparse_mla_split", "lse_combine",
     "query_step", "decode_step",
 ]
@@ -136,6 +136,17 @@ def latent_rows(pool: np.ndarray, page_table_row: np.ndarray, positions: np.ndar
     positions = np.asarray(positions, dtype=np.int64)
     pages = np.asarray(page_table_row, dtype=np.int64)[positions // PAGE]
     return bf16_decode(pool[pages, positions % PAGE])
+
+
+def latent_rows_e4m3(pool: np.ndarray, page_table_row: np.ndarray, positions: np.ndarray,
+                     kv_scale: float, page_size: int = PAGE) -> np.ndarray:
+    """Selected rows of an FP8 latent cache (the deploy page's fp8_e4m3 KV cache,
+    "GLM-5.2 推理部署"): e4m3 codes [P,page_size,576] through the page table,
+    decoded exactly and multiplied by the cache's one scale, as float64 [n,576]."""
+    positions = np.asarray(positions, dtype=np.int64)
+    pages = np.asarray(page_table_row, dtype=np.int64)[positions // page_size]
+    codes = pool[pages, positions % page_size]
+    return e4m3_decode(codes) * float(kv_scale)
 
 
 def sparse_mla(q: np.ndarray, rows: np.ndarray, scale: float) -> Tuple[np.ndarray, np.ndarray]:

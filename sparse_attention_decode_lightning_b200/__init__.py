@@ -48,6 +48,8 @@ SIGNATURES = {
                                            _I, _P, _P, _P]),
     "dsa_sparse_mla_decode_window": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _I, _I,
                                           _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
+    "dsa_sparse_mla_decode_fp8": (_I, [_P, _P, _F, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F,
+                                       _I, _P, _P, _P, _SZ, _P]),
     "dsa_lse_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "dsa_decode_step": (_I, [_I, _I, _I, _PP, _PP, _PP, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                              _PP, _PP, _I, _I, _PP, _I, _F, _I, _PP, _PP, _P, _P, _SZ, _P]),
@@ -205,6 +207,17 @@ def dsa_sparse_mla_decode_window(q, kv_pool, page_table, win_page_table, q_offse
         _ptr(q_vis), _ptr(win_vis), _ptr(idx), B, q.shape[0], q.shape[1], idx.shape[1], window,
         float(scale), num_splits, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
         "dsa_sparse_mla_decode_window")
+
+
+def dsa_sparse_mla_decode_fp8(q, kv_pool, kv_scale, page_table, q_offsets, q_vis, idx, B, scale,
+                              out, lse, ws, num_splits=0, stream=None):
+    """Sparse MLA over an e4m3 latent cache (uint8 [pages,page_size,576]) with one
+    per-tensor scale; see include/dsa.h."""
+    _check(lib().dsa_sparse_mla_decode_fp8(
+        _ptr(q), _ptr(kv_pool), float(kv_scale), kv_pool.shape[0], kv_pool.shape[1],
+        _ptr(page_table), page_table.shape[1], _ptr(q_offsets), _ptr(q_vis), _ptr(idx), B,
+        q.shape[0], q.shape[1], idx.shape[1], float(scale), num_splits, _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream)), "dsa_sparse_mla_decode_fp8")
 
 
 def dsa_lse_combine(o_parts, lse_parts, out, lse, stream=None):

@@ -16,7 +16,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                    float scale, int S, float* out, float* lse, float* o_part,
                                    float* l_part, uint32_t* err, cudaStream_t st, bool pdl,
                                    const int32_t* win_page_table, int win_max_pages,
-                                   const int32_t* win_vis, int window);
+                                   const int32_t* win_vis, int window, bool kv8, float kv_scale);
 
 namespace {
 
@@ -149,7 +149,8 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages, int 
                          int topk, float scale, int S, float* out, float* lse, void* ws,
                          const WsLayout& L, cudaStream_t st, bool pdl,
                          const int32_t* win_page_table = nullptr, int win_max_pages = 0,
-                         const int32_t* win_vis = nullptr, int window = 0) {
+                         const int32_t* win_vis = nullptr, int window = 0, bool kv8 = false,
+                         float kv_scale = 1.f) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* o_part = ws_ptr<float>(ws, L.o_part);
   float* l_part = ws_ptr<float>(ws, L.l_part);
@@ -157,7 +158,7 @@ dsa_status do_sparse_mla(const void* q, const void* kv_pool, int num_pages, int 
                                     static_cast<const __nv_bfloat16*>(kv_pool), num_pages,
                                     page_size, page_table, max_pages, q_offsets, q_vis, idx, B, Q,
                                     H, topk, scale, S, out, lse, o_part, l_part, err, st, pdl,
-                                    win_page_table, win_max_pages, win_vis, window);
+                                    win_page_table, win_max_pages, win_vis, window, kv8, kv_scale);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (S > 1) {
     e = launch_combine(o_part, l_part, Q, S, H, out, lse, st, true);
@@ -187,10 +188,11 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st, bool pdl,
                               const int32_t* win_page_table, int win_max_pages,
-                              const int32_t* win_vis, int window) {
+                              const int32_t* win_vis, int window, bool kv8, float kv_scale) {
   return launch_sparse_mla_tc(q, pool, num_pages, page_size, page_table, max_pages, q_offsets,
                               q_vis, idx, B, Q, H, topk, scale, S, out, lse, o_part, l_part, err,
-                              st, pdl, win_page_table, win_max_pages, win_vis, window);
+                              st, pdl, win_page_table, win_max_pages, win_vis, window, kv8,
+                              kv_scale);
 }
 
 }  // namespace dsa
@@ -321,6 +323,29 @@ dsa_status dsa_sparse_mla_decode_window(const void* q, const void* kv_pool, int 
                        idx, B, Q, heads, topk, scale, L.S, out, lse, ws, L,
                        static_cast<cudaStream_t>(stream), false, win_page_table, win_max_pages,
                        win_vis, window);
+}
+
+dsa_status dsa_sparse_mla_decode_fp8(const void* q, const void* kv_pool, float kv_scale,
+                                     int num_pages, int page_size, const int32_t* page_table,
+                                     int max_pages, const int32_t* q_offsets, const int32_t* q_vis,
+                                     const int32_t* idx, int B, int Q, int heads, int topk,
+                                     float scale, int num_splits, float* out, float* lse, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  if (!q_offsets || !q_vis || !ws) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Q <= 0 || topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (!(kv_scale > 0.f) || kv_scale != kv_scale || kv_scale > 3.0e38f) return DSA_ERR_INVALID_ARG;
+  if (B > DSA_MAX_BATCH || Q > 65535 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (num_splits < 0 || num_splits > DSA_MAX_SPLITS) return DSA_ERR_UNSUPPORTED;
+  dsa_status s = mla_checks(q, kv_pool, num_pages, page_size, page_table, max_pages, idx, out, lse,
+                            scale, heads);
+  if (s != DSA_OK) return s;
+  WsLayout L;
+  if (!ws_layout(Q, 1, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  return do_sparse_mla(q, kv_pool, num_pages, page_size, page_table, max_pages, q_offsets, q_vis,
+                       idx, B, Q, heads, topk, scale, L.S, out, lse, ws, L,
+                       static_cast<cudaStream_t>(stream), false, nullptr, 0, nullptr, 0, true,
+                       kv_scale);
 }
 
 dsa_status dsa_lse_combine(const float* o_parts, const float* lse_parts, int Q, int S, int heads,

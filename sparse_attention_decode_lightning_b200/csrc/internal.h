@@ -57,7 +57,8 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               float* out, float* lse, float* o_part, float* l_part,
                               uint32_t* err, cudaStream_t st, bool pdl,
                               const int32_t* win_page_table = nullptr, int win_max_pages = 0,
-                              const int32_t* win_vis = nullptr, int window = 0);
+                              const int32_t* win_vis = nullptr, int window = 0,
+                              bool kv8 = false, float kv_scale = 1.f);
 
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
                            float* out, float* lse, cudaStream_t st, bool pdl);

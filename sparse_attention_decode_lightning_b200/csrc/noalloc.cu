@@ -27,7 +27,8 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  int S, float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st, bool pdl,
                                  const int32_t* win_page_table = nullptr, int win_max_pages = 0,
-                                 const int32_t* win_vis = nullptr, int window = 0);
+                                 const int32_t* win_vis = nullptr, int window = 0,
+                                 bool kv8 = false, float kv_scale = 1.f);
 
 namespace {
 

@@ -52,6 +52,9 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 namespace dsa {
 namespace {
 
@@ -102,6 +105,7 @@ struct MlaTcArgs {
   const int32_t* idx;
   int B, Q, topk, S;
   float scale_log2;
+  float out_scale;                             // e4m3 cache: its per-tensor scale, else 1
   float* out;
   float* lse;
   float* o_part;
@@ -152,7 +156,22 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int NH>
+// two e4m3 codes (low byte first) -> two bf16, exactly: every e4m3 value has
+// at most 4 significant bits and an exponent inside bf16's range
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3);
+  __half2 h;
+  h = *reinterpret_cast<const __half2*>(&hr);
+  const float2 f = __half22float2(h);
+  return bf16x2_bits(__floats2bfloat162_rn(f.x, f.y));
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
+  return make_uint4(e4m3x2_to_bf16x2(v.x & 0xFFFFu), e4m3x2_to_bf16x2(v.x >> 16),
+                    e4m3x2_to_bf16x2(v.y & 0xFFFFu), e4m3x2_to_bf16x2(v.y >> 16));
+}
+
+template <int NH, bool KV8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_o, MlaTcArgs a) {
@@ -269,6 +288,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int s = k % NST;
       if (!(ok = warp_wait(&empty[s], ((k / NST) & 1) ^ 1, a.err))) break;
       uint8_t* stage = st + s * STAGE_BYTES;
+      if constexpr (KV8) {
+        // e4m3 rows of 576 bytes: a lane loads all its 8-byte pieces (8 dims
+        // of each of its 5 chunks of its 4 rows) before it widens them exactly
+        // to bf16 and stores them where the bf16 path's copies land
+        constexpr int RI = NR / (4 * PRODUCERS);
+        uint2 v[RI][MAXCH];
+#pragma unroll
+        for (int i = 0; i < RI; ++i) {
+          const int r = (NR / PRODUCERS) * pw + 4 * i + (lane >> 3);
+          const int j = k * NR + r;
+          const int row = j < nrows ? crd[j] : -1;
+          const uint8_t* src = pool + static_cast<size_t>(row < 0 ? 0 : row) * DSA_DIM + pu * 8;
+#pragma unroll
+          for (int c = 0; c < MAXCH; ++c) {
+            const int off = c < 4 ? (4 * static_cast<int>(rank) + c) * 64 : 512;
+            v[i][c] = row >= 0 ? __ldg(reinterpret_cast<const uint2*>(src + off)) : make_uint2(0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < RI; ++i) {
+          const int r = (NR / PRODUCERS) * pw + 4 * i + (lane >> 3);
+          uint8_t* dst = stage + r * 128 + ((pu ^ (r & 7)) * 16);
+#pragma unroll
+          for (int c = 0; c < MAXCH; ++c)
+            *reinterpret_cast<uint4*>(dst + c * CHUNK_T) = e4m3x8_to_bf16x8(v[i][c]);
+        }
+        fence_proxy_async_smem();      // generic-proxy stores, read by the tensor core
+        mbar_arrive(&full[s]);
+        continue;
+      }
 #pragma unroll
       for (int i = 0; i < NR / (4 * PRODUCERS); ++i) {
         const int r = (NR / PRODUCERS) * pw + 4 * i + (lane >> 3);
@@ -541,7 +590,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const float lt = lsum[h] + lsum[DSA_HEADS + h];
     const bool have = ok && live && ntiles > 0 && warp_wait(o_final, 0, a.err);
     if (have) tc_fence_after();
-    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    const float inv = lt > 0.f ? a.out_scale / lt : 0.f;
     // O / l leaves through shared memory: warpgroup g fills four boxes of
     // [128 heads x 32 fp32] (its columns [128g, 128g+128) of this CTA's 256)
     // in the 128-byte swizzle, then one thread stores them with TMA.  The
@@ -597,7 +646,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  int S, float* out, float* lse, float* o_part, float* l_part,
                                  uint32_t* err, cudaStream_t st, bool pdl,
                                  const int32_t* win_page_table, int win_max_pages,
-                                 const int32_t* win_vis, int window) {
+                                 const int32_t* win_vis, int window, bool kv8, float kv_scale) {
   if (Q <= 0) return cudaSuccess;
   if (H != 128 && H != 64) return cudaErrorInvalidValue;
   int page_shift = 0;
@@ -609,15 +658,17 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, DSA_DIM,
                        static_cast<uint64_t>(Q) * H, DSA_DIM * 2, 64, static_cast<uint32_t>(H)))
     return cudaErrorInvalidValue;
-  static bool attr_set[2][64] = {};
+  // one instance per (head count, cache type)
+  auto kernel = H == 128 ? (kv8 ? sparse_mla_tc_kernel<128, true> : sparse_mla_tc_kernel<128, false>)
+                         : (kv8 ? sparse_mla_tc_kernel<64, true> : sparse_mla_tc_kernel<64, false>);
+  static bool attr_set[4][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  const int hi = H == 128 ? 0 : 1;
-  if (dev >= 0 && dev < 64 && !attr_set[hi][dev]) {
-    cudaError_t e = cudaFuncSetAttribute(H == 128 ? sparse_mla_tc_kernel<128> : sparse_mla_tc_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  const int inst = (H == 128 ? 0 : 2) + (kv8 ? 1 : 0);
+  if (dev >= 0 && dev < 64 && !attr_set[inst][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[hi][dev] = true;
+    attr_set[inst][dev] = true;
   }
   // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
   // split partials [Q, S, H, 512]
@@ -628,7 +679,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
     return cudaErrorInvalidValue;
   MlaTcArgs a{q, pool, page_table, max_pages, num_pages, page_shift, win_page_table, win_max_pages,
               win_vis, window, q_offsets, q_vis, idx, B, Q, topk, S,
-              scale * 1.4426950408889634f, out, lse, o_part, l_part, err};
+              scale * kv_scale * 1.4426950408889634f, kv_scale, out, lse, o_part, l_part, err};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * Q * S), 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
@@ -639,8 +690,7 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return H == 128 ? cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<128>, tq, to, a)
-                  : cudaLaunchKernelEx(&cfg, sparse_mla_tc_kernel<64>, tq, to, a);
+  return cudaLaunchKernelEx(&cfg, kernel, tq, to, a);
 }
 
 }  // namespace dsa

@@ -203,6 +203,26 @@ def test_mla_closed_forms(nh, scale):
     assert (o == 0).all() and np.isneginf(lse).all()
 
 
+def test_fp8_rows_decode_then_scale():
+    # one e4m3 row: O = kv_scale * decoded row, LSE = scale * q . (kv_scale * row)
+    codes = _e4m3_bytes(RNG.standard_normal((1, 576)) * 3).reshape(1, 1, 576)
+    kv = 0.37
+    rows = O.latent_rows_e4m3(codes, np.array([0]), np.array([0]), kv, page_size=1)
+    dec = torch.from_numpy(codes.reshape(576).copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(rows[0], dec * kv)
+    q = O.bf16_decode(_bf16_bits(RNG.standard_normal((128, 576))))
+    o, lse = O.sparse_mla(q, rows, 1 / math.sqrt(192))
+    assert np.allclose(o, np.broadcast_to(kv * dec[:512], (128, 512)), atol=1e-12)
+    assert np.allclose(lse, (q @ (kv * dec)) / math.sqrt(192), atol=1e-12)
+    # paging: page p, slot s of a page_size-16 cache is pool[table[p], s]
+    pool = _e4m3_bytes(RNG.standard_normal((5, 16, 576))).reshape(5, 16, 576)
+    table = np.array([3, 0, 4])
+    pos = np.array([0, 17, 40, 15])
+    got = O.latent_rows_e4m3(pool, table, pos, 1.0, page_size=16)
+    want = O.e4m3_decode(np.stack([pool[3, 0], pool[0, 1], pool[4, 8], pool[3, 15]]))
+    assert np.array_equal(got, want)
+
+
 def test_lse_combine_equals_unsplit_and_ignores_empty_parts():
     scale = 1 / math.sqrt(192)
     q = O.bf16_decode(_bf16_bits(RNG.standard_normal((128, 576))))
