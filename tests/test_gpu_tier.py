@@ -187,3 +187,54 @@ def test_device_planner_refuses_a_step_beyond_its_slots():
         dsa.dsa_check_error(ws)
     assert e.value.status == 2
     assert torch.equal(pt[0], before[0])                         # sequence 0 was left as it was
+
+
+def test_device_tier_step_in_a_cuda_graph():
+    """Swap-in (plan + fetch) and sparse MLA captured once and replayed for
+    several steps with new index rows written in place: the device path needs
+    no host round trip, so the replays must follow the oracle step by step."""
+    rng = np.random.default_rng(21)
+    B, D, P, topk, heads = 2, 96, 400, 512, 64
+    host = torch.randn(B * P, PT, 576).to(torch.bfloat16).pin_memory()
+    pool = torch.zeros(B * D, PT, 576, dtype=torch.bfloat16, device=DEV)
+    pt = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    q = torch.randn(B, heads, 576).to(torch.bfloat16).to(DEV)
+    q_off = torch.arange(B + 1, dtype=torch.int32, device=DEV)
+    vis = torch.full((B,), P * PT, dtype=torch.int32, device=DEV)
+    idx = torch.full((B, topk), -1, dtype=torch.int32, device=DEV)
+    out = torch.empty(B, heads, 512, device=DEV)
+    lse = torch.empty(B, heads, device=DEV)
+    ws = dsa.workspace(B, 1, topk, 1)
+    scale = 1 / math.sqrt(256)
+    side = torch.cuda.Stream()
+    st = dsa.tier_dev_state(B, D, P, pt, stream=side)
+    trace = _trace(rng, B, P, 6, 60, 8, 1, topk)
+
+    def step():
+        dsa.dsa_tier_swap_in(st, B, D, P, idx, q_off, pt, host, pool, ws, stream=side)
+        dsa.dsa_sparse_mla_decode(q, pool, pt, q_off, vis, idx, B, scale, out, lse, ws,
+                                  num_splits=1, stream=side)
+
+    # first step eagerly (sets kernel attributes), then capture the step once
+    tier = O.TierOracle(B, D, P)
+    idx.copy_(torch.from_numpy(trace[0]))
+    torch.cuda.synchronize()
+    step()
+    side.synchronize()
+    tier.step([[list(trace[0][b])] for b in range(B)])
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    host_bits, q_np = np_bits(host).reshape(B, P * PT, 576), np_bits(q)
+    for idx_np in trace[1:]:
+        idx.copy_(torch.from_numpy(idx_np))
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        dsa.dsa_check_error(ws)
+        table, *_ = tier.step([[list(idx_np[b])] for b in range(B)])
+        assert pt.cpu().tolist() == table
+        for b in range(B):
+            sel = idx_np[b][idx_np[b] >= 0]
+            o_ref, l_ref = O.sparse_mla(O.bf16_decode(q_np[b]), O.bf16_decode(host_bits[b][sel]), scale)
+            check_attention(out[b].cpu().numpy(), lse[b].cpu().numpy(), o_ref, l_ref)
