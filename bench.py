@@ -49,6 +49,9 @@ def parse():
                     help="time the two-tier (HiSparse) decode path instead (one GPU)")
     ap.add_argument("--fp8", action="store_true",
                     help="time the sparse MLA over an e4m3 latent cache against bf16 (one GPU)")
+    ap.add_argument("--fused", action="store_true",
+                    help="time indexer + top-k as two kernels against the histogram-fused form "
+                         "on --workload (one GPU)")
     ap.add_argument("--csa", action="store_true",
                     help="time the compressed-sparse (DeepSeek-V4 CSA) decode step instead (one GPU)")
     return ap.parse_args()
@@ -781,6 +784,56 @@ def run_fp8(args):
     }
 
 
+def run_fused(args):
+    """Indexer + top-k selection of one layer of --workload, timed as the two
+    kernels the decode step uses (dsa_indexer_topk) and in the histogram-fused
+    form (dsa_indexer_topk_fused); L2 is flushed before each call."""
+    import statistics
+
+    import torch
+
+    import sparse_attention_decode_lightning_b200 as dsa
+    from synth import get_workload, make_inputs
+
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    inp = make_inputs(get_workload(args.workload), seed=args.seed, device=dev, layers_to_make=1)
+    Q, ix = inp.Q, inp.indexer[0]
+    first = bool(inp.mtp_index_share)
+    idx = {k: torch.empty(Q, inp.topk, dtype=torch.int32, device=dev) for k in ("two", "fused")}
+    ws = dsa.workspace(Q, inp.max_len, inp.topk, 0, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fns = {"two_kernel": (dsa.dsa_indexer_topk, idx["two"]),
+           "fused": (dsa.dsa_indexer_topk_fused, idx["fused"])}
+    res = {}
+    for name, (fn, out) in fns.items():
+        ts = []
+        for i in range(max(3, args.warmup) + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn(ix["q_idx"], ix["w"], ix["k_idx"], inp.seq_offsets, inp.q_offsets, inp.q_vis,
+               inp.B, inp.max_len, inp.topk, out, ws, first_only=first, stream=stream)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= max(3, args.warmup):
+                ts.append(a.elapsed_time(b) * 1e3)
+        dsa.dsa_check_error(ws)
+        res[name] = statistics.mean(ts)
+    # both forms select the same sets (rows compared sorted)
+    same = bool(torch.equal(idx["two"].sort(dim=1).values, idx["fused"].sort(dim=1).values))
+    return {
+        "metric": "indexer + top-k time: two kernels vs histogram-fused",
+        "value": res["fused"], "unit": "us", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup), "data": "synthetic",
+        "config": {"workload": args.workload, "B": inp.B, "Q": Q, "L": inp.max_len,
+                   "topk": inp.topk, "idx_heads": inp.idx_heads,
+                   "l2": "256 MiB flush before each call"},
+        "us": res, "same_sets": same,
+    }
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -801,6 +854,10 @@ def main():
     if args.fp8:
         if rank == 0:
             print(json.dumps(run_fp8(args)), flush=True)
+        return
+    if args.fused:
+        if rank == 0:
+            print(json.dumps(run_fused(args)), flush=True)
         return
     if world > 1:
         import datetime

@@ -103,8 +103,9 @@ int dsa_version(void);
  * most max_len keys, `topk` selected tokens and `num_splits` split-K parts
  * (0 = let the library choose).  The workspace holds the fp32 score rows
  * [Q, max_len], the split-K partial outputs (sized for 128 heads, so one
- * workspace serves both head counts) and the device error flag (the
- * selector keeps its histograms and candidate lists in on-chip memory).  The same workspace may be
+ * workspace serves both head counts), the fused selector's per-query
+ * first-digit histograms, counters and threshold-bin candidate lists (which
+ * dsa_indexer_topk_fused clears itself) and the device error flag.  The same workspace may be
  * reused by consecutive calls on one stream; it must be zeroed once
  * (cudaMemset) before its first use so the error flag starts clear.
  * Returns 0 for invalid sizes.
@@ -168,6 +169,26 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
                             int idx_heads, int max_len, int topk, int first_only,
                             int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
                             void* stream);
+
+/*
+ * The same call with the indexer and the selector fused through histograms:
+ * the indexer also counts, per query, the first 12-bit radix digit of every
+ * score it writes (warp-aggregated atomics), so the selector knows the
+ * threshold digit at launch, reads each score row once and resolves the
+ * threshold bin from a candidate list.  Same arguments, workspace and result
+ * (the same index sets) as dsa_indexer_topk; the call clears its histograms
+ * and counters in the workspace before the indexer.  A histogram that
+ * disagrees with its row raises DSA_ERR_DEVICE_BOUNDS.  Measured slower than
+ * dsa_indexer_topk on B200 at the built-in decode shapes (the histogram adds
+ * land in the indexer's epilogue, which bounds it), so the decode step uses
+ * the two-kernel form.
+ */
+dsa_status dsa_indexer_topk_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                                  int64_t total_keys, const int64_t* seq_offsets,
+                                  const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                                  int idx_heads, int max_len, int topk, int first_only,
+                                  int32_t* out_idx, float* out_scores, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * Sparse MLA decode in absorbed-MQA form over the selected tokens

@@ -42,6 +42,8 @@ SIGNATURES = {
     "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "dsa_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ,
                               _P]),
+    "dsa_indexer_topk_fused": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                    _P, _SZ, _P]),
     "dsa_sparse_mla_decode": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P,
                                    _P, _P, _SZ, _P]),
     "dsa_sparse_mla_decode_noalloc": (_I, [_P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _I, _I, _I, _F,
@@ -172,6 +174,15 @@ def dsa_indexer_topk(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len,
         _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
         _ptr(q_vis), B, q_idx.shape[0], q_idx.shape[1], max_len, topk, int(first_only),
         _ptr(out_idx), _ptr(out_scores), _ptr(ws), ws.numel(), _stream(stream)), "dsa_indexer_topk")
+
+
+def dsa_indexer_topk_fused(q_idx, w, k_idx, seq_offsets, q_offsets, q_vis, B, max_len, topk,
+                           out_idx, ws, out_scores=None, first_only=False, stream=None):
+    _check(lib().dsa_indexer_topk_fused(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_offsets), _ptr(q_offsets),
+        _ptr(q_vis), B, q_idx.shape[0], q_idx.shape[1], max_len, topk, int(first_only),
+        _ptr(out_idx), _ptr(out_scores), _ptr(ws), ws.numel(), _stream(stream)),
+        "dsa_indexer_topk_fused")
 
 
 def dsa_sparse_mla_decode(q, kv_pool, page_table, q_offsets, q_vis, idx, B, scale, out, lse, ws,

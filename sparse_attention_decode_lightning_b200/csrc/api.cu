@@ -66,6 +66,15 @@ bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* L) {
   w.scores = off;   off = align_up(off + static_cast<size_t>(Q) * w.ld * 4, 256);
   w.o_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * DSA_DIM_V * 4, 256);
   w.l_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * 4, 256);
+  // fused indexer -> selector: a 4096-bin histogram and 4 counters per query,
+  // and room for the threshold bin's candidates (about 1/16 of a row, at
+  // least 4096, at most 65536; a larger bin is re-read from the scores)
+  int cap = static_cast<int>(align_up(static_cast<size_t>(max_len / 16), 16));
+  cap = cap < 4096 ? 4096 : (cap > 65536 ? 65536 : cap);
+  w.cand_cap = cap;
+  w.hist = off;     off = align_up(off + static_cast<size_t>(Q) * 4096 * 4, 256);
+  w.ctr = off;      off = align_up(off + static_cast<size_t>(Q) * 16, 256);
+  w.cand = off;     off = align_up(off + static_cast<size_t>(Q) * cap * 8, 256);
   w.total = off;
   *L = w;
   return true;
@@ -126,15 +135,32 @@ dsa_status do_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t* 
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
                            int idx_heads, int max_len, int topk, int first_only, int32_t* out_idx,
-                           float* out_scores, void* ws, const WsLayout& L, cudaStream_t st) {
+                           float* out_scores, void* ws, const WsLayout& L, cudaStream_t st,
+                           bool fused = false) {
   uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
   float* scores = ws_ptr<float>(ws, L.scores);
-  cudaError_t e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B,
-                                 Q, idx_heads, first_only, scores, L.ld, err, st);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
-  // the selector starts while the indexer drains (its scores are waited for)
-  e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
-                  out_scores, err, st, true);
+  cudaError_t e;
+  if (fused) {
+    // the indexer fills per-query first-digit histograms (zeroed here, with
+    // the selector's counters that follow them) and the selector starts from
+    // them, launched while the indexer drains
+    uint32_t* hist = ws_ptr<uint32_t>(ws, L.hist);
+    e = cudaMemsetAsync(hist, 0, L.ctr - L.hist + static_cast<size_t>(Q) * 16, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
+                       idx_heads, first_only, scores, L.ld, err, st, hist);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    e = launch_topk_hist(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, hist,
+                         ws_ptr<uint32_t>(ws, L.ctr), ws_ptr<uint64_t>(ws, L.cand), L.cand_cap,
+                         out_idx, out_scores, err, st, true);
+  } else {
+    e = launch_indexer(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
+                       idx_heads, first_only, scores, L.ld, err, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    // the selector starts while the indexer drains (its scores are waited for)
+    e = launch_topk(scores, L.ld, q_offsets, q_vis, B, Q, max_len, topk, first_only, out_idx,
+                    out_scores, err, st, true);
+  }
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (first_only) {
     e = launch_expand_idx(q_offsets, B, Q, topk, out_idx, out_scores, st);
@@ -277,6 +303,24 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
   return do_indexer_topk(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
                          idx_heads, max_len, topk, first_only, out_idx, out_scores, ws, L,
                          static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_indexer_topk_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                                  int64_t total_keys, const int64_t* seq_offsets,
+                                  const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
+                                  int idx_heads, int max_len, int topk, int first_only,
+                                  int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  dsa_status s = check_common(seq_offsets, q_offsets, q_vis, B, Q, max_len, topk);
+  if (s != DSA_OK) return s;
+  if ((s = indexer_checks(q_idx, w, k_idx, total_keys, idx_heads)) != DSA_OK) return s;
+  if (!out_idx || !ws) return DSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!ws_layout(Q, max_len, topk, 1, &L)) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+  return do_indexer_topk(q_idx, w, k_idx, total_keys, seq_offsets, q_offsets, q_vis, B, Q,
+                         idx_heads, max_len, topk, first_only, out_idx, out_scores, ws, L,
+                         static_cast<cudaStream_t>(stream), true);
 }
 
 dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages, int page_size,

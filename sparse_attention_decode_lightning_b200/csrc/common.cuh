@@ -494,6 +494,38 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // scheduled as SMs free up; it still waits for this grid in pdl_wait()
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
 
+// ------------------------------------------------------------------ L2 loads
+// Loads from L2 (ld.global.cg, not cached in L1) that the compiler may not
+// move across other memory operations or barriers (volatile asm with a memory
+// clobber): for data other SMs or earlier kernels wrote, where an L1 line of
+// the same address from an earlier kernel on this SM could be stale.
+__device__ __forceinline__ uint32_t ld_l2_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t ld_l2_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float ld_l2_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float4 ld_l2_f32x4(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ misc
 // order-preserving map of fp32 to u32 (larger float -> larger key); -0 == +0
 __device__ __forceinline__ uint32_t float_key(float f) {

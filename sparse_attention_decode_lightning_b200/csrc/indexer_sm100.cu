@@ -71,10 +71,45 @@ struct IdxArgs {
   const int32_t* q_vis;
   float* scores;
   int ld;
+  uint32_t* hist;       // nullable: per query, counts of the top 12 bits of ~key(score)
   int B;
   int first_only;
   uint32_t* err;
 };
+
+// The written scores of a warp into their query's histogram of the
+// selector's first radix digit (top 12 bits of ~key(score)); lanes that fall
+// into the same bin add together.  Called by all 32 lanes from converged code
+// (a mask taken inside a divergent branch is not a safe match set); lanes
+// without a score pass valid = false.
+__device__ __forceinline__ void hist_add(uint32_t* h, bool valid, float v) {
+  const uint32_t bin = valid ? (~float_key(v)) >> 20 : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+  if (valid && static_cast<int>(threadIdx.x & 31) == __ffs(peers) - 1)
+    atomicAdd(&h[bin], static_cast<uint32_t>(__popc(peers)));
+}
+
+// A pipeline's shared-memory histogram (one query per sequence) goes to its
+// query's row in global memory and is cleared; each epilogue warp e takes
+// every EPI-th group of 32 bins.  g == nullptr only clears.
+template <int EPI>
+__device__ __forceinline__ void hist_flush(uint32_t* s_hist, uint32_t* g, int e, int lane) {
+  for (int bin = e * 32 + lane; bin < 4096; bin += 32 * EPI) {
+    const uint32_t c = s_hist[bin];
+    if (g && c) atomicAdd(&g[bin], c);
+    s_hist[bin] = 0;
+  }
+}
+
+// An epilogue warp's wait for an accumulator group.  With histograms the warp
+// gives up as a whole (hist_add needs all 32 lanes), so a lane whose bounded
+// wait ran out takes the others with it.
+template <bool HIST>
+__device__ __forceinline__ bool acc_wait(uint64_t* bar, uint32_t phase, uint32_t* err) {
+  const bool ok = mbar_wait(bar, phase, err);
+  if constexpr (HIST) return __all_sync(0xffffffffu, ok);
+  return ok;
+}
 
 // queries of sequence b that this launch scores (-1 if the entry is invalid)
 __device__ __forceinline__ int seq_queries(const IdxArgs& a, int b) {
@@ -141,7 +176,7 @@ __device__ __forceinline__ int seq_of_tile(const int* prefix, int B, int t) {
   return lo;
 }
 
-template <int HI, int EPI>
+template <int HI, int EPI, bool HIST>
 __global__ void __launch_bounds__(threads_for(EPI), 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_q, IdxArgs a) {
@@ -185,14 +220,19 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
   const int nslots = SLOTS / G;
   const uint32_t slot_cols = HI * G;
   const int qtiles = (maxq + G - 1) / G * G;      // the last pair may read one tile past nq
-  // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of qtiles tiles]
+  // per-pipeline shared memory: [ring of `stages` key tiles][query buffer of
+  // qtiles tiles][with histograms and one query per sequence: a 4096-bin
+  // histogram of the running sequence, which costs the ring one stage]
+  const bool smem_hist = HIST && maxq == 1;
   const int pipe_bytes = (DATA_BYTES / PIPES) / 1024 * 1024;
-  const int stages = min(MAX_STAGES, (pipe_bytes - qtiles * QT) / KEY_TILE);
+  const int stages =
+      min(MAX_STAGES, (pipe_bytes - qtiles * QT - (smem_hist ? 4096 * 4 : 0)) / KEY_TILE);
 
   const int pipe = warp / WPP;                     // 0 / 1
   const int pw = warp % WPP;                       // role within the pipeline
   uint8_t* keys = smem + OFF_DATA + pipe * pipe_bytes;
   uint8_t* qbuf = keys + stages * KEY_TILE;
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(qbuf + qtiles * QT);   // used if smem_hist
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR) + pipe * NBAR_PIPE;
   uint64_t* full = bars;
   uint64_t* empty = bars + MAX_STAGES;
@@ -337,6 +377,9 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(w_free);
           if (!(ok = mbar_wait(w_free, wph, a.err))) break;
+          if (smem_hist)   // the previous sequence's counts out, zeros for this one
+            hist_flush<EPI>(s_hist, cur_b >= 0 ? a.hist + static_cast<size_t>(q0) * 4096 : nullptr,
+                            pw - 2, lane);
           nq = seq_queries(a, b);
           q0 = a.q_offsets[b];
           const int64_t len = a.seq_offsets[b + 1] - a.seq_offsets[b];
@@ -364,7 +407,10 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           for (int j0 = 0; j0 < nq; j0 += G, ++n) {
             if (static_cast<int>(n & 1u) != half) continue;
             const uint32_t slot = n % nslots;
-            if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
+            if (!acc_wait<HIST>(&acc_full[slot], (n / nslots) & 1, a.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols;
             float r[2] = {0.f, 0.f};
@@ -391,8 +437,11 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[slot]);
             const int s = t * KT + row;
-            for (int jj = 0; jj < G && j0 + jj < nq; ++jj)
-              if (s < vis_s[j0 + jj]) a.scores[static_cast<size_t>(q0 + j0 + jj) * a.ld + s] = r[jj];
+            for (int jj = 0; jj < G && j0 + jj < nq; ++jj) {
+              const bool in = s < vis_s[j0 + jj];
+              if (in) a.scores[static_cast<size_t>(q0 + j0 + jj) * a.ld + s] = r[jj];
+              if constexpr (HIST) hist_add(a.hist + static_cast<size_t>(q0 + j0 + jj) * 4096, in, r[jj]);
+            }
           }
           continue;
         }
@@ -403,7 +452,10 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           for (int j0 = 0; j0 < nq; j0 += 2, ++n) {
             const uint32_t slot = n % nslots;
             const bool two = j0 + 1 < nq;
-            if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
+            if (!acc_wait<HIST>(&acc_full[slot], (n / nslots) & 1, a.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             float v[2 * HI];
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + slot * slot_cols;
@@ -436,8 +488,13 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
               r0 = a0 + a1;
               r1 = b0 + b1;
             }
-            if (s < vis_s[j0]) a.scores[static_cast<size_t>(q0 + j0) * a.ld + s] = r0;
-            if (two && s < vis_s[j0 + 1]) a.scores[static_cast<size_t>(q0 + j0 + 1) * a.ld + s] = r1;
+            const bool in0 = s < vis_s[j0], in1 = two && s < vis_s[j0 + 1];
+            if (in0) a.scores[static_cast<size_t>(q0 + j0) * a.ld + s] = r0;
+            if (in1) a.scores[static_cast<size_t>(q0 + j0 + 1) * a.ld + s] = r1;
+            if constexpr (HIST) {
+              hist_add(a.hist + static_cast<size_t>(q0 + j0) * 4096, in0, r0);
+              if (two) hist_add(a.hist + static_cast<size_t>(q0 + j0 + 1) * 4096, in1, r1);
+            }
           }
           continue;
         }
@@ -445,7 +502,10 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           const uint32_t slot = n % nslots;
           const int jj = j % G;                    // query within the slot's pair
           if (jj == 0) {
-            if (!mbar_wait(&acc_full[slot], (n / nslots) & 1, a.err)) { ok = false; break; }
+            if (!acc_wait<HIST>(&acc_full[slot], (n / nslots) & 1, a.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
           }
           float v[HI];
@@ -463,7 +523,9 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           const int q = q0 + j;
           const int vis = vis_s[j];
           const int s = t * KT + row;
-          if (s < vis) {
+          const bool in = s < vis;
+          float sc = 0.f;
+          if (in) {
             const float4* wp = reinterpret_cast<const float4*>(w_s + j * HI);
             float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
@@ -474,9 +536,24 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
               s2 = fmaf(ww.z, fmaxf(v[4 * h4 + 2], 0.f), s2);
               s3 = fmaf(ww.w, fmaxf(v[4 * h4 + 3], 0.f), s3);
             }
-            a.scores[static_cast<size_t>(q) * a.ld + s] = (s0 + s1) + (s2 + s3);
+            sc = (s0 + s1) + (s2 + s3);
+            a.scores[static_cast<size_t>(q) * a.ld + s] = sc;
+          }
+          if constexpr (HIST) {
+            if (smem_hist) {
+              if (in) atomicAdd(&s_hist[(~float_key(sc)) >> 20], 1u);
+            } else {
+              hist_add(a.hist + static_cast<size_t>(q) * 4096, in, sc);
+            }
           }
         }
+      }
+      // the last sequence's counts, once every epilogue warp has added its own
+      if (smem_hist && ok && cur_b >= 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(w_free);
+        if (mbar_wait(w_free, wph, a.err))
+          hist_flush<EPI>(s_hist, a.hist + static_cast<size_t>(q0) * 4096, pw - 2, lane);
       }
     }
   }
@@ -493,19 +570,19 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
 
 namespace {
 
-template <int HI, int EPI>
+template <int HI, int EPI, bool HIST>
 cudaError_t launch_indexer_h(const CUtensorMap& tk, const CUtensorMap& tq, const IdxArgs& args,
                              cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<HI, EPI>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<HI, EPI, HIST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  indexer_kernel<HI, EPI><<<device_sm_count(), threads_for(EPI), SMEM_BYTES, st>>>(tk, tq, args);
+  indexer_kernel<HI, EPI, HIST><<<device_sm_count(), threads_for(EPI), SMEM_BYTES, st>>>(tk, tq, args);
   return cudaGetLastError();
 }
 
@@ -515,7 +592,7 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
                            int idx_heads, int first_only, float* scores, int ld, uint32_t* err,
-                           cudaStream_t st) {
+                           cudaStream_t st, uint32_t* hist) {
   if (B <= 0 || Q <= 0 || total_keys <= 0) return cudaSuccess;
   if (idx_heads != 64 && idx_heads != 32) return cudaErrorInvalidValue;
   CUtensorMap tk, tq;
@@ -526,12 +603,21 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
                        static_cast<uint64_t>(Q) * idx_heads, DSA_IDX_DIM, DSA_IDX_DIM,
                        static_cast<uint32_t>(idx_heads)))
     return cudaErrorInvalidValue;
-  IdxArgs args{w, seq_offsets, q_offsets, q_vis, scores, ld, B, first_only, err};
+  IdxArgs args{w, seq_offsets, q_offsets, q_vis, scores, ld, hist, B, first_only, err};
   // several queries in a sequence (MTP verify): the 8-epilogue-warp instance
   const bool multi = Q > B && !first_only;
+  if (hist) {
+    if (idx_heads == 64)
+      return multi ? launch_indexer_h<64, 8, true>(tk, tq, args, st)
+                   : launch_indexer_h<64, 4, true>(tk, tq, args, st);
+    return multi ? launch_indexer_h<32, 8, true>(tk, tq, args, st)
+                 : launch_indexer_h<32, 4, true>(tk, tq, args, st);
+  }
   if (idx_heads == 64)
-    return multi ? launch_indexer_h<64, 8>(tk, tq, args, st) : launch_indexer_h<64, 4>(tk, tq, args, st);
-  return multi ? launch_indexer_h<32, 8>(tk, tq, args, st) : launch_indexer_h<32, 4>(tk, tq, args, st);
+    return multi ? launch_indexer_h<64, 8, false>(tk, tq, args, st)
+                 : launch_indexer_h<64, 4, false>(tk, tq, args, st);
+  return multi ? launch_indexer_h<32, 8, false>(tk, tq, args, st)
+               : launch_indexer_h<32, 4, false>(tk, tq, args, st);
 }
 
 }  // namespace dsa

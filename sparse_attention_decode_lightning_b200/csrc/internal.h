@@ -18,7 +18,12 @@ struct WsLayout {
   size_t scores = 0;   // fp32 [Q, ld]
   size_t o_part = 0;   // fp32 [Q, S, 128, 512]
   size_t l_part = 0;   // fp32 [Q, S, 128]
+  size_t hist = 0;     // u32 [Q, 4096]: the indexer's first-digit histograms
+  size_t ctr = 0;      // u32 [Q, 4]: the histogram selector's counters (follows hist;
+                       // both are zeroed together before each indexer launch)
+  size_t cand = 0;     // u64 [Q, cand_cap]: its threshold-bin candidates
   size_t total = 0;
+  int cand_cap = 0;
   int ld = 0;          // score row stride (elements)
   int S = 0;           // split-K parts the partial buffers hold
 };
@@ -40,12 +45,18 @@ cudaError_t launch_indexer(const uint8_t* q_idx, const float* w, const uint8_t* 
                            int64_t total_keys, const int64_t* seq_offsets,
                            const int32_t* q_offsets, const int32_t* q_vis, int B, int Q,
                            int idx_heads, int first_only, float* scores, int ld, uint32_t* err,
-                           cudaStream_t st);
+                           cudaStream_t st, uint32_t* hist = nullptr);
 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
                         const int32_t* q_vis, int B, int Q, int max_len, int topk,
                         int first_only, int32_t* out_idx, float* out_scores, uint32_t* err,
                         cudaStream_t st, bool pdl);
+
+cudaError_t launch_topk_hist(const float* scores, int ld, const int32_t* q_offsets,
+                             const int32_t* q_vis, int B, int Q, int max_len, int topk,
+                             int first_only, const uint32_t* hist, uint32_t* ctr, uint64_t* cand,
+                             int cand_cap, int32_t* out_idx, float* out_scores, uint32_t* err,
+                             cudaStream_t st, bool pdl);
 
 cudaError_t launch_expand_idx(const int32_t* q_offsets, int B, int Q, int topk,
                               int32_t* out_idx, float* out_scores, cudaStream_t st);

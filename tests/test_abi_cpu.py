@@ -98,6 +98,14 @@ def test_host_checks_reject_bad_arguments_without_a_device():
     # workspace too small
     assert L.dsa_indexer_topk(fake, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
                               null, fake, 16, null) == 6
+    # the fused form checks the same way
+    for fn in (L.dsa_indexer_topk, L.dsa_indexer_topk_fused):
+        assert fn(null, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
+                  null, fake, 1 << 30, null) == 1
+        assert fn(fake, fake, fake, 100, fake, fake, fake, 1, 1, 48, 100, 2048, 0, fake,
+                  null, fake, 1 << 30, null) == 2
+        assert fn(fake, fake, fake, 100, fake, fake, fake, 1, 1, 64, 100, 2048, 0, fake,
+                  null, fake, 16, null) == 6
     # sparse MLA: bad scale, bad split count, null page table
     assert L.dsa_sparse_mla_decode(fake, fake, 10, 64, fake, 4, fake, fake, fake, 1, 1, 128, 2048,
                                    ctypes.c_float(0.0), 0, fake, fake, fake, 1 << 30, null) == 1
