@@ -190,31 +190,31 @@ __global__ void __launch_bounds__(THREADS, 2) topk_hist_kernel(HistTopkArgs a) {
     }
 #pragma unroll
     for (int r = 0; r < UNROLL; ++r) {
-    const int g = base + r * THREADS + tid;
-    const float e[4] = {vv[r].x, vv[r].y, vv[r].z, vv[r].w};
+      const int g = base + r * THREADS + tid;
+      const float e[4] = {vv[r].x, vv[r].y, vv[r].z, vv[r].w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      // about one score in twenty is kept: a lane that keeps one takes its
-      // staging slot with a shared-memory atomic of its own
-      const int p = 4 * g + k;
-      const uint32_t u = ~float_key(e[k]);
-      const uint32_t d = u >> (32 - DIGIT);
-      if (g < g1 && p < vis && d <= t) {
-        if (d < t) {
-          const uint32_t slot = atomicAdd(&s_nt, 1u);
-          if (slot < static_cast<uint32_t>(TAKE_CAP)) s_take[slot] = static_cast<uint32_t>(p);
-        } else {
-          const uint64_t V = (static_cast<uint64_t>(u) << pb) | static_cast<uint64_t>(p);
-          const uint32_t c = atomicAdd(&s_nm, 1u);
-          if (c < static_cast<uint32_t>(MID_CAP)) {
-            s_mid[c] = V;
-          } else {                              // a crowded bin: straight to the global list
-            const uint32_t gc = atomicAdd(&ctr[1], 1u);
-            if (gc < static_cast<uint32_t>(a.cand_cap)) cand[gc] = V;
+      for (int k = 0; k < 4; ++k) {
+        // about one score in twenty is kept: a lane that keeps one takes its
+        // staging slot with a shared-memory atomic of its own
+        const int p = 4 * g + k;
+        const uint32_t u = ~float_key(e[k]);
+        const uint32_t d = u >> (32 - DIGIT);
+        if (g < g1 && p < vis && d <= t) {
+          if (d < t) {
+            const uint32_t slot = atomicAdd(&s_nt, 1u);
+            if (slot < static_cast<uint32_t>(TAKE_CAP)) s_take[slot] = static_cast<uint32_t>(p);
+          } else {
+            const uint64_t V = (static_cast<uint64_t>(u) << pb) | static_cast<uint64_t>(p);
+            const uint32_t c = atomicAdd(&s_nm, 1u);
+            if (c < static_cast<uint32_t>(MID_CAP)) {
+              s_mid[c] = V;
+            } else {                            // a crowded bin: straight to the global list
+              const uint32_t gc = atomicAdd(&ctr[1], 1u);
+              if (gc < static_cast<uint32_t>(a.cand_cap)) cand[gc] = V;
+            }
           }
         }
       }
-    }
     }
   }
   __syncthreads();
@@ -241,17 +241,26 @@ __global__ void __launch_bounds__(THREADS, 2) topk_hist_kernel(HistTopkArgs a) {
   // ---- the last CTA of the row finishes it
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&ctr[2], 1u) == static_cast<uint32_t>(cpr - 1);
+  if (tid == 0) {
+    s_last = atomicAdd(&ctr[2], 1u) == static_cast<uint32_t>(cpr - 1);
+    if (s_last) {
+      // every other CTA of the row has added its entries: one thread reads
+      // the row's totals and hands them to the block, so every thread takes
+      // the same branches (and barriers) below
+      __threadfence();
+      s_bm = ld_l2_u32(&ctr[1]);                // candidates of bin t
+      s_bt = ld_l2_u32(&ctr[0]);                // positions below the threshold digit
+      s_nt = 0;
+    }
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
-  const uint32_t n_cand = ld_l2_u32(&ctr[1]);
+  const uint32_t n_cand = s_bm;
   const bool from_list = n_cand <= static_cast<uint32_t>(a.cand_cap);
   if (n_cand != n_bin && tid == 0) raise_error(a.err, DEVERR_BOUNDS);   // histogram and row disagree
-  // the row's positions below the threshold digit are all written: bin t's
-  // keys take the slots after them, numbered by a shared counter
-  const uint32_t base0 = ld_l2_u32(&ctr[0]);
-  if (tid == 0) s_nt = 0;
+  // bin t's keys take the slots after the row's positions below the
+  // threshold digit, numbered by a shared counter
+  const uint32_t base0 = s_bt;
   __syncthreads();                              // s_h (staging) is reused below
 
   // the need smallest V of bin t, by radix passes of FDIGIT bits over the
