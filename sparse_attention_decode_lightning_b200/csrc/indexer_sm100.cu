@@ -573,15 +573,12 @@ namespace {
 template <int HI, int EPI, bool HIST>
 cudaError_t launch_indexer_h(const CUtensorMap& tk, const CUtensorMap& tq, const IdxArgs& args,
                              cudaStream_t st) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<HI, EPI, HIST>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_done[64];
+  const cudaError_t e = set_once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(indexer_kernel<HI, EPI, HIST>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
   indexer_kernel<HI, EPI, HIST><<<device_sm_count(), threads_for(EPI), SMEM_BYTES, st>>>(tk, tq, args);
   return cudaGetLastError();
 }

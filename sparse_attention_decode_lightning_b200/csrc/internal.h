@@ -2,6 +2,8 @@
 // workspace carve-up and the kernel launchers.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -32,6 +34,21 @@ struct WsLayout {
 bool encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                      uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
                      uint32_t box_inner, uint32_t box_rows);
+
+// Runs `set` (cudaFuncSetAttribute calls) once per device and remembers the
+// success in `done` (device ids below 64; other ids run `set` on every call).
+// Safe from several host threads: a race at most runs the idempotent `set`
+// twice.
+template <typename F>
+inline cudaError_t set_once_per_device(std::atomic<bool> (&done)[64], F&& set) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const cudaError_t e = set();
+  if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* out);
 // a latent-cache page of page_size tokens: a power of two from 1 to 1024, and

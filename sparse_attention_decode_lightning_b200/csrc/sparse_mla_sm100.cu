@@ -661,15 +661,12 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   // one instance per (head count, cache type)
   auto kernel = H == 128 ? (kv8 ? sparse_mla_tc_kernel<128, true> : sparse_mla_tc_kernel<128, false>)
                          : (kv8 ? sparse_mla_tc_kernel<64, true> : sparse_mla_tc_kernel<64, false>);
-  static bool attr_set[4][64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
+  static std::atomic<bool> attr_done[4][64];
   const int inst = (H == 128 ? 0 : 2) + (kv8 ? 1 : 0);
-  if (dev >= 0 && dev < 64 && !attr_set[inst][dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[inst][dev] = true;
-  }
+  const cudaError_t ea = set_once_per_device(attr_done[inst], [kernel] {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (ea != cudaSuccess) return ea;
   // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
   // split partials [Q, S, H, 512]
   CUtensorMap to;

@@ -670,15 +670,12 @@ dsa_status dsa_tier_swap_in(void* dev_state, size_t state_bytes, int B, int dev_
   int32_t* copies = reinterpret_cast<int32_t*>(base + L.copies);
   const int N = pow2_at_least(dev_slots);
   const size_t smem = static_cast<size_t>(N) * 8 + static_cast<size_t>(dev_slots) * 4 + static_cast<size_t>(N) * 4;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(tier_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(DEV_MAX_SLOTS) * 16) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_done[64];
+  if (set_once_per_device(attr_done, [] {
+        return cudaFuncSetAttribute(tier_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(DEV_MAX_SLOTS) * 16);
+      }) != cudaSuccess)
+    return DSA_ERR_CUDA;
   if (cudaMemsetAsync(hdr, 0, 16, st) != cudaSuccess) return DSA_ERR_CUDA;   // this step's counters
   tier_plan_kernel<<<B, PLAN_THREADS, smem, st>>>(
       hdr, reinterpret_cast<int32_t*>(base + L.stamp), reinterpret_cast<int32_t*>(base + L.page_of_slot),

@@ -495,10 +495,11 @@ int topk_cluster_size(int rows, int max_len, int cap) {
 // non-portable) when at least one such cluster fits, else 8.  Queried once
 // per device; a handful of long rows (1M context) then gets twice the CTAs.
 int max_cluster_for_device(size_t smem) {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];  // 0 until queried; racing queries store the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAX_CLUSTER;
-  if (cached[dev]) return cached[dev];
+  const int known = cached[dev].load(std::memory_order_relaxed);
+  if (known) return known;
   int cap = MAX_CLUSTER;
   if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
       cudaSuccess) {
@@ -518,7 +519,7 @@ int max_cluster_for_device(size_t smem) {
       cap = MAX_CLUSTER_NP;
   }
   cudaGetLastError();   // a refused query leaves no sticky error behind
-  cached[dev] = cap;
+  cached[dev].store(cap, std::memory_order_relaxed);
   return cap;
 }
 
@@ -531,16 +532,12 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* q_offsets,
   const int rows = first_only ? B : Q;
   if (rows <= 0) return cudaSuccess;
   if (rows > 65535 || topk > DSA_MAX_TOPK) return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes(SLICE_CAP)));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_done[64];
+  const cudaError_t ea = set_once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem_bytes(SLICE_CAP)));
+  });
+  if (ea != cudaSuccess) return ea;
   // beyond the portable 8 CTAs only when 8 would leave slices longer than the
   // on-chip copy (merging 16 histograms costs more than it saves otherwise)
   int C = topk_cluster_size(rows, max_len, MAX_CLUSTER);

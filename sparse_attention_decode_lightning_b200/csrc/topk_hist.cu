@@ -344,19 +344,16 @@ cudaError_t launch_topk_hist(const float* scores, int ld, const int32_t* q_offse
   if (cpr < 1) cpr = 1;
   // the same shared-memory carve-out as the indexer it overlaps, so that an SM
   // need not drain to change its L1/shared split when this kernel arrives
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(topk_hist_kernel,
-                                         cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         cudaSharedmemCarveoutMaxShared);
+  static std::atomic<bool> attr_done[64];
+  const cudaError_t ea = set_once_per_device(attr_done, [] {
+    const cudaError_t e = cudaFuncSetAttribute(topk_hist_kernel,
+                                               cudaFuncAttributePreferredSharedMemoryCarveout,
+                                               cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             STAGE_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+    return cudaFuncSetAttribute(topk_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                STAGE_BYTES);
+  });
+  if (ea != cudaSuccess) return ea;
   HistTopkArgs a{scores, ld, q_offsets, q_vis, B, Q, topk, first_only, hist, ctr, cand, cand_cap,
                  out_idx, out_scores, err};
   cudaLaunchConfig_t cfg = {};
