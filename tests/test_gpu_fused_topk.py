@@ -118,3 +118,32 @@ def test_fused_selection_many_rows(dirty, hi):
         dsa.dsa_indexer_topk_fused(qi, w, k, seq_off, q_off, vis, B, L, topk, idx, ws)
         dsa.dsa_check_error(ws)
         _check_rows(scores, idx, vis, topk)
+
+
+def test_fused_out_scores_match_the_selected_positions():
+    """out_scores: the score of each selected position as the indexer wrote
+    it, and -inf in the padding of a row with fewer visible keys than topk."""
+    lens = [150000, 9000, 1500]
+    topk = 2048
+    k, qi, w = _inputs("normal", lens, 1, seed=23)
+    B = Q = len(lens)
+    seq_off = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int64, device=DEV)
+    q_off = torch.arange(B + 1, dtype=torch.int32, device=DEV)
+    vis = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    L = max(lens)
+    ld = ((L + 63) // 64) * 64
+    scores = torch.full((Q, ld), float("nan"), device=DEV)
+    ws2 = dsa.workspace(Q, L, topk, 1)
+    dsa.dsa_indexer_scores(qi, w, k, seq_off, q_off, vis, B, L, scores, ws2)
+    dsa.dsa_check_error(ws2)
+    idx = torch.empty(Q, topk, dtype=torch.int32, device=DEV)
+    osc = torch.full((Q, topk), float("nan"), device=DEV)
+    ws = dsa.workspace(Q, L, topk, 1)
+    dsa.dsa_indexer_topk_fused(qi, w, k, seq_off, q_off, vis, B, L, topk, idx, ws, out_scores=osc)
+    dsa.dsa_check_error(ws)
+    _check_rows(scores, idx, vis, topk)
+    sc, ix, os_ = scores.cpu().numpy(), idx.cpu().numpy(), osc.cpu().numpy()
+    for q in range(Q):
+        sel = ix[q] >= 0
+        assert np.array_equal(os_[q][sel], sc[q][ix[q][sel]]), q
+        assert np.all(np.isneginf(os_[q][~sel])), q
