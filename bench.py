@@ -86,6 +86,27 @@ def measured_traffic(kernel_file: str, profile: str):
     return int(fields["traffic_bytes_per_launch"])
 
 
+def gpu_local_cpus(dev) -> set:
+    """CPUs of the GPU's own NUMA node (the sysfs local_cpulist of its PCI
+    function) that this process may run on; empty when unknown."""
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        with open(f"/sys/bus/pci/devices/{bdf}/local_cpulist") as f:
+            text = f.read().strip()
+        cpus = set()
+        for part in text.split(","):
+            if "-" in part:
+                a, b = part.split("-")
+                cpus.update(range(int(a), int(b) + 1))
+            elif part:
+                cpus.add(int(part))
+        return cpus & os.sched_getaffinity(0)
+    except (OSError, ValueError, AttributeError, RuntimeError):
+        return set()
+
+
 def reduce_over_ranks(local_ms: float, world: int, dist=None, device=None) -> float:
     """Slowest rank's device time (ms): the job finishes when its last rank does."""
     if world <= 1 or dist is None:
@@ -351,8 +372,19 @@ def run_ours(args, rank, world, local_rank):
             h.copy_(src)
             return h
 
-        h_in = [host_input(t) for t in qi + wl_ + qs]
-        h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs + lses]
+        # pinned pages land on the NUMA node of the thread that allocates them:
+        # allocate from the GPU's own node so the copies do not cross sockets
+        saved_cpus = os.sched_getaffinity(0)
+        local_cpus = gpu_local_cpus(dev)
+        numa_bound = bool(local_cpus) and local_cpus != saved_cpus
+        if numa_bound:
+            os.sched_setaffinity(0, local_cpus)
+        try:
+            h_in = [host_input(t) for t in qi + wl_ + qs]
+            h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs + lses]
+        finally:
+            if numa_bound:
+                os.sched_setaffinity(0, saved_cpus)
         d_in = [[torch.empty_like(t) if t is not None else None for t in qi + wl_ + qs]
                 for _ in range(nb)]
         d_res = [[torch.empty_like(o) for o in outs + lses] for _ in range(nb)]
@@ -405,7 +437,9 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": ("inputs from write-combined pinned host memory" if wc_ptrs else
                         "inputs from pinned host memory") +
-                       ", outputs to pinned host memory; copies on two copy streams overlap "
+                       ", outputs to pinned host memory" +
+                       (" (allocated from the GPU's NUMA-local CPUs)" if numa_bound else "") +
+                       "; copies on two copy streams overlap "
                        "compute (double-buffered); 256 MiB L2 flush inside every step"}
         dsa.dsa_check_error(ws, stream)
         torch.cuda.synchronize(dev)
