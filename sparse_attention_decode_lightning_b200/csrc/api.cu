@@ -240,7 +240,7 @@ const char* dsa_status_string(int s) {
   }
 }
 
-int dsa_version(void) { return 200; }
+int dsa_version(void) { return 300; }
 
 int dsa_choose_splits(int Q, int topk, int num_splits) {
   if (Q <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || num_splits < 0 || num_splits > DSA_MAX_SPLITS)

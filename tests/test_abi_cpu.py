@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_library_loads_and_reports_version_and_status_names():
     L = dsa.lib()
-    assert L.dsa_version() == 200
+    assert L.dsa_version() == 300
     for code, name in dsa.STATUS.items():
         assert dsa.dsa_status_string(code) == name
     assert dsa.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
