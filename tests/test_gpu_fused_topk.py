@@ -1,14 +1,16 @@
 """The fused indexer -> selector path (dsa_indexer_topk_fused): the indexer
 emits per-query histograms of the selector's first radix digit and the
 selector starts from them.  Its index sets must equal, exactly and ties
-included, a full sort by (score desc, position asc) of the fp32 scores the
-same indexer writes (dsa_indexer_scores), over ordinary, all-equal,
+included, the oracle's selection (oracle.topk_select: a full sort by score
+desc, position asc) over the fp32 scores the same indexer writes
+(dsa_indexer_scores), over ordinary, all-equal,
 tied and narrow-band score rows, single and multi-query sequences."""
 import numpy as np
 import pytest
 import torch
 
 import sparse_attention_decode_lightning_b200 as dsa
+from oracle import topk_select
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -37,10 +39,10 @@ def _inputs(case, lens, T, seed, hi=64):
 
 
 def _expected(scores_row, vis, topk):
-    s = scores_row[:vis].astype(np.float32)
-    s = np.where(s == 0, np.float32(0), s)          # -0 == +0
-    order = np.lexsort((np.arange(vis), -s.astype(np.float64)))
-    return set(order[:min(topk, vis)].tolist())
+    """The oracle's selection (stable sort by score desc, position asc; -0 ==
+    +0) over the fp32 scores the GPU indexer wrote, as a set."""
+    sel = topk_select(scores_row[:vis].astype(np.float32), topk)
+    return set(sel[sel >= 0].tolist())
 
 
 @pytest.mark.parametrize("case", ["normal", "all_zero", "tied_keys", "narrow"])
