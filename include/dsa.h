@@ -178,10 +178,11 @@ dsa_status dsa_indexer_topk(const uint8_t* q_idx, const float* w, const uint8_t*
  * threshold bin from a candidate list.  Same arguments, workspace and result
  * (the same index sets) as dsa_indexer_topk; the call clears its histograms
  * and counters in the workspace before the indexer.  A histogram that
- * disagrees with its row raises DSA_ERR_DEVICE_BOUNDS.  Measured slower than
- * dsa_indexer_topk on B200 at the built-in decode shapes (the histogram adds
- * land in the indexer's epilogue, which bounds it), so the decode step uses
- * the two-kernel form.
+ * disagrees with its row raises DSA_ERR_DEVICE_BOUNDS.  On B200 it measured
+ * slower than dsa_indexer_topk for batch-32 decode at 128K (134.8 against
+ * 123.6 us: the histogram adds land in the indexer's epilogue, which bounds
+ * it) and slightly faster for 4 sequences at 1M (130.9 against 133.6 us), so
+ * the decode step uses the two-kernel form.
  */
 dsa_status dsa_indexer_topk_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                                   int64_t total_keys, const int64_t* seq_offsets,
