@@ -68,8 +68,17 @@ def test_workspace_bytes_arithmetic():
     # error flag + fp32 score row + one partial output and its LSE row
     assert small >= 256 + 8192 * 4 + 128 * 512 * 4 + 128 * 4
     assert f(32, 131072, 2048, 1) >= 32 * 131072 * 4
-    # the selector's working set is on chip: nothing per key beyond the fp32 score
+    # per key, nothing beyond the fp32 score and the fused selector's candidate
+    # room (1/16 of a row of u64 keys)
     assert f(32, 131072, 2048, 1) < 32 * 131072 * 4 + (64 << 20)
+    # every documented region fits: error word, scores [Q, ld], one split's
+    # partials, and the fused selector's u32 histograms [Q, 4096], counters
+    # [Q, 4] and candidate lists [Q, cap], cap = max_len/16 clamped to 4096-65536
+    for Q, L in ((1, 8192), (32, 131072), (4, 1 << 20), (3, 1000)):
+        cap = min(max(L // 16, 4096), 65536)
+        ld = (L + 63) // 64 * 64
+        base = 256 + Q * ld * 4 + Q * 128 * 512 * 4 + Q * 128 * 4
+        assert f(Q, L, 2048, 1) >= base + Q * 4096 * 4 + Q * 16 + Q * cap * 8, (Q, L)
     assert f(4, 1 << 20, 2048, 16) > f(4, 1 << 20, 2048, 1)
     assert f(4, 1 << 20, 2048, 16) - f(4, 1 << 20, 2048, 1) >= 4 * 15 * 128 * 512 * 4
 
