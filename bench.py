@@ -144,15 +144,59 @@ def algorithmic_bytes(inp):
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """Clock and throttle-reason samples for the timed region: NVML polled about
+    every millisecond from a thread (the samples taken between region_begin
+    and region_end are the ones reported), with nvidia-smi at 200 ms as the
+    fallback when NVML is unavailable or saw nothing inside the region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, device=None):
+        import threading
         self.gpu = gpu_index
+        self.device = device
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         self.p = None
+        self.nvml_rows = []          # (time, sm MHz, max sm MHz, power W, reason mask)
+        self.stop = threading.Event()
+        self.thread = None
+        self.nvml = None
+        self.t0 = self.t1 = None
+
+    def _nvml_start(self):
+        import threading
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            if self.device is not None:
+                pr = torch.cuda.get_device_properties(self.device)
+                bdf = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bdf)
+            else:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            return
+
+        def poll():
+            while not self.stop.is_set():
+                try:
+                    t = time.perf_counter()
+                    row = (t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                           pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
+                           pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(reasons(h)))
+                except Exception:
+                    return
+                self.nvml_rows.append(row)
+                self.stop.wait(0.001)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def __enter__(self):
         try:
@@ -161,16 +205,50 @@ class Clocks:
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+        self._nvml_start()
         time.sleep(0.3)
         return self
 
+    def region_begin(self):
+        self.t0 = time.perf_counter()
+
+    def region_end(self):
+        self.t1 = time.perf_counter()
+
     def __exit__(self, *a):
+        self.stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.nvml is not None and (self.thread is None or not self.thread.is_alive()):
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.p is not None:
             self.p.terminate()
             try:
                 self.p.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.p.kill()
+
+    def _nvml_summary(self):
+        if self.t0 is None or self.t1 is None or self.nvml is None:
+            return None
+        rows = [r for r in self.nvml_rows if self.t0 <= r[0] <= self.t1]
+        if not rows:
+            return None
+        masks = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+                 "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+                 "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+                 "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
+        seen = 0
+        for r in rows:
+            seen |= r[4]
+        reasons = sorted(n for n, c in masks.items() if seen & int(getattr(self.nvml, c, 0)))
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(r[2] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[3] for r in rows),
+                "source": "NVML, ~1 ms polling inside the timed region"}
 
     def summary(self):
         self.f.flush()
@@ -181,6 +259,9 @@ class Clocks:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.f.name)
+        inside = self._nvml_summary()
+        if inside is not None:
+            return inside
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
 
@@ -192,12 +273,13 @@ class Clocks:
         sm = [num(r[1]) for r in rows if num(r[1]) is not None]
         mx = [num(r[2]) for r in rows if num(r[2]) is not None]
         pw = [num(r[3]) for r in rows if num(r[3]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        reasons = sorted({n for r in rows for n, v in zip(self.REASONS, r[5:9])
+                          if v.lower().startswith("active")})
         loaded = [s for s, p in zip(sm, pw) if p is not None and p > 300] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+                "samples": len(rows), "power_w_max": max(pw) if pw else None,
+                "source": "nvidia-smi, 200 ms sampling around the timed region"}
 
 
 def host_subproblem(inp, b):
@@ -297,8 +379,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- timed region: K steps, L2 flushed between steps (outside the events)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    with Clocks(local_rank) as clk:
+    with Clocks(local_rank, dev) as clk:
         barrier()
+        clk.region_begin()
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
@@ -307,6 +390,7 @@ def run_ours(args, rank, world, local_rank):
             evs[i][1].record(stream)
         barrier()
         t_wall = time.perf_counter() - t_wall
+        clk.region_end()
     clocks = clk.summary()
     dsa.dsa_check_error(ws, stream)
     step_ms = [a.elapsed_time(b) for a, b in evs]
