@@ -445,8 +445,7 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
     }
     s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
                       max_pages, q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S,
-                      out_layers[l],
-                      lse_layers[l], ws, L, st, true);
+                      out_layers[l], lse_layers[l], ws, L, st, true);
     if (s != DSA_OK) return s;
   }
   return DSA_OK;
