@@ -20,6 +20,9 @@ Sources (pages are cited by title and section):
           kv rank of 512 with a 64-d RoPE part, a 32-head FP8 indexer of head
           dim 128.  Every function below takes its head counts from the
           arrays it is given, so both models' shapes go through the same code.
+  [ARCH-2.3] same page, section 2.3 DeepSeek-V4: compressed sparse attention
+          (CSA) keeps the top-k of a 4x compressed KV cache plus a 128-token
+          sliding window of raw tokens.
   [GLM-INF] "GLM-5.2 推理部署" (inference deployment), MTP draft + verify flow:
           top-K = 2048 indices computed at draft step 1 and reused by later
           steps; verify appends the drafts and runs one prefill-style forward.
@@ -34,7 +37,11 @@ Readings where the pages are silent (each is listed in the design notes):
     log-sum-exp is the natural log of sum_j exp(scale * q.c_j);
   * split-K: the context is cut into S contiguous equal ranges, each attends to
     the selected tokens inside it, and the partial results are merged exactly
-    through their log-sum-exps; an empty range has LSE = -inf and weight 0.
+    through their log-sum-exps; an empty range has LSE = -inf and weight 0;
+  * CSA window: a query that sees win_vis raw tokens attends to the last
+    `window` of them (fewer when win_vis < window), in the same softmax as its
+    selected compressed entries; how entries are compressed is learned and
+    outside this path, so the compressed rows are inputs.
 """
 import math
 from typing import Dict, List, Optional, Sequence, Tuple
@@ -52,6 +59,7 @@ __all__ = [
     "e4m3_table", "e4m3_decode", "bf16_decode",
     "indexer_scores", "topk_select", "latent_rows", "latent_rows_e4m3",
     "sparse_mla", "sparse_mla_split", "lse_combine",
+    "csa_window_positions", "csa_window_attention",
     "query_step", "decode_step",
 ]
 
@@ -201,6 +209,33 @@ def sparse_mla_split(q: np.ndarray, rows: np.ndarray, positions: np.ndarray, con
         sel = (positions >= lo) & (positions < hi)
         o_parts[c], lse_parts[c] = sparse_mla(q, rows[sel], scale)
     return lse_combine(o_parts, lse_parts)
+
+
+# --------------------------------------------------------------------------
+# DeepSeek-V4 CSA: selected compressed entries plus a raw sliding window
+# [ARCH-2.3] "大语言模型结构总览", section 2.3 DeepSeek-V4: the KV cache is
+# compressed 4x along the sequence, DSA selects the top-1024 (Pro) or top-512
+# (Flash) compressed entries, and a 128-token sliding window of uncompressed
+# tokens is attended as well, for locality.
+# --------------------------------------------------------------------------
+def csa_window_positions(win_vis: int, window: int) -> np.ndarray:
+    """The raw tokens of a query's sliding window: the `window` most recent of
+    the win_vis visible raw positions, win_vis-window .. win_vis-1, with the
+    positions below 0 (a window that starts before the first token) left out."""
+    lo = max(0, int(win_vis) - int(window))
+    return np.arange(lo, int(win_vis), dtype=np.int64)
+
+
+def csa_window_attention(q: np.ndarray, pool: np.ndarray, page_row_c: np.ndarray,
+                         page_row_raw: np.ndarray, selected: np.ndarray, win_vis: int,
+                         window: int, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """One query of CSA decode attention: a single softmax over the selected
+    compressed entries (positions of the compressed cache, through page_row_c)
+    together with the raw window rows (through page_row_raw), both caches in
+    the same latent pool.  q float64 [H,576]; returns (O [H,512], LSE [H])."""
+    rows_c = latent_rows(pool, page_row_c, np.asarray(selected, dtype=np.int64))
+    rows_w = latent_rows(pool, page_row_raw, csa_window_positions(win_vis, window))
+    return sparse_mla(q, np.concatenate([rows_c, rows_w]), scale)
 
 
 # --------------------------------------------------------------------------

@@ -41,10 +41,9 @@ def _case(seed, B, L_raw, heads=128, ratio=4):
 
 
 def _oracle(pool_b, ct_b, rt_b, q_b, sel, wv, window, scale):
-    rows_c = O.latent_rows(pool_b, ct_b, sel)
-    win = np.arange(max(0, wv - window), wv)
-    rows_w = O.latent_rows(pool_b, rt_b, win)
-    return O.sparse_mla(O.bf16_decode(q_b), np.concatenate([rows_c, rows_w]), scale)
+    # the window rule (the last `window` raw tokens, none below 0) is the
+    # oracle's own, pinned in test_oracle_pins.py
+    return O.csa_window_attention(O.bf16_decode(q_b), pool_b, ct_b, rt_b, sel, wv, window, scale)
 
 
 @pytest.mark.parametrize("topk,window,S,heads", [(512, 128, 1, 128), (1024, 128, 4, 128),

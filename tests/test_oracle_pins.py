@@ -345,6 +345,66 @@ def test_page_ratios_stated_for_128k():
         assert abs(vals[name] - float(stated)) <= float(tol), (name, vals[name])
 
 
+# ---------------------------------------------------------------- CSA window
+PAGE_T = 64          # tokens per latent-cache page of the oracle
+
+
+def _csa_case(seed, n_pages=8, one_row=False):
+    rng = np.random.default_rng(seed)
+    vals = rng.standard_normal((n_pages, PAGE_T, 576))
+    if one_row:
+        vals[:] = rng.standard_normal(576)
+    pool = _bf16_bits(vals)
+    perm = rng.permutation(n_pages)
+    return rng, pool, perm[:2], perm[2:]          # compressed pages, raw pages
+
+
+def test_csa_window_zero_is_sparse_mla():
+    rng, pool, pc, pr = _csa_case(1)
+    q = O.bf16_decode(_bf16_bits(rng.standard_normal((64, 576))))
+    sel = rng.choice(2 * PAGE_T, 37, replace=False)
+    o, l = O.csa_window_attention(q, pool, pc, pr, sel, 150, 0, 0.07)
+    o2, l2 = O.sparse_mla(q, O.latent_rows(pool, pc, sel), 0.07)
+    assert np.array_equal(o, o2) and np.array_equal(l, l2)
+
+
+@pytest.mark.parametrize("win_vis,window", [(200, 128), (5, 128), (0, 16)])
+def test_csa_identical_rows_closed_form(win_vis, window):
+    """Every row the same latent c: O = c[:512] and LSE = scale q.c + ln(n), with
+    n = the selected entries plus the window tokens at or after position 0."""
+    rng, pool, pc, pr = _csa_case(2, one_row=True)
+    c = O.bf16_decode(pool[0, 0])
+    q = O.bf16_decode(_bf16_bits(rng.standard_normal((128, 576))))
+    sel = rng.choice(2 * PAGE_T, 9, replace=False)
+    o, l = O.csa_window_attention(q, pool, pc, pr, sel, win_vis, window, 0.05)
+    n = 9 + min(window, win_vis)
+    assert np.allclose(o, np.broadcast_to(c[:512], o.shape), rtol=0, atol=1e-12)
+    assert np.allclose(l, 0.05 * (q @ c) + math.log(n), rtol=0, atol=1e-12)
+
+
+def test_csa_window_before_token_zero_keeps_only_nonnegative_tokens():
+    rng, pool, pc, pr = _csa_case(3)
+    q = O.bf16_decode(_bf16_bits(rng.standard_normal((128, 576))))
+    sel = rng.choice(2 * PAGE_T, 20, replace=False)
+    o, l = O.csa_window_attention(q, pool, pc, pr, sel, 5, 128, 0.06)
+    o2, l2 = O.csa_window_attention(q, pool, pc, pr, sel, 5, 5, 0.06)
+    assert np.array_equal(o, o2) and np.array_equal(l, l2)
+    assert np.array_equal(O.csa_window_positions(5, 128), np.arange(5))
+
+
+@pytest.mark.parametrize("win_vis", [1, 64, 300])
+def test_csa_one_token_window_is_the_latest_raw_token(win_vis):
+    """No selected entry and a window of 1: the attention is the latent of raw
+    token win_vis-1 (a softmax over one row), LSE = scale q.c."""
+    rng, pool, pc, pr = _csa_case(4)
+    q = O.bf16_decode(_bf16_bits(rng.standard_normal((64, 576))))
+    o, l = O.csa_window_attention(q, pool, pc, pr, np.zeros(0, np.int64), win_vis, 1, 0.08)
+    t = win_vis - 1
+    c = O.bf16_decode(pool[pr[t // PAGE_T], t % PAGE_T])
+    assert np.allclose(o, np.broadcast_to(c[:512], o.shape), rtol=0, atol=1e-12)
+    assert np.allclose(l, 0.08 * (q @ c), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- planted slips
 def test_planted_mistakes_are_caught(monkeypatch):
     """Each slip planted in the oracle must make a pin fail."""
@@ -369,7 +429,21 @@ def test_planted_mistakes_are_caught(monkeypatch):
         o, l = real_mla(q, rows, scale)
         return real_mla(q, np.concatenate([rows[:, 64:], rows[:, :64]], 1), scale)[0], l
 
-    caught = []
+    import oracle.dsa_oracle as OD
+    real_window = OD.csa_window_positions
+
+    def window_shifted(win_vis, window):
+        return real_window(win_vis, window) - 1
+
+    monkeypatch.setattr(OD, "csa_window_positions", window_shifted)
+    try:
+        test_csa_one_token_window_is_the_latest_raw_token(64)
+        window_caught = False
+    except (AssertionError, IndexError):
+        window_caught = True
+    monkeypatch.setattr(OD, "csa_window_positions", real_window)
+
+    caught = [("window", window_caught)]
     for name, fn, attr, pins in [
         ("relu", no_relu, "indexer_scores", [lambda: test_indexer_relu_sign_identity(32),
                                              lambda: test_indexer_one_hot_keys_closed_form(64)]),
