@@ -43,6 +43,8 @@ def parse():
                     help="CPU work budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip timing the other synthetic configs after the headline one")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's sequence count (small profiling cases)")
     ap.add_argument("--tier", action="store_true",
@@ -329,6 +331,110 @@ def oracle_sample(inp, seconds):
 
 
 # ---------------------------------------------------------------- our arm
+# BASELINE's five synthetic configs (MTP verify in both modes), timed one
+# after another in the default run: config 1 is the headline `value`
+PER_WORKLOAD = ["decode_b1_ctx8k", "decode_b32_ctx128k", "indexshare4_b64_ctx16k_128k",
+                "mtp_verify_b16_t8_ctx128k", "mtp_verify_reuse_b16_t8_ctx128k",
+                "decode_b4_ctx1m_split16"]
+
+
+class StepRunner:
+    """One workload's device buffers and its decode step through the binding."""
+
+    def __init__(self, inp, dsa, dev, stream):
+        import torch
+        self.inp, self.dsa, self.stream = inp, dsa, stream
+        Q, G, n = inp.Q, inp.index_share, inp.n_layers
+        self.ws = dsa.workspace(Q, inp.max_len, inp.topk, inp.num_splits, device=dev)
+        self.outs = [torch.empty(Q, inp.heads, 512, device=dev) for _ in range(n)]
+        self.lses = [torch.empty(Q, inp.heads, device=dev) for _ in range(n)]
+        ng = (n + G - 1) // G
+        self.idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=dev)
+        self.qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
+        self.wl = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
+        self.kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
+        self.qs = [L["q"] for L in inp.layers]
+        self.pools = [L["pool"] for L in inp.layers]
+        self.pts = [inp.page_table] * n
+
+    def step(self, q_layers=None, qi=None, wl=None, out_layers=None, lse_layers=None):
+        inp = self.inp
+        self.dsa.dsa_decode_step(qi or self.qi, wl or self.wl, self.kl, inp.seq_offsets,
+                                 inp.q_offsets, inp.q_vis, inp.B, inp.max_len, inp.topk,
+                                 q_layers or self.qs, self.pools, self.pts, inp.scale,
+                                 out_layers or self.outs, lse_layers or self.lses, self.idx,
+                                 self.ws, index_share=inp.index_share,
+                                 mtp_index_share=inp.mtp_index_share,
+                                 num_splits=inp.num_splits, stream=self.stream)
+
+    def stage_times(self, flush, steps):
+        """The same kernels as the step, decomposed (indexer, top-k, one layer's
+        sparse MLA with its merge), each timed live with CUDA events; ms."""
+        import torch
+        inp, dsa, stream = self.inp, self.dsa, self.stream
+        scores = torch.empty(inp.Q, ((inp.max_len + 63) // 64) * 64, device=self.idx.device)
+        first = inp.mtp_index_share
+        evs = []
+        for _ in range(steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+            dsa.dsa_indexer_scores(self.qi[0], self.wl[0], self.kl[0], inp.seq_offsets,
+                                   inp.q_offsets, inp.q_vis, inp.B, inp.max_len, scores, self.ws,
+                                   first_only=first, stream=stream)
+            e[1].record(stream)
+            dsa.dsa_topk_select(scores, inp.q_offsets, inp.q_vis, inp.B, inp.max_len, inp.topk,
+                                self.idx[0], self.ws, first_only=first, stream=stream)
+            e[2].record(stream)
+            dsa.dsa_sparse_mla_decode(self.qs[0], self.pools[0], self.pts[0], inp.q_offsets,
+                                      inp.q_vis, self.idx[0], inp.B, inp.scale, self.outs[0],
+                                      self.lses[0], self.ws, num_splits=inp.num_splits,
+                                      stream=stream)
+            e[3].record(stream)
+            evs.append(e)
+        torch.cuda.synchronize(self.idx.device)
+        dsa.dsa_check_error(self.ws, stream)
+        return {"indexer": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+                "topk": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+                "mla": statistics.mean(e[2].elapsed_time(e[3]) for e in evs)}
+
+
+def time_steps(runner, flush, steps, warmup, dev):
+    """Device time of each of `steps` decode steps (L2 flushed before each step,
+    outside the events), after `warmup` untimed steps; ms per step."""
+    import torch
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        runner.step()
+    runner.dsa.dsa_check_error(runner.ws, runner.stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(runner.stream)
+        runner.step()
+        evs[i][1].record(runner.stream)
+    torch.cuda.synchronize(dev)
+    runner.dsa.dsa_check_error(runner.ws, runner.stream)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def workload_summary(inp, step_ms, stages, hbm):
+    """Per-workload figures of merit: step time, query-tokens/s, the step's
+    roofline fraction (indexer keys + gathered latents over the step time)
+    and the indexer's fraction of the measured copy bandwidth."""
+    key_b, gat_b = algorithmic_bytes(inp)
+    ms = statistics.mean(step_ms)
+    ng = (inp.n_layers + inp.index_share - 1) // inp.index_share
+    idx_gbs = key_b // ng / (stages["indexer"] / 1e3) / 1e9
+    return {"step_us": ms * 1e3, "q_tok_s": inp.Q / (ms / 1e3),
+            "step_roofline_frac_of_measured": (key_b + gat_b) / (ms / 1e3) / 1e9 / hbm,
+            "step_roofline_frac_of_8tbs": (key_b + gat_b) / (ms / 1e3) / 8e12,
+            "indexer_frac_of_measured": idx_gbs / hbm,
+            "stages_us": {k: v * 1e3 for k, v in stages.items()},
+            "bytes_per_step": key_b + gat_b, "queries_per_step": inp.Q}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -345,26 +451,13 @@ def run_ours(args, rank, world, local_rank):
     wl = get_workload(args.workload, **({"B": args.batch} if args.batch else {}))
     inp = make_inputs(wl, seed=args.seed + rank, device=dev)
     Q, G, n = inp.Q, inp.index_share, inp.n_layers
+    ng = (n + G - 1) // G
     S = inp.num_splits
     stream = torch.cuda.current_stream(dev)
-    ws = dsa.workspace(Q, inp.max_len, inp.topk, S, device=dev)
-    outs = [torch.empty(Q, inp.heads, 512, device=dev) for _ in range(n)]
-    lses = [torch.empty(Q, inp.heads, device=dev) for _ in range(n)]
-    ng = (n + G - 1) // G
-    idx = torch.empty(ng, Q, inp.topk, dtype=torch.int32, device=dev)
-    qi = [inp.indexer[l // G]["q_idx"] if l % G == 0 else None for l in range(n)]
-    wl_ = [inp.indexer[l // G]["w"] if l % G == 0 else None for l in range(n)]
-    kl = [inp.indexer[l // G]["k_idx"] if l % G == 0 else None for l in range(n)]
-    qs = [L["q"] for L in inp.layers]
-    pools = [L["pool"] for L in inp.layers]
-    pts = [inp.page_table] * n
+    runner = StepRunner(inp, dsa, dev, stream)
+    ws, outs, lses, idx = runner.ws, runner.outs, runner.lses, runner.idx
+    qi, wl_, kl, qs, pools, pts = runner.qi, runner.wl, runner.kl, runner.qs, runner.pools, runner.pts
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def step(q_layers=qs, out_layers=outs, lse_layers=lses):
-        dsa.dsa_decode_step(qi, wl_, kl, inp.seq_offsets, inp.q_offsets, inp.q_vis, inp.B,
-                            inp.max_len, inp.topk, q_layers, pools, pts, inp.scale, out_layers,
-                            lse_layers, idx, ws, index_share=G, mtp_index_share=inp.mtp_index_share,
-                            num_splits=S, stream=stream)
 
     def barrier():
         if dist is not None:
@@ -373,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
-        step()
+        runner.step()
     dsa.dsa_check_error(ws, stream)
 
     # ---- timed region: K steps, L2 flushed between steps (outside the events)
@@ -386,7 +479,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.steps):
             flush.zero_()
             evs[i][0].record(stream)
-            step()
+            runner.step()
             evs[i][1].record(stream)
         barrier()
         t_wall = time.perf_counter() - t_wall
@@ -397,29 +490,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = reduce_over_ranks(sum(step_ms), world, dist, dev)
 
     # ---- per-kernel breakdown of the same step, live (decomposed calls, same kernels)
-    scores = torch.empty(Q, ((inp.max_len + 63) // 64) * 64, device=dev)
-    first = inp.mtp_index_share
-    stage = {"indexer": [], "topk": [], "mla": []}
-    for i in range(args.steps):
-        flush.zero_()
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        e[0].record(stream)
-        dsa.dsa_indexer_scores(qi[0], wl_[0], kl[0], inp.seq_offsets, inp.q_offsets, inp.q_vis,
-                               inp.B, inp.max_len, scores, ws, first_only=first, stream=stream)
-        e[1].record(stream)
-        dsa.dsa_topk_select(scores, inp.q_offsets, inp.q_vis, inp.B, inp.max_len, inp.topk,
-                            idx[0], ws, first_only=first, stream=stream)
-        e[2].record(stream)
-        dsa.dsa_sparse_mla_decode(qs[0], pools[0], pts[0], inp.q_offsets, inp.q_vis, idx[0], inp.B,
-                                  inp.scale, outs[0], lses[0], ws, num_splits=S, stream=stream)
-        e[3].record(stream)
-        stage["_ev"] = stage.get("_ev", []) + [e]
-    torch.cuda.synchronize(dev)
-    for e in stage.pop("_ev"):
-        stage["indexer"].append(e[0].elapsed_time(e[1]))
-        stage["topk"].append(e[1].elapsed_time(e[2]))
-        stage["mla"].append(e[2].elapsed_time(e[3]))
-    dsa.dsa_check_error(ws, stream)
+    stages = runner.stage_times(flush, args.steps)
 
     # ---- end to end through the public API with host buffers: every step
     # copies its inputs from pinned host memory, runs the decode step and reads
@@ -533,7 +604,7 @@ def run_ours(args, rank, world, local_rank):
 
     key_b, gat_b = algorithmic_bytes(inp)
     hbm, hbm_kind = peaks()
-    idx_ms = statistics.mean(stage["indexer"])
+    idx_ms = stages["indexer"]
     idx_bytes = key_b // ((n + G - 1) // G)
     achieved = idx_bytes / (idx_ms / 1e3) / 1e9
     step_mean_ms = total_ms / args.steps
@@ -554,7 +625,7 @@ def run_ours(args, rank, world, local_rank):
                           "achieved_gbs": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9,
                           "frac_of_measured": (key_b + gat_b) / (step_mean_ms / 1e3) / 1e9 / hbm,
                           "frac_of_8tbs": (key_b + gat_b) / (step_mean_ms / 1e3) / 8e12},
-        "stages_ms": {k: statistics.mean(v) for k, v in stage.items()},
+        "stages_ms": stages,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
@@ -562,6 +633,25 @@ def run_ours(args, rank, world, local_rank):
         v, sample, cores = oracle_sample(inp, args.cpu_seconds)
         res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
+    if world == 1 and not args.no_per_workload and not args.batch and wl.name == DEFAULT_WORKLOAD:
+        # every synthetic config, each timed the same way (its own warm-up,
+        # K steps with the L2 flushed before each, the live stage split); the
+        # CPU and end-to-end legs stay with the headline config
+        per = {}
+        own = workload_summary(inp, step_ms, stages, hbm)
+        del runner, ws, outs, lses, idx, qi, wl_, kl, qs, pools, pts
+        for name in PER_WORKLOAD:
+            if name == wl.name:
+                per[name] = own
+                continue
+            w2 = get_workload(name)
+            inp2 = make_inputs(w2, seed=args.seed, device=dev)
+            r2 = StepRunner(inp2, dsa, dev, stream)
+            ms2 = time_steps(r2, flush, args.steps, args.warmup, dev)
+            per[name] = workload_summary(inp2, ms2, r2.stage_times(flush, args.steps), hbm)
+            del r2, inp2
+            torch.cuda.empty_cache()
+        res["per_workload"] = per
     return res
 
 

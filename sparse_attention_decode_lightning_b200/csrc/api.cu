@@ -8,16 +8,6 @@
 
 namespace dsa {
 
-cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool,
-                                   int num_pages, int page_size, const int32_t* page_table,
-                                   int max_pages,
-                                   const int32_t* q_offsets, const int32_t* q_vis,
-                                   const int32_t* idx, int B, int Q, int H, int topk,
-                                   float scale, int S, float* out, float* lse, float* o_part,
-                                   float* l_part, uint32_t* err, cudaStream_t st, bool pdl,
-                                   const int32_t* win_page_table, int win_max_pages,
-                                   const int32_t* win_vis, int window, bool kv8, float kv_scale);
-
 namespace {
 
 constexpr int B200_SMS = 148;

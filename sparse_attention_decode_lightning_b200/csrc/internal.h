@@ -88,6 +88,18 @@ cudaError_t launch_sparse_mla(const __nv_bfloat16* q, const __nv_bfloat16* pool,
                               const int32_t* win_vis = nullptr, int window = 0,
                               bool kv8 = false, float kv_scale = 1.f);
 
+// the sparse MLA kernel itself (sparse_mla_sm100.cu): o_part / l_part hold
+// the split partials when S > 1; err may be null (nothing is reported)
+cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
+                                 int page_size, const int32_t* page_table, int max_pages,
+                                 const int32_t* q_offsets, const int32_t* q_vis,
+                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
+                                 int S, float* out, float* lse, float* o_part, float* l_part,
+                                 uint32_t* err, cudaStream_t st, bool pdl,
+                                 const int32_t* win_page_table = nullptr, int win_max_pages = 0,
+                                 const int32_t* win_vis = nullptr, int window = 0,
+                                 bool kv8 = false, float kv_scale = 1.f);
+
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
                            float* out, float* lse, cudaStream_t st, bool pdl);
 

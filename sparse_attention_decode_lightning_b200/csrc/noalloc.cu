@@ -20,16 +20,6 @@
 
 namespace dsa {
 
-cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                                 int page_size, const int32_t* page_table, int max_pages,
-                                 const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
-                                 int S, float* out, float* lse, float* o_part, float* l_part,
-                                 uint32_t* err, cudaStream_t st, bool pdl,
-                                 const int32_t* win_page_table = nullptr, int win_max_pages = 0,
-                                 const int32_t* win_vis = nullptr, int window = 0,
-                                 bool kv8 = false, float kv_scale = 1.f);
-
 namespace {
 
 constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;   // 16 MiB per device

@@ -75,7 +75,7 @@ constexpr int OFF_X = OFF_ST + NST * STAGE_BYTES;
 constexpr int OFF_MX = OFF_X + 2 * X_BYTES;    // [2 tiles][2 warpgroups][128 heads] partial maxima
 constexpr int OFF_CRD = OFF_MX + 2 * 2 * DSA_HEADS * 4;
 constexpr int OFF_BAR = OFF_CRD + DSA_MAX_TOPK * 4;
-constexpr int NBAR = 2 * NST + 4 * 2 + 2;
+constexpr int NBAR = 2 * NST + 5 * 2 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "sparse MLA shared memory exceeds the sm_100 limit");
@@ -113,17 +113,31 @@ struct MlaTcArgs {
   uint32_t* err;
 };
 
-__device__ __forceinline__ int seq_of_query(const int32_t* q_offsets, int B, int q) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (q_offsets[mid] <= q) lo = mid; else hi = mid - 1;
+// Sequence of query q: the largest b < B with q_offsets[b] <= q, found by a
+// full warp in rounds of 32 parallel probes (one round for B <= 32, three
+// for B = 2048) instead of a chain of dependent loads.
+__device__ __forceinline__ int seq_of_query_warp(const int32_t* q_offsets, int B, int q, int lane) {
+  int lo = 0, hi = B;                  // q_offsets[lo] <= q; the answer lies in [lo, hi)
+  while (hi - lo > 1) {
+    const int step = (hi - lo + 31) / 32;
+    const int i = lo + lane * step;
+    const uint32_t m = __ballot_sync(0xffffffffu, i < hi && __ldg(q_offsets + i) <= q);
+    lo += (31 - __clz(m)) * step;      // lane 0 probes lo itself, so m != 0
+    hi = min(hi, lo + step);
   }
   return lo;
 }
 
+
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   const bool ok = mbar_wait(bar, parity, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// the same for a barrier that the peer CTA arrives on (acquire at cluster scope)
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const bool ok = mbar_wait_cluster(bar, parity, err);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -190,7 +204,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* p_full = s_full + 2;         // [2] P of a tile is in its slot
   uint64_t* slot_free = p_full + 2;      // [2] PV of the slot's tile is done
   uint64_t* x_full = slot_free + 2;      // [2] the peer's partial scores arrived
-  uint64_t* o_final = x_full + 2;        // last PV
+  uint64_t* x_free = x_full + 2;         // [2] the peer has read my partial from its slot
+  uint64_t* o_final = x_free + 2;        // last PV
   uint64_t* q_ready = o_final + 1;       // query slice in TMEM / shared memory
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
@@ -199,7 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   pdl_trigger();
   const int unit = blockIdx.x >> 1;
   const int q = unit / a.S, split = unit % a.S;
-  const int b = seq_of_query(a.q_offsets, a.B, q);
+  const int b = seq_of_query_warp(a.q_offsets, a.B, q, lane);
   int vis = a.q_vis[q];
   if (vis < 0) vis = 0;
   const int total = a.topk + a.window;             // selected entries, then the window
@@ -219,6 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&p_full[i], SMX_WARPS);  // one arrival per softmax warp
       mbar_init(&slot_free[i], 1);
       mbar_init(&x_full[i], 1);   // armed with the tile's bytes; the peer's st.async complete them
+      mbar_init(&x_free[i], SMX_WARPS);      // remote arrivals of the peer's softmax warps
     }
     mbar_init(o_final, 1);
     mbar_init(q_ready, 5);             // 4 query-loading warps + thread 0 with the RoPE bytes
@@ -398,51 +414,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t peer = rank ^ 1u;
     const uint32_t peer_x = map_to_rank(smem_u32(xb), peer);
     const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
+    const uint32_t peer_xfree = map_to_rank(smem_u32(x_free), peer);
     // partial scores are exchanged by push: each CTA stores its partial into
     // the peer's shared memory with st.async and reads the peer's from its own
-    if (g == 0 && live) {
-      // this CTA's 256 latent query dims of head h -> tensor memory (bf16 pairs)
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float w[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = __ldg(src + c * 8 + i);
-          w[4 * i + 0] = __uint_as_float(v.x);
-          w[4 * i + 1] = __uint_as_float(v.y);
-          w[4 * i + 2] = __uint_as_float(v.z);
-          w[4 * i + 3] = __uint_as_float(v.w);
-        }
-        tmem_st32(lane_base + Q_COL + c * 32, w);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-    }
     if (g == 0) {
+      if (live) {
+        // head h's 256 latent query dims of this CTA -> tensor memory (bf16 pairs)
+        const uint4* src = reinterpret_cast<const uint4*>(
+            a.q + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float w[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 v = __ldg(src + c * 8 + i);
+            w[4 * i + 0] = __uint_as_float(v.x);
+            w[4 * i + 1] = __uint_as_float(v.y);
+            w[4 * i + 2] = __uint_as_float(v.z);
+            w[4 * i + 3] = __uint_as_float(v.w);
+          }
+          tmem_st32(lane_base + Q_COL + c * 32, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
     float m_use = -INFINITY, l = 0.f;                // l: this warpgroup's rows only
     bool ok = true;
-    for (int t = 0; t < ntiles && ok; ++t) {
+    // A wait that runs out clears ok; the warp then skips its remaining waits
+    // and data movement but keeps every barrier arrival, so no other warp of
+    // the block is left waiting on it.
+    for (int t = 0; t < ntiles; ++t) {
       const int sb = t & 1;
       const uint32_t ph = (t >> 1) & 1;
-      if (!live) {
-        // no heads in these lanes: only the tile-max barrier and the P arrival
-        named_barrier(1, 32 * SMX_WARPS);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sb]);
-        continue;
-      }
       const int j = t * NR + 32 * g + lane;
       const uint32_t vm = __ballot_sync(0xffffffffu, j < nrows && crd[j] >= 0);
-      if (!(ok = warp_wait(&s_full[sb], ph, a.err))) break;
-      tc_fence_after();
       float z[32];
-      tmem_ld32(lane_base + S_COL + sb * NR + 32 * g, z);
-      tmem_ld_wait();
+      float mt0 = -INFINITY, mt1 = -INFINITY;
+      const float sl = a.scale_log2;
       // my partial -> the peer's receive slot, pushed with st.async: every
       // 16-byte store completes its bytes on the peer's x_full[sb], whose
       // expected count (the whole 24 KB tile) one thread of the peer arms.
@@ -451,119 +462,136 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // three words, a quarter fewer bytes over the ~16 B/cycle DSMEM link.
       // Slot layout [16-byte chunk k][warpgroup][head]: a warp's chunk k is
       // 512 contiguous bytes, bank-conflict free; the peer fills mine alike.
+      // The peer's slot sb is written again only after the peer has read
+      // tile t-2 from it (its remote arrival on x_free[sb]).
+      // My receive slot of tile t-1 has been read (its values went into
+      // tile t-1's softmax, which is finished): the peer may push tile t+1
+      // into it.  The arrival needs no release fence, which would also wait
+      // for this thread's own remote stores (measured ~9 us a launch against
+      // ~2 us for this form).
+      if (t >= 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(peer_xfree + ((t - 1) & 1) * 8);
+      }
       if (g == 0 && quarter == 0 && lane == 0)
         mbar_arrive_expect_tx(&x_full[sb], static_cast<uint32_t>(NH) * (NR * 3));
-      uint32_t u[32];
+      if (live) {
+        if (ok) ok = warp_wait(&s_full[sb], ph, a.err);
+        tc_fence_after();
+        tmem_ld32(lane_base + S_COL + sb * NR + 32 * g, z);
+        tmem_ld_wait();
+        uint32_t u[32];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) u[r] = round_to_24bit(z[r]);
-      const uint32_t xoff = sb * X_BYTES + (g * DSA_HEADS + h) * 16;
+        for (int r = 0; r < 32; ++r) u[r] = round_to_24bit(z[r]);
+        const uint32_t xoff = sb * X_BYTES + (g * DSA_HEADS + h) * 16;
+        if (ok && t >= 2) ok = warp_wait_cluster(&x_free[sb], ((t >> 1) - 1) & 1, a.err);
+        if (ok) {
 #pragma unroll
-      for (int k = 0; k < 6; ++k) {
-        // chunk k holds words 4k .. 4k+3 of the 24 packed words (values 16k/3 ..)
-        uint32_t w[4];
+          for (int k = 0; k < 6; ++k) {
+            // chunk k holds words 4k .. 4k+3 of the 24 packed words (values 16k/3 ..)
+            uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = pack24_word(u, 4 * k + e);
-        st_async_v4(peer_x + xoff + k * (2 * DSA_HEADS * 16), __uint_as_float(w[0]),
-                    __uint_as_float(w[1]), __uint_as_float(w[2]), __uint_as_float(w[3]),
-                    peer_xfull + sb * 8);
-      }
-      const bool got = mbar_wait_cluster(&x_full[sb], ph, a.err);
-      if (!(ok = __all_sync(0xffffffffu, got))) break;
-      float4 xs[8];
-      {
-        uint32_t pw[24];
-#pragma unroll
-        for (int k = 0; k < 6; ++k) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (2 * DSA_HEADS * 16));
-          pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          xs[i].x = __uint_as_float(unpack24(pw, 4 * i + 0));
-          xs[i].y = __uint_as_float(unpack24(pw, 4 * i + 1));
-          xs[i].z = __uint_as_float(unpack24(pw, 4 * i + 2));
-          xs[i].w = __uint_as_float(unpack24(pw, 4 * i + 3));
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 32; ++r) z[r] = __uint_as_float(u[r]);
-      // own + peer: rank 0 adds S0 + S1, rank 1 adds S1 + S0; fp32 addition
-      // commutes, so both CTAs hold the same z
-      float mt0 = -INFINITY, mt1 = -INFINITY;
-      const float sl = a.scale_log2;
-      if (vm == 0xffffffffu) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          z[4 * i + 0] = (z[4 * i + 0] + xs[i].x) * sl;
-          z[4 * i + 1] = (z[4 * i + 1] + xs[i].y) * sl;
-          z[4 * i + 2] = (z[4 * i + 2] + xs[i].z) * sl;
-          z[4 * i + 3] = (z[4 * i + 3] + xs[i].w) * sl;
-          mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
-          mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float s4[4] = {xs[i].x, xs[i].y, xs[i].z, xs[i].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = 4 * i + e;
-            z[r] = ((vm >> r) & 1u) ? (z[r] + s4[e]) * sl : -INFINITY;
+            for (int e = 0; e < 4; ++e) w[e] = pack24_word(u, 4 * k + e);
+            st_async_v4(peer_x + xoff + k * (2 * DSA_HEADS * 16), __uint_as_float(w[0]),
+                        __uint_as_float(w[1]), __uint_as_float(w[2]), __uint_as_float(w[3]),
+                        peer_xfull + sb * 8);
           }
-          mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
-          mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+        }
+        if (ok) ok = warp_wait_cluster(&x_full[sb], ph, a.err);
+        float4 xs[8];
+        {
+          uint32_t pw[24];
+#pragma unroll
+          for (int k = 0; k < 6; ++k) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (2 * DSA_HEADS * 16));
+            pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            xs[i].x = __uint_as_float(unpack24(pw, 4 * i + 0));
+            xs[i].y = __uint_as_float(unpack24(pw, 4 * i + 1));
+            xs[i].z = __uint_as_float(unpack24(pw, 4 * i + 2));
+            xs[i].w = __uint_as_float(unpack24(pw, 4 * i + 3));
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 32; ++r) z[r] = __uint_as_float(u[r]);
+        // own + peer: rank 0 adds S0 + S1, rank 1 adds S1 + S0; fp32 addition
+        // commutes, so both CTAs hold the same z
+        if (vm == 0xffffffffu) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            z[4 * i + 0] = (z[4 * i + 0] + xs[i].x) * sl;
+            z[4 * i + 1] = (z[4 * i + 1] + xs[i].y) * sl;
+            z[4 * i + 2] = (z[4 * i + 2] + xs[i].z) * sl;
+            z[4 * i + 3] = (z[4 * i + 3] + xs[i].w) * sl;
+            mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
+            mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float s4[4] = {xs[i].x, xs[i].y, xs[i].z, xs[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = 4 * i + e;
+              z[r] = ((vm >> r) & 1u) ? (z[r] + s4[e]) * sl : -INFINITY;
+            }
+            mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
+            mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+          }
         }
       }
       // tile maximum over both warpgroups' rows
       float* mxt = mx + (t & 1) * 2 * DSA_HEADS;
       mxt[g * DSA_HEADS + h] = fmaxf(mt0, mt1);
       named_barrier(1, 32 * SMX_WARPS);
-      const float mt = fmaxf(mxt[h], mxt[DSA_HEADS + h]);
-      // running max, moved only when it grows by more than 8 (a factor 2^8);
-      // identical in both warpgroups and both CTAs
-      float alpha = 1.f;
-      bool resc = false;
-      if (mt > m_use + 8.f) {
-        if (m_use != -INFINITY) {
-          alpha = fast_exp2(m_use - mt);
-          resc = true;
+      if (live) {
+        const float mt = fmaxf(mxt[h], mxt[DSA_HEADS + h]);
+        // running max, moved only when it grows by more than 8 (a factor 2^8);
+        // identical in both warpgroups and both CTAs
+        float alpha = 1.f;
+        bool resc = false;
+        if (mt > m_use + 8.f) {
+          if (m_use != -INFINITY) {
+            alpha = fast_exp2(m_use - mt);
+            resc = true;
+          }
+          m_use = mt;
         }
-        m_use = mt;
-      }
-      const float m_eff = m_use == -INFINITY ? 0.f : m_use;   // exp2(-inf - m_eff) = 0
-      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+        const float m_eff = m_use == -INFINITY ? 0.f : m_use;   // exp2(-inf - m_eff) = 0
+        float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
 #pragma unroll
-      for (int r = 0; r < 32; r += 4) {
-        z[r + 0] = fast_exp2(z[r + 0] - m_eff);
-        z[r + 1] = fast_exp2(z[r + 1] - m_eff);
-        z[r + 2] = fast_exp2(z[r + 2] - m_eff);
-        z[r + 3] = fast_exp2(z[r + 3] - m_eff);
-        ps0 += z[r + 0];
-        ps1 += z[r + 1];
-        ps2 += z[r + 2];
-        ps3 += z[r + 3];
-      }
-      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
-      // O is rescaled (rarely: only when the running max moves) after PV(t-1)
-      // has finished, which completes phase (t-1)/2 of slot_free[(t-1)&1];
-      // PV(t+1) needs P(t+1), so that barrier cannot have moved further.
-      // Without a rescale P(t) is published at once, and PV(t-1) runs
-      // behind the scores MMA of tile t+1 without holding up the softmax.
-      if (g == 0 && __any_sync(0xffffffffu, resc)) {
-        if (t >= 1 && !(ok = warp_wait(&slot_free[(t - 1) & 1], ((t - 1) >> 1) & 1, a.err))) break;
-        tc_fence_after();
-        for (int c = 0; c < 256 / 32; ++c) {
-          float o[32];
-          tmem_ld32(lane_base + O_COL + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(lane_base + O_COL + c * 32, o);
+        for (int r = 0; r < 32; r += 4) {
+          z[r + 0] = fast_exp2(z[r + 0] - m_eff);
+          z[r + 1] = fast_exp2(z[r + 1] - m_eff);
+          z[r + 2] = fast_exp2(z[r + 2] - m_eff);
+          z[r + 3] = fast_exp2(z[r + 3] - m_eff);
+          ps0 += z[r + 0];
+          ps1 += z[r + 1];
+          ps2 += z[r + 2];
+          ps3 += z[r + 3];
         }
-      }
-      // P as bf16 hi (slot columns [16g, 16g+16)) + lo ([32+16g, 32+16g+16)),
-      // two rows per column
-      {
+        l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
+        // O is rescaled (rarely: only when the running max moves) after PV(t-1)
+        // has finished, which completes phase (t-1)/2 of slot_free[(t-1)&1];
+        // PV(t+1) needs P(t+1), so that barrier cannot have moved further.
+        // Without a rescale P(t) is published at once, and PV(t-1) runs
+        // behind the scores MMA of tile t+1 without holding up the softmax.
+        if (g == 0 && __any_sync(0xffffffffu, resc)) {
+          if (ok && t >= 1) ok = warp_wait(&slot_free[(t - 1) & 1], ((t - 1) >> 1) & 1, a.err);
+          tc_fence_after();
+          for (int c = 0; c < 256 / 32; ++c) {
+            float o[32];
+            tmem_ld32(lane_base + O_COL + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(lane_base + O_COL + c * 32, o);
+          }
+        }
+        // P as bf16 hi (slot columns [16g, 16g+16)) + lo ([32+16g, 32+16g+16)),
+        // two rows per column
         float hi[16], lo[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
@@ -575,8 +603,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tmem_st16(lane_base + S_COL + sb * NR + 16 * g, hi);
         tmem_st16(lane_base + S_COL + sb * NR + 32 + 16 * g, lo);
+        tmem_st_wait();
       }
-      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[sb]);
