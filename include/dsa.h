@@ -290,9 +290,11 @@ dsa_status dsa_sparse_mla_decode_fp8(const void* q, const void* kv_pool, float k
  *   that device current); make that first call before any stream capture.
  *   All calls share the array and it keeps the last call's contents; calls
  *   whose work overlaps on the GPU (other streams, or several devices'
- *   threads racing on one device) race on it.  Nothing in it needs to start
- *   at zero.  Out-of-range indices or pages are skipped as in
- *   dsa_sparse_mla_decode but are not reported (there is no error word).
+ *   threads racing on one device) race on it.  Out-of-range indices or pages
+ *   are skipped as in dsa_sparse_mla_decode; they, and an expired
+ *   device-side wait, raise a flag in an error word at the start of the
+ *   array (zero when the library loads), which dsa_noalloc_check_error reads
+ *   and clears.  Nothing else in the array needs to start at zero.
  */
 dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool, int num_pages,
                                          int page_size, const int32_t* page_table, int max_pages,
@@ -300,6 +302,16 @@ dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* kv_pool, int
                                          const int32_t* idx, int B, int Q, int heads, int topk,
                                          float scale, int num_splits, float* out, float* lse,
                                          void* stream);
+
+/*
+ * The error word of dsa_sparse_mla_decode_noalloc on the current device:
+ * synchronises `stream`, reads the word and clears it.  Returns DSA_OK,
+ * DSA_ERR_DEVICE_BOUNDS (an index or page outside its range was skipped),
+ * DSA_ERR_TIMEOUT (a bounded device-side wait expired; the output of that
+ * call is not valid) or DSA_ERR_CUDA.  It allocates nothing either; the pages
+ * have no counterpart of it.
+ */
+dsa_status dsa_noalloc_check_error(void* stream);
 
 /*
  * Merge of split-K partial attentions (exact LSE combine).
@@ -442,6 +454,19 @@ dsa_status dsa_tier_swap_in(void* dev_state, size_t state_bytes, int B, int dev_
 dsa_status dsa_tier_dev_stats(const void* dev_state, int64_t* stats /* host int64 [5] */,
                               void* stream);
 const int32_t* dsa_tier_dev_copies(const void* dev_state, int B, int dev_slots, int max_pages);
+
+/*
+ * Self-test of the device-side failure detection (the pages have no
+ * counterpart; it exercises the library's own safety net).  One small kernel
+ * waits twice, with the library's bounded waits, on a barrier that never
+ * completes, each wait giving up after limit_us microseconds (1 .. 2,000,000;
+ * the library's own limit is 2 s), and raises the timeout flag in the error
+ * word of `ws` (>= 256 bytes, a workspace from dsa_workspace_bytes
+ * qualifies).  The kernel holds no copy, tensor memory or peer CTA, so it
+ * simply returns; a following dsa_check_error returns DSA_ERR_TIMEOUT and
+ * clears the flag, and the context stays usable.
+ */
+dsa_status dsa_selftest_bounded_wait(int limit_us, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Synchronises `stream`, reads and clears the workspace's device error flag.

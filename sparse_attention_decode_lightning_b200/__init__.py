@@ -65,6 +65,8 @@ SIGNATURES = {
     "dsa_tier_dev_stats": (_I, [_P, _P, _P]),
     "dsa_tier_dev_copies": (_P, [_P, _I, _I, _I]),
     "dsa_check_error": (_I, [_P, _P]),
+    "dsa_noalloc_check_error": (_I, [_P]),
+    "dsa_selftest_bounded_wait": (_I, [_I, _P, _SZ, _P]),
 }
 
 _lib = None
@@ -341,3 +343,14 @@ def dsa_tier_dev_copies(dev_state, B, dev_slots, max_pages, n):
 
 def dsa_check_error(ws, stream=None):
     _check(lib().dsa_check_error(_ptr(ws), _stream(stream)), "dsa_check_error")
+
+
+def dsa_selftest_bounded_wait(limit_us, ws, stream=None):
+    """Makes the library's bounded device-side waits run out (see include/dsa.h)."""
+    _check(lib().dsa_selftest_bounded_wait(int(limit_us), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_selftest_bounded_wait")
+
+
+def dsa_noalloc_check_error(stream=None):
+    """Reads and clears dsa_sparse_mla_decode_noalloc's error word (synchronises)."""
+    _check(lib().dsa_noalloc_check_error(_stream(stream)), "dsa_noalloc_check_error")

@@ -6,11 +6,22 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace dsa {
 
 namespace {
 
 constexpr int B200_SMS = 148;
+
+// NVTX range over a scope (header-only NVTX v3: no library to link; the
+// ranges cost nothing unless a profiler collects them)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -424,15 +435,19 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
   if (!ws_layout(Q, max_len, topk, num_splits, &L)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // host-side ranges: they mark when each stage's launches are enqueued
+  NvtxRange step_range("dsa_decode_step");
   for (int l = 0; l < n_layers; ++l) {
     const int g = l / index_share;
     int32_t* idx_g = idx_out + static_cast<size_t>(g) * Q * topk;
     if (l % index_share == 0) {
+      NvtxRange r("dsa_indexer_topk");
       s = do_indexer_topk(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys, seq_offsets,
                           q_offsets, q_vis, B, Q, idx_heads, max_len, topk, mtp_index_share, idx_g,
                           nullptr, ws, L, st);
       if (s != DSA_OK) return s;
     }
+    NvtxRange r("dsa_sparse_mla");
     s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
                       max_pages, q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S,
                       out_layers[l], lse_layers[l], ws, L, st, true);

@@ -80,17 +80,23 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// WAIT_LIMIT_NS, raises DEVERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// limit_ns nanoseconds of %globaltimer, raises DEVERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       raise_error(err, DEVERR_TIMEOUT);
       return false;
     }
   }
+}
+
+// the same with the library's limit, WAIT_LIMIT_NS
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  return mbar_wait_for(bar, parity, err, WAIT_LIMIT_NS);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -480,16 +486,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // bounded wait with acquire at cluster scope (for arrivals from the peer CTA)
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ bool mbar_wait_cluster_for(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                                      uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 1023u) == 0 && globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if ((it & 1023u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       raise_error(err, DEVERR_TIMEOUT);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  return mbar_wait_cluster_for(bar, parity, err, WAIT_LIMIT_NS);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

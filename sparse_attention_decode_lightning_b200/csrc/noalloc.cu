@@ -13,6 +13,9 @@
 // code its name is only a host-side stand-in, not a device address, so the
 // address is looked up once per device with cudaGetSymbolAddress (with that
 // device current) and cached; the first call on a device does that set-up.
+// Its first 256 bytes hold the device error word (zero when the library is
+// loaded, cleared again by dsa_noalloc_check_error); the split-K partials
+// follow.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,6 +28,7 @@ namespace {
 constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;   // 16 MiB per device
 constexpr size_t PART_O_BYTES = size_t(DSA_DIM_V) * 4;   // one head of one (query, split) output
 constexpr size_t PART_L_BYTES = 4;
+constexpr size_t ERR_BYTES = 256;                         // the error word, padded
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
@@ -76,21 +80,41 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const void* q, const void* k
   const int S = choose_splits(Q, topk, num_splits);
   const size_t parts = static_cast<size_t>(Q) * S * heads;      // (query, split, head) partials
   const size_t need = S > 1 ? parts * (PART_O_BYTES + PART_L_BYTES) : 0;
-  if (need > NOALLOC_SCRATCH_BYTES) return DSA_ERR_UNSUPPORTED;   // beyond the fixed array
+  if (need > NOALLOC_SCRATCH_BYTES - ERR_BYTES) return DSA_ERR_UNSUPPORTED;   // beyond the fixed array
   dsa_status st = DSA_OK;
   uint8_t* scratch = static_cast<uint8_t*>(scratch_ptr(&st));
   if (!scratch) return st;
-  float* o_part = reinterpret_cast<float*>(scratch);
-  float* l_part = reinterpret_cast<float*>(scratch + parts * PART_O_BYTES);
+  uint32_t* err = reinterpret_cast<uint32_t*>(scratch);
+  float* o_part = reinterpret_cast<float*>(scratch + ERR_BYTES);
+  float* l_part = reinterpret_cast<float*>(scratch + ERR_BYTES + parts * PART_O_BYTES);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // every partial is written by the kernel before the merge reads it, so the
-  // array needs no clearing; range violations are skipped but not reported
+  // every partial is written by the kernel before the merge reads it, so only
+  // the error word needs to start at zero (it does when the library loads,
+  // and dsa_noalloc_check_error clears it after reading)
   if (launch_sparse_mla_tc(static_cast<const __nv_bfloat16*>(q),
                            static_cast<const __nv_bfloat16*>(kv_pool), num_pages, page_size, page_table,
                            max_pages, q_offsets, q_vis, idx, B, Q, heads, topk, scale, S, out, lse,
-                           o_part, l_part, nullptr, s, false) != cudaSuccess)
+                           o_part, l_part, err, s, false) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (S > 1 && launch_combine(o_part, l_part, Q, S, heads, out, lse, s, true) != cudaSuccess)
     return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+extern "C" dsa_status dsa_noalloc_check_error(void* stream) {
+  dsa_status st = DSA_OK;
+  uint8_t* scratch = static_cast<uint8_t*>(scratch_ptr(&st));
+  if (!scratch) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  uint32_t flag = 0;
+  if (cudaMemcpy(&flag, scratch, sizeof(flag), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (flag) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(scratch, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  if (flag & DEVERR_TIMEOUT) return DSA_ERR_TIMEOUT;
+  if (flag & DEVERR_BOUNDS) return DSA_ERR_DEVICE_BOUNDS;
   return DSA_OK;
 }
