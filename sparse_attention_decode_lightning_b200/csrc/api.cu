@@ -437,21 +437,42 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // host-side ranges: they mark when each stage's launches are enqueued
   NvtxRange step_range("dsa_decode_step");
-  for (int l = 0; l < n_layers; ++l) {
-    const int g = l / index_share;
+  for (int l0 = 0; l0 < n_layers; l0 += index_share) {
+    const int g = l0 / index_share;
+    const int l1 = l0 + index_share < n_layers ? l0 + index_share : n_layers;
     int32_t* idx_g = idx_out + static_cast<size_t>(g) * Q * topk;
-    if (l % index_share == 0) {
+    {
       NvtxRange r("dsa_indexer_topk");
-      s = do_indexer_topk(q_idx_layers[l], w_layers[l], k_idx_layers[l], total_keys, seq_offsets,
-                          q_offsets, q_vis, B, Q, idx_heads, max_len, topk, mtp_index_share, idx_g,
-                          nullptr, ws, L, st);
+      s = do_indexer_topk(q_idx_layers[l0], w_layers[l0], k_idx_layers[l0], total_keys,
+                          seq_offsets, q_offsets, q_vis, B, Q, idx_heads, max_len, topk,
+                          mtp_index_share, idx_g, nullptr, ws, L, st);
       if (s != DSA_OK) return s;
     }
     NvtxRange r("dsa_sparse_mla");
-    s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
-                      max_pages, q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S,
-                      out_layers[l], lse_layers[l], ws, L, st, true);
-    if (s != DSA_OK) return s;
+    if (L.S == 1) {
+      // the layers that share this index set run as one grid over (layer,
+      // query): no launch waits for the last wave of the layer before it
+      for (int c0 = l0; c0 < l1; c0 += MLA_MAX_LAYERS_PER_LAUNCH) {
+        const int n = l1 - c0 < MLA_MAX_LAYERS_PER_LAUNCH ? l1 - c0 : MLA_MAX_LAYERS_PER_LAUNCH;
+        MlaLayerPtrs lp[MLA_MAX_LAYERS_PER_LAUNCH];
+        for (int i = 0; i < n; ++i)
+          lp[i] = {static_cast<const __nv_bfloat16*>(q_layers[c0 + i]),
+                   static_cast<const __nv_bfloat16*>(pool_layers[c0 + i]),
+                   page_table_layers[c0 + i], out_layers[c0 + i], lse_layers[c0 + i]};
+        if (launch_sparse_mla_layers(lp, n, num_pages, page_size, max_pages, q_offsets, q_vis,
+                                     idx_g, B, Q, heads, topk, scale, 1, nullptr, nullptr,
+                                     ws_ptr<uint32_t>(ws, L.err), st, true) != cudaSuccess)
+          return DSA_ERR_CUDA;
+      }
+      continue;
+    }
+    // with split-K the partial buffers hold one layer at a time
+    for (int l = l0; l < l1; ++l) {
+      s = do_sparse_mla(q_layers[l], pool_layers[l], num_pages, page_size, page_table_layers[l],
+                        max_pages, q_offsets, q_vis, idx_g, B, Q, heads, topk, scale, L.S,
+                        out_layers[l], lse_layers[l], ws, L, st, true);
+      if (s != DSA_OK) return s;
+    }
   }
   return DSA_OK;
 }

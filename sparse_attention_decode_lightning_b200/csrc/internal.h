@@ -100,6 +100,25 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  const int32_t* win_vis = nullptr, int window = 0,
                                  bool kv8 = false, float kv_scale = 1.f);
 
+// Several layers that share one index set (IndexShare) in one grid of
+// (layer, query, split) units; L <= 4, and L > 1 only with S == 1
+struct MlaLayerPtrs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* pool;
+  const int32_t* page_table;
+  float* out;
+  float* lse;
+};
+constexpr int MLA_MAX_LAYERS_PER_LAUNCH = 4;
+cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_pages,
+                                     int page_size, int max_pages, const int32_t* q_offsets,
+                                     const int32_t* q_vis, const int32_t* idx, int B, int Q, int H,
+                                     int topk, float scale, int S, float* o_part, float* l_part,
+                                     uint32_t* err, cudaStream_t st, bool pdl,
+                                     const int32_t* win_page_table = nullptr, int win_max_pages = 0,
+                                     const int32_t* win_vis = nullptr, int window = 0,
+                                     bool kv8 = false, float kv_scale = 1.f);
+
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
                            float* out, float* lse, cudaStream_t st, bool pdl);
 

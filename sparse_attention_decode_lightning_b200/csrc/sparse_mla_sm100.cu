@@ -86,10 +86,15 @@ constexpr uint32_t S_COL = 256;
 constexpr uint32_t Q_COL = 384;
 constexpr uint32_t TMEM_COLS = 512;
 
+// Layers of one launch (IndexShare: the layers that share an index set run
+// as one grid; their units are (layer, query, split))
+constexpr int MAX_LAYERS = MLA_MAX_LAYERS_PER_LAUNCH;
+
 struct MlaTcArgs {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* pool;
-  const int32_t* page_table;
+  const __nv_bfloat16* q[MAX_LAYERS];
+  const __nv_bfloat16* pool[MAX_LAYERS];
+  const int32_t* page_table[MAX_LAYERS];
+  int L;                                       // layers in this launch (1 with split-K)
   int max_pages;
   int num_pages;
   int page_shift;                              // log2 of the tokens per cache page
@@ -106,8 +111,8 @@ struct MlaTcArgs {
   int B, Q, topk, S;
   float scale_log2;
   float out_scale;                             // e4m3 cache: its per-tensor scale, else 1
-  float* out;
-  float* lse;
+  float* out[MAX_LAYERS];
+  float* lse[MAX_LAYERS];
   float* o_part;
   float* l_part;
   uint32_t* err;
@@ -185,10 +190,15 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
                     e4m3x2_to_bf16x2(v.y & 0xFFFFu), e4m3x2_to_bf16x2(v.y >> 16));
 }
 
+// the per-layer tensor maps: RoPE query dims, and the output
+struct MlaMaps {
+  CUtensorMap q[MAX_LAYERS];
+  CUtensorMap o[MAX_LAYERS];
+};
+
 template <int NH, bool KV8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                         const __grid_constant__ CUtensorMap tmap_o, MlaTcArgs a) {
+    sparse_mla_tc_kernel(const __grid_constant__ MlaMaps maps, const __grid_constant__ MlaTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -213,7 +223,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   pdl_trigger();
   const int unit = blockIdx.x >> 1;
-  const int q = unit / a.S, split = unit % a.S;
+  const int layer = unit / (a.Q * a.S);
+  const int q = (unit % (a.Q * a.S)) / a.S, split = unit % a.S;
   const int b = seq_of_query_warp(a.q_offsets, a.B, q, lane);
   int vis = a.q_vis[q];
   if (vis < 0) vis = 0;
@@ -247,9 +258,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   if (tid == 0) {
-    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&maps.q[layer]);
     mbar_arrive_expect_tx(q_ready, NH * 128);
-    tma_load_2d(qrope, &tmap_q, 8 * 64, q * NH, q_ready);
+    tma_load_2d(qrope, &maps.q[layer], 8 * 64, q * NH, q_ready);
   }
   // the selected indices (and the error word) come from the kernel before
   pdl_wait();
@@ -273,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int sx = sv[k];
-      const int32_t* tab = win[k] ? a.win_page_table : a.page_table;
+      const int32_t* tab = win[k] ? a.win_page_table : a.page_table[layer];
       const int mp = win[k] ? a.win_max_pages : a.max_pages;
       const bool ok = sx >= 0 && sx < (win[k] ? wvis : vis) && (sx >> a.page_shift) < mp;
       pg[k] = ok ? tab[static_cast<size_t>(b) * mp + (sx >> a.page_shift)] : -1;
@@ -298,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // of row r lands at r*128 + ((u ^ (r & 7)) * 16)
     const int pw = warp == 0 ? 0 : warp - (1 + SMX_WARPS);
     const int pu = lane & 7;
-    const uint8_t* pool = reinterpret_cast<const uint8_t*>(a.pool);
+    const uint8_t* pool = reinterpret_cast<const uint8_t*>(a.pool[layer]);
     bool ok = true;
     for (int k = 0; k < ntiles && ok; ++k) {
       const int s = k % NST;
@@ -332,8 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         fence_proxy_async_smem();      // generic-proxy stores, read by the tensor core
         mbar_arrive(&full[s]);
-        continue;
-      }
+      } else {
 #pragma unroll
       for (int i = 0; i < NR / (4 * PRODUCERS); ++i) {
         const int r = (NR / PRODUCERS) * pw + 4 * i + (lane >> 3);
@@ -350,6 +360,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // arrives once this lane's copies of the tile have landed; the producer
       // never blocks on its own copies
       cp_async_arrive_noinc(&full[s]);
+      }
     }
     cp_async_wait<0>();                 // nothing in flight when the CTA retires
   } else if (warp == 1) {
@@ -421,7 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (live) {
         // head h's 256 latent query dims of this CTA -> tensor memory (bf16 pairs)
         const uint4* src = reinterpret_cast<const uint4*>(
-            a.q + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
+            a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float w[32];
@@ -623,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // [128 heads x 32 fp32] (its columns [128g, 128g+128) of this CTA's 256)
     // in the 128-byte swizzle, then one thread stores them with TMA.  The
     // stage ring and the exchange slots are idle once the last PV is done.
-    float* lrow = a.S == 1 ? a.lse + static_cast<size_t>(q) * NH + h
+    float* lrow = a.S == 1 ? a.lse[layer] + static_cast<size_t>(q) * NH + h
                            : a.l_part + (static_cast<size_t>(q) * a.S + split) * NH + h;
     const int orow0 = (a.S == 1 ? q : q * a.S + split) * NH;
     uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
@@ -646,7 +657,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     named_barrier(2 + g, 128);
     if (gt == 128 * g) {
       for (int c = 0; c < 128 / 32; ++c)
-        tma_store_2d(&tmap_o, box0 + c * OBOX_BYTES, static_cast<int>(rank) * 256 + 128 * g + 32 * c,
+        tma_store_2d(&maps.o[layer], box0 + c * OBOX_BYTES, static_cast<int>(rank) * 256 + 128 * g + 32 * c,
                      orow0);
       bulk_commit_group();
       bulk_wait_all_read();   // the shared-memory boxes may be released; the grid's end publishes O
@@ -667,25 +678,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
-                                 int page_size, const int32_t* page_table, int max_pages,
-                                 const int32_t* q_offsets, const int32_t* q_vis,
-                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
-                                 int S, float* out, float* lse, float* o_part, float* l_part,
-                                 uint32_t* err, cudaStream_t st, bool pdl,
-                                 const int32_t* win_page_table, int win_max_pages,
-                                 const int32_t* win_vis, int window, bool kv8, float kv_scale) {
+cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_pages,
+                                     int page_size, int max_pages, const int32_t* q_offsets,
+                                     const int32_t* q_vis, const int32_t* idx, int B, int Q, int H,
+                                     int topk, float scale, int S, float* o_part, float* l_part,
+                                     uint32_t* err, cudaStream_t st, bool pdl,
+                                     const int32_t* win_page_table, int win_max_pages,
+                                     const int32_t* win_vis, int window, bool kv8, float kv_scale) {
   if (Q <= 0) return cudaSuccess;
   if (H != 128 && H != 64) return cudaErrorInvalidValue;
+  // several layers in one grid only without split-K (the partial buffers hold one layer)
+  if (L < 1 || L > MAX_LAYERS || (L > 1 && S != 1)) return cudaErrorInvalidValue;
   int page_shift = 0;
   while ((1 << page_shift) < page_size) ++page_shift;
   if (page_size <= 0 || (1 << page_shift) != page_size) return cudaErrorInvalidValue;
-  // RoPE query dims: boxes of H heads x 64 bf16 (rows past H in shared memory
-  // are never read into a head's result)
-  CUtensorMap tq;
-  if (!encode_tiled_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, DSA_DIM,
-                       static_cast<uint64_t>(Q) * H, DSA_DIM * 2, 64, static_cast<uint32_t>(H)))
-    return cudaErrorInvalidValue;
+  MlaMaps maps;
+  for (int l = 0; l < L; ++l) {
+    // RoPE query dims: boxes of H heads x 64 bf16 (rows past H in shared
+    // memory are never read into a head's result)
+    if (!encode_tiled_2d(&maps.q[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, layers[l].q, DSA_DIM,
+                         static_cast<uint64_t>(Q) * H, DSA_DIM * 2, 64, static_cast<uint32_t>(H)))
+      return cudaErrorInvalidValue;
+    // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
+    // split partials [Q, S, H, 512]
+    if (!encode_tiled_2d(&maps.o[l], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S == 1 ? layers[l].out : o_part,
+                         DSA_DIM_V, static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4,
+                         32, static_cast<uint32_t>(H)))
+      return cudaErrorInvalidValue;
+  }
+  for (int l = L; l < MAX_LAYERS; ++l) {
+    maps.q[l] = maps.q[0];
+    maps.o[l] = maps.o[0];
+  }
   // one instance per (head count, cache type)
   auto kernel = H == 128 ? (kv8 ? sparse_mla_tc_kernel<128, true> : sparse_mla_tc_kernel<128, false>)
                          : (kv8 ? sparse_mla_tc_kernel<64, true> : sparse_mla_tc_kernel<64, false>);
@@ -695,18 +719,37 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   });
   if (ea != cudaSuccess) return ea;
-  // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
-  // split partials [Q, S, H, 512]
-  CUtensorMap to;
-  if (!encode_tiled_2d(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S == 1 ? out : o_part, DSA_DIM_V,
-                       static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4, 32,
-                       static_cast<uint32_t>(H)))
-    return cudaErrorInvalidValue;
-  MlaTcArgs a{q, pool, page_table, max_pages, num_pages, page_shift, win_page_table, win_max_pages,
-              win_vis, window, q_offsets, q_vis, idx, B, Q, topk, S,
-              scale * kv_scale * 1.4426950408889634f, kv_scale, out, lse, o_part, l_part, err};
+  MlaTcArgs a = {};
+  for (int l = 0; l < MAX_LAYERS; ++l) {
+    const MlaLayerPtrs& y = layers[l < L ? l : 0];
+    a.q[l] = y.q;
+    a.pool[l] = y.pool;
+    a.page_table[l] = y.page_table;
+    a.out[l] = y.out;
+    a.lse[l] = y.lse;
+  }
+  a.L = L;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.page_shift = page_shift;
+  a.win_page_table = win_page_table;
+  a.win_max_pages = win_max_pages;
+  a.win_vis = win_vis;
+  a.window = window;
+  a.q_offsets = q_offsets;
+  a.q_vis = q_vis;
+  a.idx = idx;
+  a.B = B;
+  a.Q = Q;
+  a.topk = topk;
+  a.S = S;
+  a.scale_log2 = scale * kv_scale * 1.4426950408889634f;
+  a.out_scale = kv_scale;
+  a.o_part = o_part;
+  a.l_part = l_part;
+  a.err = err;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * Q * S), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * L * Q * S), 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -715,7 +758,21 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kernel, tq, to, a);
+  return cudaLaunchKernelEx(&cfg, kernel, maps, a);
+}
+
+cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* pool, int num_pages,
+                                 int page_size, const int32_t* page_table, int max_pages,
+                                 const int32_t* q_offsets, const int32_t* q_vis,
+                                 const int32_t* idx, int B, int Q, int H, int topk, float scale,
+                                 int S, float* out, float* lse, float* o_part, float* l_part,
+                                 uint32_t* err, cudaStream_t st, bool pdl,
+                                 const int32_t* win_page_table, int win_max_pages,
+                                 const int32_t* win_vis, int window, bool kv8, float kv_scale) {
+  const MlaLayerPtrs one = {q, pool, page_table, out, lse};
+  return launch_sparse_mla_layers(&one, 1, num_pages, page_size, max_pages, q_offsets, q_vis, idx,
+                                  B, Q, H, topk, scale, S, o_part, l_part, err, st, pdl,
+                                  win_page_table, win_max_pages, win_vis, window, kv8, kv_scale);
 }
 
 }  // namespace dsa
