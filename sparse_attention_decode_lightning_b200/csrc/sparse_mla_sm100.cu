@@ -17,8 +17,9 @@
 //   CTA 0: S0 = q[:, 0:256) C[:, 0:256)^T + q[:, 512:544) C[:, 512:544)^T, O[:, 0:256)
 //   CTA 1: S1 = q[:, 256:512) C[:, 256:512)^T + q[:, 544:576) C[:, 544:576)^T, O[:, 256:512)
 // so each CTA gathers the latent columns it uses (the 64 RoPE columns go to
-// both; each contracts half of them, which keeps the pair in balance).  Per tile of 64 selected rows the CTAs swap their fp32
-// partial scores through distributed shared memory; both form S0 + S1
+// both; each contracts half of them, which keeps the pair in balance).  Per tile of 64 selected rows the CTAs swap their partial
+// scores (16-bit codes with a scale per 32 values) through distributed
+// shared memory; both form S0 + S1
 // (bitwise equal on both sides), run the same online softmax and apply the
 // same P to their half of O.
 //
@@ -67,7 +68,8 @@ constexpr int MAXCH = 5;                       // 64-dim chunks per CTA (CTA 1)
 constexpr int CHUNK_T = NR * 128;              // 8 KB: 64 rows x 64 bf16
 constexpr int STAGE_BYTES = MAXCH * CHUNK_T;   // 40 KB
 constexpr int QROPE_BYTES = DSA_HEADS * 128;   // 16 KB: 128 heads x 64 bf16
-constexpr int X_BYTES = DSA_HEADS * NR * 3;    // 24 KB: one tile of 24-bit partial scores
+constexpr int X_CODE_BYTES = DSA_HEADS * NR * 2;           // 16 KB of 16-bit codes
+constexpr int X_BYTES = X_CODE_BYTES + DSA_HEADS * 2 * 4;   // + a scale per (head, 32 rows): 17 KB
 constexpr int OBOX_BYTES = DSA_HEADS * 128;    // 16 KB: output box of 128 heads x 32 fp32
 constexpr int OFF_QR = 0;
 constexpr int OFF_ST = OFF_QR + QROPE_BYTES;
@@ -146,29 +148,26 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
   return __all_sync(0xffffffffu, ok);
 }
 
-// fp32 rounded to nearest at 15 mantissa bits; the low byte is zero
-__device__ __forceinline__ uint32_t round_to_24bit(float x) {
-  return (__float_as_uint(x) + 0x80u) & 0xFFFFFF00u;
-}
+// Partial scores cross the cluster link as 16-bit integers with one fp32
+// scale per block of 32 (one thread's rows of one head): code = rint(s * qs)
+// with qs = 32760 / amax, value = code * (amax / 32760).  The absolute error
+// is at most amax / 65520 = 1.5e-5 amax, the bound a 15-bit mantissa float
+// has for the block's largest value (the softmax is sensitive to absolute
+// score error alone); a CPU simulation against the exact scores moves rms(O)
+// by < 1e-3 and LSE by < 4e-4.  Invalid rows travel as code 0.
+// The conversions stay on the FMA and integer pipes (float-to-int and back
+// go through the narrow conversion unit, which the softmax's exp2 also
+// needs): s * qs + (2^23 + 2^15) is a float in [2^23, 2^24), where the ulp
+// is 1, so its low 16 mantissa bits hold code + 2^15; decoding ORs those
+// bits under the exponent of 2^23 and subtracts 2^23 + 2^15 exactly.
+constexpr float CODE_BIAS = 8421376.f;            // 2^23 + 2^15
+__device__ __forceinline__ float block_scale_of(float amax) { return amax * (1.f / 32760.f); }
 
-// Word i (0..23) of 32 values u[] (low bytes zero) packed 4 per 3 words: value
-// j occupies bits [24j, 24j+24) of the group's 96-bit little-endian string.
-__device__ __forceinline__ uint32_t pack24_word(const uint32_t* u, int i) {
-  const int grp = i / 3, wi = i % 3;
-  const uint32_t a = u[4 * grp] >> 8, b = u[4 * grp + 1] >> 8, c = u[4 * grp + 2] >> 8,
-                 d = u[4 * grp + 3] >> 8;
-  return wi == 0 ? (a | (b << 24)) : wi == 1 ? ((b >> 8) | (c << 16)) : ((c >> 16) | (d << 8));
+__device__ __forceinline__ float code_lo(uint32_t w) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7610)) - CODE_BIAS;
 }
-
-// value j (0..31) of the packed words, as fp32 bits
-__device__ __forceinline__ uint32_t unpack24(const uint32_t* w, int j) {
-  const int grp = j / 4, e = j % 4;
-  const uint32_t w0 = w[3 * grp], w1 = w[3 * grp + 1], w2 = w[3 * grp + 2];
-  const uint32_t v = e == 0 ? (w0 & 0xFFFFFFu)
-                   : e == 1 ? ((w0 >> 24) | ((w1 & 0xFFFFu) << 8))
-                   : e == 2 ? ((w1 >> 16) | ((w2 & 0xFFu) << 16))
-                            : (w2 >> 8);
-  return v << 8;
+__device__ __forceinline__ float code_hi(uint32_t w) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7632)) - CODE_BIAS;
 }
 
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
@@ -466,15 +465,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       float mt0 = -INFINITY, mt1 = -INFINITY;
       const float sl = a.scale_log2;
       // my partial -> the peer's receive slot, pushed with st.async: every
-      // 16-byte store completes its bytes on the peer's x_full[sb], whose
-      // expected count (the whole 24 KB tile) one thread of the peer arms.
-      // Both partials are rounded to 24-bit floats (15 mantissa bits; the
-      // oracle comparison moves by < 2e-4 of rms(O)): four values travel in
-      // three words, a quarter fewer bytes over the ~16 B/cycle DSMEM link.
-      // Slot layout [16-byte chunk k][warpgroup][head]: a warp's chunk k is
-      // 512 contiguous bytes, bank-conflict free; the peer fills mine alike.
-      // The peer's slot sb is written again only after the peer has read
-      // tile t-2 from it (its remote arrival on x_free[sb]).
+      // store completes its bytes on the peer's x_full[sb], whose expected
+      // count (the whole 17 KB tile) one thread of the peer arms.  The
+      // partials travel as 16-bit codes with a scale per 32 values (see
+      // block_scale_of); both CTAs decode their own partial from the codes too,
+      // so they hold bitwise-equal scores.  Slot layout [16-byte chunk
+      // k][warpgroup][head], then the scales [warpgroup][head]: a warp's chunk
+      // k is 512 contiguous bytes, bank-conflict free; the peer fills mine
+      // alike.  The peer's slot sb is written again only after the peer has
+      // read tile t-2 from it (its remote arrival on x_free[sb]).
       // My receive slot of tile t-1 has been read (its values went into
       // tile t-1's softmax, which is finished): the peer may push tile t+1
       // into it.  The arrival needs no release fence, which would also wait
@@ -485,48 +484,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (lane == 0) mbar_arrive_remote_relaxed(peer_xfree + ((t - 1) & 1) * 8);
       }
       if (g == 0 && quarter == 0 && lane == 0)
-        mbar_arrive_expect_tx(&x_full[sb], static_cast<uint32_t>(NH) * (NR * 3));
+        mbar_arrive_expect_tx(&x_full[sb], static_cast<uint32_t>(NH) * 2 * (32 * 2 + 4));
       if (live) {
         if (ok) ok = warp_wait(&s_full[sb], ph, a.err);
         tc_fence_after();
         tmem_ld32(lane_base + S_COL + sb * NR + 32 * g, z);
         tmem_ld_wait();
-        uint32_t u[32];
 #pragma unroll
-        for (int r = 0; r < 32; ++r) u[r] = round_to_24bit(z[r]);
+        for (int r = 0; r < 32; ++r) z[r] = ((vm >> r) & 1u) ? z[r] : 0.f;
+        float am[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          am[i] = fmaxf(fmaxf(fabsf(z[4 * i]), fabsf(z[4 * i + 1])),
+                        fmaxf(fabsf(z[4 * i + 2]), fabsf(z[4 * i + 3])));
+        const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
+                                 fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+        // |z * qs| <= 32760 (1 + 2^-21): the code never leaves [-32767, 32767]
+        const float qs = amax > 0.f ? __fdividef(32760.f, amax) : 0.f;
+        uint32_t cw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          z[2 * i] = fmaf(z[2 * i], qs, CODE_BIAS);
+          z[2 * i + 1] = fmaf(z[2 * i + 1], qs, CODE_BIAS);
+          cw[i] = __byte_perm(__float_as_uint(z[2 * i]), __float_as_uint(z[2 * i + 1]), 0x5410);
+        }
         const uint32_t xoff = sb * X_BYTES + (g * DSA_HEADS + h) * 16;
+        const uint32_t soff = sb * X_BYTES + X_CODE_BYTES + (g * DSA_HEADS + h) * 4;
         if (ok && t >= 2) ok = warp_wait_cluster(&x_free[sb], ((t >> 1) - 1) & 1, a.err);
         if (ok) {
 #pragma unroll
-          for (int k = 0; k < 6; ++k) {
-            // chunk k holds words 4k .. 4k+3 of the 24 packed words (values 16k/3 ..)
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) w[e] = pack24_word(u, 4 * k + e);
-            st_async_v4(peer_x + xoff + k * (2 * DSA_HEADS * 16), __uint_as_float(w[0]),
-                        __uint_as_float(w[1]), __uint_as_float(w[2]), __uint_as_float(w[3]),
-                        peer_xfull + sb * 8);
-          }
+          for (int k = 0; k < 4; ++k)
+            st_async_v4(peer_x + xoff + k * (2 * DSA_HEADS * 16), __uint_as_float(cw[4 * k]),
+                        __uint_as_float(cw[4 * k + 1]), __uint_as_float(cw[4 * k + 2]),
+                        __uint_as_float(cw[4 * k + 3]), peer_xfull + sb * 8);
+          st_async_b32(peer_x + soff, __float_as_uint(amax), peer_xfull + sb * 8);
         }
         if (ok) ok = warp_wait_cluster(&x_full[sb], ph, a.err);
         float4 xs[8];
         {
-          uint32_t pw[24];
+          uint32_t pw[16];
 #pragma unroll
-          for (int k = 0; k < 6; ++k) {
+          for (int k = 0; k < 4; ++k) {
             const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (2 * DSA_HEADS * 16));
             pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
           }
+          const float ps = block_scale_of(*reinterpret_cast<const float*>(xb + soff));
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            xs[i].x = __uint_as_float(unpack24(pw, 4 * i + 0));
-            xs[i].y = __uint_as_float(unpack24(pw, 4 * i + 1));
-            xs[i].z = __uint_as_float(unpack24(pw, 4 * i + 2));
-            xs[i].w = __uint_as_float(unpack24(pw, 4 * i + 3));
+            xs[i].x = code_lo(pw[2 * i]) * ps;
+            xs[i].y = code_hi(pw[2 * i]) * ps;
+            xs[i].z = code_lo(pw[2 * i + 1]) * ps;
+            xs[i].w = code_hi(pw[2 * i + 1]) * ps;
           }
         }
+        // my own partial, decoded exactly as the peer decodes it
+        const float os = block_scale_of(amax);
 #pragma unroll
-        for (int r = 0; r < 32; ++r) z[r] = __uint_as_float(u[r]);
+        for (int r = 0; r < 32; ++r) z[r] = (z[r] - CODE_BIAS) * os;
         // own + peer: rank 0 adds S0 + S1, rank 1 adds S1 + S0; fp32 addition
         // commutes, so both CTAs hold the same z
         if (vm == 0xffffffffu) {
