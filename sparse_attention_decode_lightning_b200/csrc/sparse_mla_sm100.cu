@@ -490,8 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_after();
         tmem_ld32(lane_base + S_COL + sb * NR + 32 * g, z);
         tmem_ld_wait();
-#pragma unroll
-        for (int r = 0; r < 32; ++r) z[r] = ((vm >> r) & 1u) ? z[r] : 0.f;
+        // rows that select nothing were gathered as zeros, so their partial
+        // scores are exactly 0 and leave amax alone
         float am[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -520,51 +520,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           st_async_b32(peer_x + soff, __float_as_uint(amax), peer_xfull + sb * 8);
         }
         if (ok) ok = warp_wait_cluster(&x_full[sb], ph, a.err);
-        float4 xs[8];
-        {
-          uint32_t pw[16];
+        uint32_t pw[16];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (2 * DSA_HEADS * 16));
-            pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
-          }
-          const float ps = block_scale_of(*reinterpret_cast<const float*>(xb + soff));
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            xs[i].x = code_lo(pw[2 * i]) * ps;
-            xs[i].y = code_hi(pw[2 * i]) * ps;
-            xs[i].z = code_lo(pw[2 * i + 1]) * ps;
-            xs[i].w = code_hi(pw[2 * i + 1]) * ps;
-          }
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (2 * DSA_HEADS * 16));
+          pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
         }
-        // my own partial, decoded exactly as the peer decodes it
-        const float os = block_scale_of(amax);
+        // z = (S0 + S1) * sl with S_i = code_i * scale_i: both CTAs evaluate
+        // fma(c0, k0, c1 * k1), c0 and k0 from rank 0's partial, so they hold
+        // bitwise-equal z.  My own codes are still in z as code + CODE_BIAS.
+        const float k_own = block_scale_of(amax) * sl;
+        const float k_peer = block_scale_of(*reinterpret_cast<const float*>(xb + soff)) * sl;
+        if (rank == 0) {
 #pragma unroll
-        for (int r = 0; r < 32; ++r) z[r] = (z[r] - CODE_BIAS) * os;
-        // own + peer: rank 0 adds S0 + S1, rank 1 adds S1 + S0; fp32 addition
-        // commutes, so both CTAs hold the same z
-        if (vm == 0xffffffffu) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            z[4 * i + 0] = (z[4 * i + 0] + xs[i].x) * sl;
-            z[4 * i + 1] = (z[4 * i + 1] + xs[i].y) * sl;
-            z[4 * i + 2] = (z[4 * i + 2] + xs[i].z) * sl;
-            z[4 * i + 3] = (z[4 * i + 3] + xs[i].w) * sl;
-            mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
-            mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+          for (int i = 0; i < 16; ++i) {
+            z[2 * i] = fmaf(z[2 * i] - CODE_BIAS, k_own, code_lo(pw[i]) * k_peer);
+            z[2 * i + 1] = fmaf(z[2 * i + 1] - CODE_BIAS, k_own, code_hi(pw[i]) * k_peer);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float s4[4] = {xs[i].x, xs[i].y, xs[i].z, xs[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = 4 * i + e;
-              z[r] = ((vm >> r) & 1u) ? (z[r] + s4[e]) * sl : -INFINITY;
-            }
-            mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
-            mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
+          for (int i = 0; i < 16; ++i) {
+            z[2 * i] = fmaf(code_lo(pw[i]), k_peer, (z[2 * i] - CODE_BIAS) * k_own);
+            z[2 * i + 1] = fmaf(code_hi(pw[i]), k_peer, (z[2 * i + 1] - CODE_BIAS) * k_own);
           }
+        }
+        if (vm != 0xffffffffu) {
+#pragma unroll
+          for (int r = 0; r < 32; ++r) z[r] = ((vm >> r) & 1u) ? z[r] : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          mt0 = fmaxf(mt0, fmaxf(z[4 * i + 0], z[4 * i + 1]));
+          mt1 = fmaxf(mt1, fmaxf(z[4 * i + 2], z[4 * i + 3]));
         }
       }
       // tile maximum over both warpgroups' rows
