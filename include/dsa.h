@@ -103,7 +103,9 @@ int dsa_version(void);
  * most max_len keys, `topk` selected tokens and `num_splits` split-K parts
  * (0 = let the library choose).  The workspace holds the fp32 score rows
  * [Q, max_len], the split-K partial outputs (sized for 128 heads, so one
- * workspace serves both head counts), the fused selector's per-query
+ * workspace serves both head counts; Q x splits of them plus one per SM pair,
+ * which dsa_decode_step uses to split the last, partial wave of the grouped
+ * IndexShare attention), the fused selector's per-query
  * first-digit histograms, counters and threshold-bin candidate lists (which
  * dsa_indexer_topk_fused clears itself) and the device error flag.  The same workspace may be
  * reused by consecutive calls on one stream; it must be zeroed once

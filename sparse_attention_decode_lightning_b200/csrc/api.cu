@@ -13,6 +13,7 @@ namespace dsa {
 namespace {
 
 constexpr int B200_SMS = 148;
+constexpr int TAIL_PARTS = B200_SMS / 2;
 
 // NVTX range over a scope (header-only NVTX v3: no library to link; the
 // ranges cost nothing unless a profiler collects them)
@@ -65,8 +66,11 @@ bool ws_layout(int Q, int max_len, int topk, int num_splits, WsLayout* L) {
   size_t off = 0;
   w.err = off;      off = align_up(off + 256, 256);
   w.scores = off;   off = align_up(off + static_cast<size_t>(Q) * w.ld * 4, 256);
-  w.o_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * DSA_DIM_V * 4, 256);
-  w.l_part = off;   off = align_up(off + static_cast<size_t>(Q) * w.S * DSA_HEADS * 4, 256);
+  // the split partials of Q x S units, plus room for the tail of a grouped
+  // MLA launch (at most one partial per SM pair, see dsa_decode_step)
+  w.parts = static_cast<size_t>(Q) * w.S + TAIL_PARTS;
+  w.o_part = off;   off = align_up(off + w.parts * DSA_HEADS * DSA_DIM_V * 4, 256);
+  w.l_part = off;   off = align_up(off + w.parts * DSA_HEADS * 4, 256);
   // fused indexer -> selector: a 4096-bin histogram and 4 counters per query,
   // and room for the threshold bin's candidates (about 1/16 of a row, at
   // least 4096, at most 65536; a larger bin is re-read from the scores)
@@ -450,8 +454,12 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
     }
     NvtxRange r("dsa_sparse_mla");
     if (L.S == 1) {
-      // the layers that share this index set run as one grid over (layer,
-      // query): no launch waits for the last wave of the layer before it
+      // The layers that share this index set run as one grid over (layer,
+      // query) units, each on an SM pair.  When the units leave a last wave
+      // that fills at most half of the pairs, those tail units run as a
+      // second grid cut into splits (merged by LSE), so the last wave takes
+      // a fraction of a unit's time instead of a whole one.
+      const int pairs = TAIL_PARTS;
       for (int c0 = l0; c0 < l1; c0 += MLA_MAX_LAYERS_PER_LAUNCH) {
         const int n = l1 - c0 < MLA_MAX_LAYERS_PER_LAUNCH ? l1 - c0 : MLA_MAX_LAYERS_PER_LAUNCH;
         MlaLayerPtrs lp[MLA_MAX_LAYERS_PER_LAUNCH];
@@ -459,10 +467,30 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
           lp[i] = {static_cast<const __nv_bfloat16*>(q_layers[c0 + i]),
                    static_cast<const __nv_bfloat16*>(pool_layers[c0 + i]),
                    page_table_layers[c0 + i], out_layers[c0 + i], lse_layers[c0 + i]};
+        const int units = n * Q;
+        const int waves = units / pairs, tail = units % pairs;
+        int tail_s = tail > 0 ? pairs / tail : 1;
+        const int max_s = topk / 64 < DSA_MAX_SPLITS ? topk / 64 : DSA_MAX_SPLITS;
+        if (tail_s > max_s) tail_s = max_s;
+        const bool split_tail = waves >= 1 && tail > 0 && tail_s >= 2;
+        const int head = split_tail ? waves * pairs : units;
+        uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
         if (launch_sparse_mla_layers(lp, n, num_pages, page_size, max_pages, q_offsets, q_vis,
-                                     idx_g, B, Q, heads, topk, scale, 1, nullptr, nullptr,
-                                     ws_ptr<uint32_t>(ws, L.err), st, true) != cudaSuccess)
+                                     idx_g, B, Q, heads, topk, scale, 1, nullptr, nullptr, err, st,
+                                     true, nullptr, 0, nullptr, 0, false, 1.f, 0,
+                                     head) != cudaSuccess)
           return DSA_ERR_CUDA;
+        if (split_tail) {
+          float* o_part = ws_ptr<float>(ws, L.o_part);
+          float* l_part = ws_ptr<float>(ws, L.l_part);
+          if (launch_sparse_mla_layers(lp, n, num_pages, page_size, max_pages, q_offsets, q_vis,
+                                       idx_g, B, Q, heads, topk, scale, tail_s, o_part, l_part,
+                                       err, st, true, nullptr, 0, nullptr, 0, false, 1.f, head,
+                                       tail) != cudaSuccess ||
+              launch_combine_layers(o_part, l_part, tail, tail_s, heads, head, Q, lp, n, st,
+                                    true) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        }
       }
       continue;
     }

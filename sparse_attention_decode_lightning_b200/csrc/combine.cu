@@ -17,22 +17,35 @@ namespace {
 
 constexpr int HEADS_PER_CTA = 8;               // 8 heads x 512 outputs, 16 per thread
 constexpr int CTHREADS = HEADS_PER_CTA * DSA_DIM_V / 16;
+constexpr int MAX_OUT = MLA_MAX_LAYERS_PER_LAUNCH;
 
-__global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __restrict__ o_part,
-                                                               const float* __restrict__ l_part,
-                                                               int S, int H,
-                                                               float* __restrict__ out,
-                                                               float* __restrict__ lse) {
+// Partial row i (of n) belongs to unit gi = g0 + i, i.e. query gi % Q of the
+// output layer gi / Q (a single output: g0 = 0, Q = n).
+struct CombineArgs {
+  const float* o_part;
+  const float* l_part;
+  int S, H, g0, Q;
+  float* out[MAX_OUT];
+  float* lse[MAX_OUT];
+};
+
+__global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const __grid_constant__ CombineArgs a) {
   pdl_trigger();
   pdl_wait();                                   // the partials come from the previous kernel
-  // CTA: query q, heads [h0, h0 + 8), 128-float quarters [k0, k1) of the 512
-  // outputs; thread: head h0 + tid / 32, float4 column tid % 32 of each quarter
+  // CTA: partial unit i, heads [h0, h0 + 8), 128-float quarters [k0, k1) of
+  // the 512 outputs; thread: head h0 + tid / 32, float4 column tid % 32 of
+  // each quarter
+  const int S = a.S, H = a.H;
   const int k0 = blockIdx.y * 4 / gridDim.y, k1 = (blockIdx.y + 1) * 4 / gridDim.y;
-  const int q = blockIdx.x / (H / HEADS_PER_CTA);
+  const int i = blockIdx.x / (H / HEADS_PER_CTA);
   const int h = (blockIdx.x % (H / HEADS_PER_CTA)) * HEADS_PER_CTA + (threadIdx.x >> 5);
   const int c4 = threadIdx.x & 31;              // float4 column within each 128-float quarter
-  const size_t qh = static_cast<size_t>(q) * H + h;
-  const float* lp = l_part + static_cast<size_t>(q) * S * H + h;
+  const int gi = a.g0 + i;
+  const int layer = gi / a.Q;
+  const size_t qh = static_cast<size_t>(gi % a.Q) * H + h;
+  float* const out = a.out[layer];
+  float* const lse = a.lse[layer];
+  const float* lp = a.l_part + static_cast<size_t>(i) * S * H + h;
   float m = -INFINITY;
   for (int c = 0; c < S; ++c) m = fmaxf(m, lp[static_cast<size_t>(c) * H]);
   float4* o = reinterpret_cast<float4*>(out + qh * DSA_DIM_V) + c4;
@@ -54,7 +67,7 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
     const float wc = expf(lc - m);
     tot += wc;
     const float4* v = reinterpret_cast<const float4*>(
-                          o_part + ((static_cast<size_t>(q) * S + c) * H + h) * DSA_DIM_V) + c4;
+                          a.o_part + ((static_cast<size_t>(i) * S + c) * H + h) * DSA_DIM_V) + c4;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (k < k0 || k >= k1) continue;
@@ -75,12 +88,14 @@ __global__ void __launch_bounds__(CTHREADS) lse_combine_kernel(const float* __re
 
 }  // namespace
 
-cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
-                           float* out, float* lse, cudaStream_t st, bool pdl) {
-  if (Q <= 0) return cudaSuccess;
+namespace {
+
+cudaError_t launch_combine_args(const CombineArgs& args, int n, cudaStream_t st, bool pdl) {
+  if (n <= 0) return cudaSuccess;
+  const int H = args.H;
   if (H <= 0 || H % HEADS_PER_CTA) return cudaErrorInvalidValue;
   // cut the 512 outputs into parts until the grid covers twice the SMs
-  const int ctas = Q * (H / HEADS_PER_CTA);
+  const int ctas = n * (H / HEADS_PER_CTA);
   const int sms = device_sm_count();
   const int parts = ctas >= 2 * sms ? 1 : (2 * ctas >= 2 * sms ? 2 : 4);
   cudaLaunchConfig_t cfg = {};
@@ -92,7 +107,44 @@ cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int 
   add_pdl_attr(attr, &na, pdl);
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, lse_combine_kernel, o_part, l_part, S, H, out, lse);
+  return cudaLaunchKernelEx(&cfg, lse_combine_kernel, args);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
+                           float* out, float* lse, cudaStream_t st, bool pdl) {
+  CombineArgs args = {};
+  args.o_part = o_part;
+  args.l_part = l_part;
+  args.S = S;
+  args.H = H;
+  args.g0 = 0;
+  args.Q = Q > 0 ? Q : 1;
+  for (int l = 0; l < MAX_OUT; ++l) {
+    args.out[l] = out;
+    args.lse[l] = lse;
+  }
+  return launch_combine_args(args, Q, st, pdl);
+}
+
+cudaError_t launch_combine_layers(const float* o_part, const float* l_part, int n_units, int S,
+                                  int H, int g0, int Q, const MlaLayerPtrs* layers, int L,
+                                  cudaStream_t st, bool pdl) {
+  if (L < 1 || L > MAX_OUT || Q <= 0 || g0 < 0 || g0 + n_units > L * Q)
+    return cudaErrorInvalidValue;
+  CombineArgs args = {};
+  args.o_part = o_part;
+  args.l_part = l_part;
+  args.S = S;
+  args.H = H;
+  args.g0 = g0;
+  args.Q = Q;
+  for (int l = 0; l < MAX_OUT; ++l) {
+    args.out[l] = layers[l < L ? l : 0].out;
+    args.lse[l] = layers[l < L ? l : 0].lse;
+  }
+  return launch_combine_args(args, n_units, st, pdl);
 }
 
 }  // namespace dsa

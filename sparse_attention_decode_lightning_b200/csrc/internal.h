@@ -18,8 +18,8 @@ namespace dsa {
 struct WsLayout {
   size_t err = 0;      // uint32 error flag (+ padding)
   size_t scores = 0;   // fp32 [Q, ld]
-  size_t o_part = 0;   // fp32 [Q, S, 128, 512]
-  size_t l_part = 0;   // fp32 [Q, S, 128]
+  size_t o_part = 0;   // fp32 [parts, 128, 512]
+  size_t l_part = 0;   // fp32 [parts, 128]
   size_t hist = 0;     // u32 [Q, 4096]: the indexer's first-digit histograms
   size_t ctr = 0;      // u32 [Q, 4]: the histogram selector's counters (follows hist;
                        // both are zeroed together before each indexer launch)
@@ -27,7 +27,8 @@ struct WsLayout {
   size_t total = 0;
   int cand_cap = 0;
   int ld = 0;          // score row stride (elements)
-  int S = 0;           // split-K parts the partial buffers hold
+  int S = 0;           // split-K parts chosen for Q queries
+  size_t parts = 0;    // (unit, split) partials the buffers hold: Q * S + one per SM pair
 };
 
 // 2-D tensor map, 128-byte swizzle, no OOB fill value (zeros)
@@ -100,8 +101,11 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
                                  const int32_t* win_vis = nullptr, int window = 0,
                                  bool kv8 = false, float kv_scale = 1.f);
 
-// Several layers that share one index set (IndexShare) in one grid of
-// (layer, query, split) units; L <= 4, and L > 1 only with S == 1
+// Several layers that share one index set (IndexShare) in one grid: units
+// gi = layer * Q + query for gi in [g0, g0 + n_units) (default: all L * Q),
+// each cut into S splits.  With S == 1 every unit writes its layer's O and
+// LSE; with S > 1 the partials of unit gi, split c go to row
+// ((gi - g0) * S + c) of o_part [n_units, S, H, 512] / l_part [n_units, S, H].
 struct MlaLayerPtrs {
   const __nv_bfloat16* q;
   const __nv_bfloat16* pool;
@@ -117,7 +121,13 @@ cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_
                                      uint32_t* err, cudaStream_t st, bool pdl,
                                      const int32_t* win_page_table = nullptr, int win_max_pages = 0,
                                      const int32_t* win_vis = nullptr, int window = 0,
-                                     bool kv8 = false, float kv_scale = 1.f);
+                                     bool kv8 = false, float kv_scale = 1.f, int g0 = 0,
+                                     int n_units = -1);
+// The split merge for partial rows laid out as above: row i is unit g0 + i,
+// written to its layer's O and LSE
+cudaError_t launch_combine_layers(const float* o_part, const float* l_part, int n_units, int S,
+                                  int H, int g0, int Q, const MlaLayerPtrs* layers, int L,
+                                  cudaStream_t st, bool pdl);
 
 cudaError_t launch_combine(const float* o_part, const float* l_part, int Q, int S, int H,
                            float* out, float* lse, cudaStream_t st, bool pdl);

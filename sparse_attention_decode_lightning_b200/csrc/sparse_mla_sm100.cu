@@ -96,7 +96,8 @@ struct MlaTcArgs {
   const __nv_bfloat16* q[MAX_LAYERS];
   const __nv_bfloat16* pool[MAX_LAYERS];
   const int32_t* page_table[MAX_LAYERS];
-  int L;                                       // layers in this launch (1 with split-K)
+  int L;                                       // layers whose pointers this launch holds
+  int g0;                                      // first (layer, query) unit of this launch
   int max_pages;
   int num_pages;
   int page_shift;                              // log2 of the tokens per cache page
@@ -222,8 +223,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   pdl_trigger();
   const int unit = blockIdx.x >> 1;
-  const int layer = unit / (a.Q * a.S);
-  const int q = (unit % (a.Q * a.S)) / a.S, split = unit % a.S;
+  // (layer, query) unit gi = layer * Q + q, split `split` of it; with split-K
+  // the partials of this launch's units are numbered from g0
+  const int gu = unit / a.S, split = unit % a.S;
+  const int gi = a.g0 + gu;
+  const int layer = gi / a.Q;
+  const int q = gi % a.Q;
   const int b = seq_of_query_warp(a.q_offsets, a.B, q, lane);
   int vis = a.q_vis[q];
   if (vis < 0) vis = 0;
@@ -636,8 +641,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // in the 128-byte swizzle, then one thread stores them with TMA.  The
     // stage ring and the exchange slots are idle once the last PV is done.
     float* lrow = a.S == 1 ? a.lse[layer] + static_cast<size_t>(q) * NH + h
-                           : a.l_part + (static_cast<size_t>(q) * a.S + split) * NH + h;
-    const int orow0 = (a.S == 1 ? q : q * a.S + split) * NH;
+                           : a.l_part + (static_cast<size_t>(gu) * a.S + split) * NH + h;
+    const int orow0 = (a.S == 1 ? q : gu * a.S + split) * NH;
     uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
     for (int c = 0; c < 128 / 32 && live; ++c) {
       float o[32];
@@ -685,11 +690,13 @@ cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_
                                      int topk, float scale, int S, float* o_part, float* l_part,
                                      uint32_t* err, cudaStream_t st, bool pdl,
                                      const int32_t* win_page_table, int win_max_pages,
-                                     const int32_t* win_vis, int window, bool kv8, float kv_scale) {
+                                     const int32_t* win_vis, int window, bool kv8, float kv_scale,
+                                     int g0, int n_units) {
   if (Q <= 0) return cudaSuccess;
   if (H != 128 && H != 64) return cudaErrorInvalidValue;
-  // several layers in one grid only without split-K (the partial buffers hold one layer)
-  if (L < 1 || L > MAX_LAYERS || (L > 1 && S != 1)) return cudaErrorInvalidValue;
+  if (L < 1 || L > MAX_LAYERS || S < 1) return cudaErrorInvalidValue;
+  if (n_units < 0) n_units = L * Q - g0;
+  if (g0 < 0 || n_units <= 0 || g0 + n_units > L * Q) return cudaErrorInvalidValue;
   int page_shift = 0;
   while ((1 << page_shift) < page_size) ++page_shift;
   if (page_size <= 0 || (1 << page_shift) != page_size) return cudaErrorInvalidValue;
@@ -701,10 +708,10 @@ cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_
                          static_cast<uint64_t>(Q) * H, DSA_DIM * 2, 64, static_cast<uint32_t>(H)))
       return cudaErrorInvalidValue;
     // output boxes of H heads x 32 fp32 into O [Q, H, 512] (S = 1) or the
-    // split partials [Q, S, H, 512]
+    // split partials [n_units, S, H, 512]
     if (!encode_tiled_2d(&maps.o[l], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S == 1 ? layers[l].out : o_part,
-                         DSA_DIM_V, static_cast<uint64_t>(Q) * (S == 1 ? 1 : S) * H, DSA_DIM_V * 4,
-                         32, static_cast<uint32_t>(H)))
+                         DSA_DIM_V, static_cast<uint64_t>(S == 1 ? Q : n_units * S) * H,
+                         DSA_DIM_V * 4, 32, static_cast<uint32_t>(H)))
       return cudaErrorInvalidValue;
   }
   for (int l = L; l < MAX_LAYERS; ++l) {
@@ -730,6 +737,7 @@ cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_
     a.lse[l] = y.lse;
   }
   a.L = L;
+  a.g0 = g0;
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.page_shift = page_shift;
@@ -750,7 +758,7 @@ cudaError_t launch_sparse_mla_layers(const MlaLayerPtrs* layers, int L, int num_
   a.l_part = l_part;
   a.err = err;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * L * Q * S), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * n_units * S), 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
@@ -773,7 +781,8 @@ cudaError_t launch_sparse_mla_tc(const __nv_bfloat16* q, const __nv_bfloat16* po
   const MlaLayerPtrs one = {q, pool, page_table, out, lse};
   return launch_sparse_mla_layers(&one, 1, num_pages, page_size, max_pages, q_offsets, q_vis, idx,
                                   B, Q, H, topk, scale, S, o_part, l_part, err, st, pdl,
-                                  win_page_table, win_max_pages, win_vis, window, kv8, kv_scale);
+                                  win_page_table, win_max_pages, win_vis, window, kv8, kv_scale,
+                                  0, Q);
 }
 
 }  // namespace dsa

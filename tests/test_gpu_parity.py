@@ -245,6 +245,27 @@ def test_indexshare_layers_use_the_leader_indices():
         assert torch.equal(out, outs[l]) and torch.equal(lse, lses[l])
 
 
+@pytest.mark.parametrize("B", [20, 25])
+def test_indexshare_tail_split_matches_oracle(B):
+    """Four layers x B queries leave a last wave of at most half the SM pairs,
+    which runs as split units merged by LSE (B = 25: the split tail starts in
+    layer 2 and ends in layer 3)."""
+    inp = make_inputs(get_workload("indexshare4_b64_ctx16k_128k", B=B, L_range=(2500, 6000)),
+                      seed=12, device=DEV)
+    pairs = 74
+    units = inp.n_layers * inp.Q
+    assert units >= pairs and units % pairs <= pairs // 2
+    outs, lses, idx = run_decode_step(inp, num_splits=1)    # one split: the grouped launch
+    host = oracle_inputs(inp)
+    ix = idx.cpu().numpy()
+    for l in range(inp.n_layers):
+        lay = host["layers"][l]
+        for q in range(inp.Q):
+            o_ref, l_ref = oracle_attention_for_idx(lay["pool"], host["page_table"][q], lay["q"][q],
+                                                    ix[0, q], inp.scale)
+            check_attention(outs[l][q].cpu().numpy(), lses[l][q].cpu().numpy(), o_ref, l_ref)
+
+
 def test_device_bounds_are_flagged_not_faulted():
     inp = make_inputs(get_workload("decode_b32_ctx128k", B=2, L=3000), seed=9, device=DEV)
     bad_pt = inp.page_table.clone()
