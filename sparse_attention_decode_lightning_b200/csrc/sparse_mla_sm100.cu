@@ -26,11 +26,13 @@
 // Tensor memory (512 columns): O half [0,256) | S/P slot 0 [256,320) |
 // S/P slot 1 [320,384) | the CTA's 256 latent query dims [384,512) (bf16
 // pairs).  The scores MMA reads those from tensor memory and the RoPE query
-// dims from shared memory; the softmax overwrites a slot's scores with P as bf16
-// hi + lo halves (p ~= hi + lo to ~16 significant bits: a single bf16 P
-// costs ~1% of the output RMS once the running max is stale), which the PV
-// MMA reads from tensor memory against V (MN-major, N = 256) in shared
-// memory.
+// dims from shared memory; the softmax overwrites a slot's scores with P as
+// fp16 (11 significant bits; a single bf16 P cost ~1.6% of the output RMS
+// once the running max is stale, fp16 ~0.3% in a CPU model), which the PV MMA
+// reads from tensor memory against V (MN-major, N = 256) in shared memory.
+// The tile's value dims are bf16 for the scores MMA and are rewritten in
+// place as fp16 (exact in fp16's normal range) by the producer warps between
+// the two MMAs, since both operands of an MMA share one type.
 //
 // Latent rows are gathered through the page table with 16-byte cp.async by
 // four producer warps (4 rows x 128 bytes per warp instruction, written in
@@ -77,7 +79,7 @@ constexpr int OFF_X = OFF_ST + NST * STAGE_BYTES;
 constexpr int OFF_MX = OFF_X + 2 * X_BYTES;    // [2 tiles][2 warpgroups][128 heads] partial maxima
 constexpr int OFF_CRD = OFF_MX + 2 * 2 * DSA_HEADS * 4;
 constexpr int OFF_BAR = OFF_CRD + DSA_MAX_TOPK * 4;
-constexpr int NBAR = 2 * NST + 5 * 2 + 2;
+constexpr int NBAR = 3 * NST + 5 * 2 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "sparse MLA shared memory exceeds the sm_100 limit");
@@ -171,6 +173,17 @@ __device__ __forceinline__ float code_hi(uint32_t w) {
   return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7632)) - CODE_BIAS;
 }
 
+// two fp32 -> fp16 pair (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// two bf16 (low half first) -> two fp16: exact for magnitudes 2^-14 .. 65504
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return f16x2_bits(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
@@ -217,6 +230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* x_free = x_full + 2;         // [2] the peer has read my partial from its slot
   uint64_t* o_final = x_free + 2;        // last PV
   uint64_t* q_ready = o_final + 1;       // query slice in TMEM / shared memory
+  uint64_t* v_ready = q_ready + 1;       // [NST] a stage's value dims are fp16
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,6 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     mbar_init(o_final, 1);
     mbar_init(q_ready, 5);             // 4 query-loading warps + thread 0 with the RoPE bytes
+    for (int i = 0; i < NST; ++i) mbar_init(&v_ready[i], PRODUCERS);   // one per producer warp
     mbar_fence_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, TMEM_COLS);
@@ -315,9 +330,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int pu = lane & 7;
     const uint8_t* pool = reinterpret_cast<const uint8_t*>(a.pool[layer]);
     bool ok = true;
-    for (int k = 0; k < ntiles && ok; ++k) {
+    // Between its scores MMA and its PV MMA, tile t's value dims (this CTA's
+    // 256 latent columns) are rewritten in place as fp16, the type of P; the
+    // producers do it two tiles behind the copies they issue, each for its own
+    // rows.  bf16 -> fp16 is exact for magnitudes 2^-14 .. 65504; smaller
+    // values keep fp16's subnormal spacing 2^-24.
+    // gather tile k into its stage (after that stage's last PV)
+    auto gather = [&](int k) -> bool {
       const int s = k % NST;
-      if (!(ok = warp_wait(&empty[s], ((k / NST) & 1) ^ 1, a.err))) break;
+      if (!warp_wait(&empty[s], ((k / NST) & 1) ^ 1, a.err)) return false;
       uint8_t* stage = st + s * STAGE_BYTES;
       if constexpr (KV8) {
         // e4m3 rows of 576 bytes: a lane loads all its 8-byte pieces (8 dims
@@ -365,13 +386,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // never blocks on its own copies
       cp_async_arrive_noinc(&full[s]);
       }
+      return true;
+    };
+    // tile t's value dims -> fp16, between its scores MMA and its PV
+    auto convert = [&](int t) -> bool {
+        const int s = t % NST;
+        // the scores MMA has read the tile (its copies are complete too)
+        if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, a.err)) return false;
+        if (!warp_wait(&full[s], (t / NST) & 1, a.err)) return false;
+        uint8_t* stage = st + s * STAGE_BYTES;
+#pragma unroll 4
+        for (int i = lane; i < (NR / PRODUCERS) * 4 * 8; i += 32) {
+          // piece i of this producer's rows: chunk i / (rows * 8), row, 16-byte piece
+          const int c = i / ((NR / PRODUCERS) * 8);
+          const int rr = (i / 8) % (NR / PRODUCERS);
+          uint4* pc = reinterpret_cast<uint4*>(stage + c * CHUNK_T +
+                                               ((NR / PRODUCERS) * pw + rr) * 128 + (i % 8) * 16);
+          const uint4 v = *pc;
+          *pc = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                           bf16x2_to_f16x2(v.w));
+        }
+        fence_proxy_async_smem();      // generic-proxy stores, read by the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&v_ready[s]);
+        return true;
+    };
+    // The copies run ahead: the first NST tiles are issued before any
+    // conversion; later, tile k-2 (whose scores MMA is long done) is
+    // converted before tile k waits for its stage.
+    for (int k = 0; k < ntiles + 2 && ok; ++k) {
+      if (k < NST && k < ntiles) ok = gather(k);
+      if (ok && k >= 2) ok = convert(k - 2);
+      if (ok && k >= NST && k < ntiles) ok = gather(k);
     }
     cp_async_wait<0>();                 // nothing in flight when the CTA retires
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_s = umma_idesc(1 /*BF16*/, DSA_HEADS, NR);
-      constexpr uint32_t idesc_pv = umma_idesc(1 /*BF16*/, DSA_HEADS, 256, 0, 1);
+      constexpr uint32_t idesc_pv = umma_idesc(0 /*F16*/, DSA_HEADS, 256, 0, 1);
       bool ok = mbar_wait(q_ready, 0, a.err);
       tc_fence_after();
       const uint32_t qra = smem_u32(qrope);
@@ -402,14 +455,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (u >= 1) {
           const int t = u - 1, pbuf = t & 1, s = t % NST;
           if (!(ok = mbar_wait(&p_full[pbuf], (t >> 1) & 1, a.err))) break;
+          if (!(ok = mbar_wait(&v_ready[s], (t / NST) & 1, a.err))) break;
+          fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t pa = tmem + S_COL + pbuf * NR;   // P_hi cols [0,32), P_lo [32,64)
+          const uint32_t pa = tmem + S_COL + pbuf * NR;   // P (fp16 pairs) in cols [0,32)
           const uint32_t va = smem_u32(st + s * STAGE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 2 * (NR / 16); ++kk) {
-            // k-steps 0..3: P_hi x rows 16kk..; 4..7: P_lo x the same rows
+          for (int kk = 0; kk < NR / 16; ++kk) {
+            // k-step kk: P x rows 16kk .. 16kk+15 of V (fp16, MN-major)
             mma_f16_ts(tmem + O_COL, pa + kk * 8,
-                       umma_desc_sw128_mn(va + (kk & 3) * 2048, CHUNK_T, 1024), idesc_pv,
+                       umma_desc_sw128_mn(va + kk * 2048, CHUNK_T, 1024), idesc_pv,
                        (t > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&slot_free[pbuf]);
@@ -607,19 +662,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tmem_st32(lane_base + O_COL + c * 32, o);
           }
         }
-        // P as bf16 hi (slot columns [16g, 16g+16)) + lo ([32+16g, 32+16g+16)),
-        // two rows per column
-        float hi[16], lo[16];
+        // P as fp16 (slot columns [16g, 16g+16)), two rows per column; P
+        // <= 2^8 under the lazy maximum, inside fp16's range, with 11
+        // significant bits (a single bf16 P cost ~1.6% of rms(O), fp16 ~0.3%)
+        float pk[16];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const __nv_bfloat162 hv = __floats2bfloat162_rn(z[2 * jj], z[2 * jj + 1]);
-          const float2 hf = __bfloat1622float2(hv);
-          const __nv_bfloat162 lv = __floats2bfloat162_rn(z[2 * jj] - hf.x, z[2 * jj + 1] - hf.y);
-          hi[jj] = __uint_as_float(bf16x2_bits(hv));
-          lo[jj] = __uint_as_float(bf16x2_bits(lv));
-        }
-        tmem_st16(lane_base + S_COL + sb * NR + 16 * g, hi);
-        tmem_st16(lane_base + S_COL + sb * NR + 32 + 16 * g, lo);
+        for (int jj = 0; jj < 16; ++jj)
+          pk[jj] = __uint_as_float(f16x2_bits(z[2 * jj], z[2 * jj + 1]));
+        tmem_st16(lane_base + S_COL + sb * NR + 16 * g, pk);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -644,30 +694,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                            : a.l_part + (static_cast<size_t>(gu) * a.S + split) * NH + h;
     const int orow0 = (a.S == 1 ? q : gu * a.S + split) * NH;
     uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
-    for (int c = 0; c < 128 / 32 && live; ++c) {
-      float o[32];
-      if (have) {
-        tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
-        tmem_ld_wait();
-      }
-      uint8_t* row = box0 + c * OBOX_BYTES + h * 128;
+    // box by box: the TMA store of box c reads shared memory while box c+1
+    // is filled
+    for (int c = 0; c < 128 / 32; ++c) {
+      if (live) {
+        float o[32];
+        if (have) {
+          tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
+          tmem_ld_wait();
+        }
+        uint8_t* row = box0 + c * OBOX_BYTES + h * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 w = have && lt > 0.f ? make_float4(o[4 * j] * inv, o[4 * j + 1] * inv,
-                                                        o[4 * j + 2] * inv, o[4 * j + 3] * inv)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(row + ((j ^ (h & 7)) << 4)) = w;
+        for (int j = 0; j < 8; ++j) {
+          const float4 w = have && lt > 0.f ? make_float4(o[4 * j] * inv, o[4 * j + 1] * inv,
+                                                          o[4 * j + 2] * inv, o[4 * j + 3] * inv)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(row + ((j ^ (h & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier(2 + g, 128);
+      if (gt == 128 * g) {
+        tma_store_2d(&maps.o[layer], box0 + c * OBOX_BYTES,
+                     static_cast<int>(rank) * 256 + 128 * g + 32 * c, orow0);
+        bulk_commit_group();
       }
     }
-    fence_proxy_async_smem();
-    named_barrier(2 + g, 128);
-    if (gt == 128 * g) {
-      for (int c = 0; c < 128 / 32; ++c)
-        tma_store_2d(&maps.o[layer], box0 + c * OBOX_BYTES, static_cast<int>(rank) * 256 + 128 * g + 32 * c,
-                     orow0);
-      bulk_commit_group();
-      bulk_wait_all_read();   // the shared-memory boxes may be released; the grid's end publishes O
-    }
+    // the shared-memory boxes may be released; the grid's end publishes O
+    if (gt == 128 * g) bulk_wait_all_read();
     if (rank == 0 && g == 0 && live)
       *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
     (void)gt;

@@ -41,8 +41,10 @@ def _same(a_outs, a_lses, a_idx, b_outs, b_lses, b_idx):
     for o1, l1, o2, l2 in zip(a_outs, a_lses, b_outs, b_lses):
         r = o1.square().mean().sqrt()
         # same rows, another order: the tiles, running maxima and split parts
-        # regroup the fp32 sums (observed ~5e-5 of rms; parity's bar is 1e-2)
-        assert (o1 - o2).abs().max() <= 1e-3 * r
+        # regroup the fp32 sums, and P is rounded to fp16 relative to a running
+        # maximum that moves at other tiles (observed ~3.4e-3 of rms); the
+        # bound is parity's bar against the oracle, 1e-2 of rms
+        assert (o1 - o2).abs().max() <= 1e-2 * r
         assert (l1 - l2).abs().max() <= 1e-4
 
 
