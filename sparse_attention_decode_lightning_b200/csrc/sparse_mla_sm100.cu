@@ -7,10 +7,10 @@
 //   LSE[h] = ln sum_j exp(z_j).
 //
 // H = 128 or 64 heads.  The MMAs always have M = 128 (the tensor core's full
-// rate shape); with H = 64 the upper 64 TMEM lanes carry no head, and the
-// warps that own them (lane quarters 2 and 3) skip the exchange, the
-// softmax and the output, keeping only their barrier arrivals, so the
-// partial-score exchange moves half the bytes.
+// rate shape); with H = 64 the upper 64 TMEM lanes hold the same 64 heads
+// again, and each copy of a head takes half of every tile's rows (see
+// softmax_dup64), so all eight softmax warps work on 16 scores a thread and
+// the partial-score exchange moves about half the bytes.
 //
 // Work unit: (query, split) on a cluster of two CTAs that divide the
 // contraction dims and the output:
@@ -209,6 +209,249 @@ struct MlaMaps {
   CUtensorMap o[MAX_LAYERS];
 };
 
+// Softmax and epilogue for 64 heads (GLM-5.2).  The MMAs keep M = 128, so
+// the query heads are duplicated: TMEM lanes 64..127 hold heads 0..63 again,
+// and the two copies of a head split each tile's rows.  Warp (g, quarter)
+// owns head (quarter & 1) * 32 + lane and the row block blk = 2g +
+// (quarter >> 1) of 16 rows: lanes 0..63 take blocks 0 and 2, lanes 64..127
+// blocks 1 and 3.  Each copy writes P for its own rows and zeros for the
+// rows of the other copy, so O[h] + O[h + 64] is the head's output; the
+// epilogue adds the two through shared memory.  All eight softmax warps work,
+// 16 scores a thread, where the plain layout leaves lanes 64..127 idle.
+constexpr int DUP_HEADS = 64;
+constexpr int DUP_BLOCKS = 4;                                  // 16-row blocks of a tile
+constexpr int DUP_CODE_BYTES = DUP_HEADS * NR * 2;            // 8 KB of codes a tile
+static_assert(DUP_CODE_BYTES + DUP_HEADS * DUP_BLOCKS * 4 <= X_BYTES, "exchange slot");
+
+__device__ __forceinline__ void softmax_dup64(
+    const MlaTcArgs& a, const MlaMaps& maps, uint8_t* smem, uint32_t tmem, int layer, int q,
+    int split, int gu, int ntiles, int nrows, const int* crd, uint8_t* xb, float* mx,
+    uint64_t* s_full, uint64_t* p_full, uint64_t* slot_free, uint64_t* x_full, uint64_t* x_free,
+    uint64_t* o_final, uint64_t* q_ready, int warp, int lane, int tid, uint32_t rank) {
+  constexpr int NH = DUP_HEADS;
+  const int g = (warp - 2) >> 2;
+  const int gt = tid - 64;
+  const int quarter = warp & 3;
+  const int h = (quarter & 1) * 32 + lane;                     // head of this lane
+  const int blk = 2 * g + (quarter >> 1);                      // its 16 rows of a tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  const uint32_t peer = rank ^ 1u;
+  const uint32_t peer_x = map_to_rank(smem_u32(xb), peer);
+  const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
+  const uint32_t peer_xfree = map_to_rank(smem_u32(x_free), peer);
+  if (g == 0) {
+    // head h's 256 latent query dims of this CTA -> both of its TMEM lanes
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float w[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(src + c * 8 + i);
+        w[4 * i + 0] = __uint_as_float(v.x);
+        w[4 * i + 1] = __uint_as_float(v.y);
+        w[4 * i + 2] = __uint_as_float(v.z);
+        w[4 * i + 3] = __uint_as_float(v.w);
+      }
+      tmem_st32(lane_base + Q_COL + c * 32, w);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_ready);
+  }
+  float m_use = -INFINITY, l = 0.f;                            // l: this block's rows only
+  bool ok = true;
+  const float sl = a.scale_log2;
+  const float zeros[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int t = 0; t < ntiles; ++t) {
+    const int sb = t & 1;
+    const uint32_t ph = (t >> 1) & 1;
+    const int j = t * NR + 16 * blk + lane;
+    const uint32_t vm = __ballot_sync(0xffffffffu, lane < 16 && j < nrows && crd[j] >= 0);
+    float z[16];
+    // my receive slot of tile t-1 has been read: the peer may push tile t+1
+    if (t >= 1) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(peer_xfree + ((t - 1) & 1) * 8);
+    }
+    if (g == 0 && quarter == 0 && lane == 0)
+      mbar_arrive_expect_tx(&x_full[sb], static_cast<uint32_t>(NH) * DUP_BLOCKS * (16 * 2 + 4));
+    if (ok) ok = warp_wait(&s_full[sb], ph, a.err);
+    tc_fence_after();
+    tmem_ld16(lane_base + S_COL + sb * NR + 16 * blk, z);
+    tmem_ld_wait();
+    // 16-bit codes with one scale per block (as block_scale_of describes);
+    // rows that select nothing were gathered as zeros
+    float am[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      am[i] = fmaxf(fmaxf(fabsf(z[4 * i]), fabsf(z[4 * i + 1])), fmaxf(fabsf(z[4 * i + 2]), fabsf(z[4 * i + 3])));
+    const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+    const float qs = amax > 0.f ? __fdividef(32760.f, amax) : 0.f;
+    uint32_t cw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      z[2 * i] = fmaf(z[2 * i], qs, CODE_BIAS);
+      z[2 * i + 1] = fmaf(z[2 * i + 1], qs, CODE_BIAS);
+      cw[i] = __byte_perm(__float_as_uint(z[2 * i]), __float_as_uint(z[2 * i + 1]), 0x5410);
+    }
+    // slot layout [16-byte chunk k][block][head], then the scales [block][head]
+    const uint32_t xoff = sb * X_BYTES + (blk * NH + h) * 16;
+    const uint32_t soff = sb * X_BYTES + DUP_CODE_BYTES + (blk * NH + h) * 4;
+    if (ok && t >= 2) ok = warp_wait_cluster(&x_free[sb], ((t >> 1) - 1) & 1, a.err);
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        st_async_v4(peer_x + xoff + k * (DUP_BLOCKS * NH * 16), __uint_as_float(cw[4 * k]),
+                    __uint_as_float(cw[4 * k + 1]), __uint_as_float(cw[4 * k + 2]),
+                    __uint_as_float(cw[4 * k + 3]), peer_xfull + sb * 8);
+      st_async_b32(peer_x + soff, __float_as_uint(amax), peer_xfull + sb * 8);
+    }
+    if (ok) ok = warp_wait_cluster(&x_full[sb], ph, a.err);
+    uint32_t pw[8];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xb + xoff + k * (DUP_BLOCKS * NH * 16));
+      pw[4 * k] = v.x; pw[4 * k + 1] = v.y; pw[4 * k + 2] = v.z; pw[4 * k + 3] = v.w;
+    }
+    // z = (S0 + S1) * sl, evaluated alike on both CTAs (c0, k0 from rank 0)
+    const float k_own = block_scale_of(amax) * sl;
+    const float k_peer = block_scale_of(*reinterpret_cast<const float*>(xb + soff)) * sl;
+    if (rank == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        z[2 * i] = fmaf(z[2 * i] - CODE_BIAS, k_own, code_lo(pw[i]) * k_peer);
+        z[2 * i + 1] = fmaf(z[2 * i + 1] - CODE_BIAS, k_own, code_hi(pw[i]) * k_peer);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        z[2 * i] = fmaf(code_lo(pw[i]), k_peer, (z[2 * i] - CODE_BIAS) * k_own);
+        z[2 * i + 1] = fmaf(code_hi(pw[i]), k_peer, (z[2 * i + 1] - CODE_BIAS) * k_own);
+      }
+    }
+    if (vm != 0xFFFFu) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) z[r] = ((vm >> r) & 1u) ? z[r] : -INFINITY;
+    }
+    float m4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m4[i] = fmaxf(fmaxf(z[4 * i], z[4 * i + 1]), fmaxf(z[4 * i + 2], z[4 * i + 3]));
+    // tile maximum of head h over the four blocks (both copies of the head)
+    float* mxt = mx + (t & 1) * DUP_BLOCKS * NH;
+    mxt[blk * NH + h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    named_barrier(1, 32 * SMX_WARPS);
+    const float mtile = fmaxf(fmaxf(mxt[h], mxt[NH + h]), fmaxf(mxt[2 * NH + h], mxt[3 * NH + h]));
+    // running max, moved only when it grows by more than 8; identical in
+    // every warp holding head h and in both CTAs
+    float alpha = 1.f;
+    bool resc = false;
+    if (mtile > m_use + 8.f) {
+      if (m_use != -INFINITY) {
+        alpha = fast_exp2(m_use - mtile);
+        resc = true;
+      }
+      m_use = mtile;
+    }
+    const float m_eff = m_use == -INFINITY ? 0.f : m_use;
+    float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; r += 4) {
+      z[r + 0] = fast_exp2(z[r + 0] - m_eff);
+      z[r + 1] = fast_exp2(z[r + 1] - m_eff);
+      z[r + 2] = fast_exp2(z[r + 2] - m_eff);
+      z[r + 3] = fast_exp2(z[r + 3] - m_eff);
+      ps0 += z[r + 0];
+      ps1 += z[r + 1];
+      ps2 += z[r + 2];
+      ps3 += z[r + 3];
+    }
+    l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
+    // both copies' O lanes are rescaled (by the g == 0 warps, every lane)
+    // after PV(t-1), as in the 128-head layout
+    if (g == 0 && __any_sync(0xffffffffu, resc)) {
+      if (ok && t >= 1) ok = warp_wait(&slot_free[(t - 1) & 1], ((t - 1) >> 1) & 1, a.err);
+      tc_fence_after();
+      for (int c = 0; c < 256 / 32; ++c) {
+        float o[32];
+        tmem_ld32(lane_base + O_COL + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+        tmem_st32(lane_base + O_COL + c * 32, o);
+      }
+    }
+    // P (fp16 pairs) for my 16 rows, zeros for the other copy's block
+    float pk[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) pk[jj] = __uint_as_float(f16x2_bits(z[2 * jj], z[2 * jj + 1]));
+    tmem_st8(lane_base + S_COL + sb * NR + 8 * blk, pk);
+    tmem_st8(lane_base + S_COL + sb * NR + 8 * (blk ^ 1), zeros);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&p_full[sb]);
+  }
+  // ---- epilogue: l over the four blocks; O = (O[h] + O[h + 64]) / l
+  // (group g writes columns [128g, 128g+128) of this CTA's 256); LSE from CTA 0
+  float* lsum = mx;                                            // reuse: [4][64]
+  named_barrier(1, 32 * SMX_WARPS);
+  lsum[blk * NH + h] = l;
+  named_barrier(1, 32 * SMX_WARPS);
+  const float lt = (lsum[h] + lsum[NH + h]) + (lsum[2 * NH + h] + lsum[3 * NH + h]);
+  const bool have = ok && ntiles > 0 && warp_wait(o_final, 0, a.err);
+  if (have) tc_fence_after();
+  const float inv = lt > 0.f ? a.out_scale / lt : 0.f;
+  float* lrow = a.S == 1 ? a.lse[layer] + static_cast<size_t>(q) * NH + h
+                         : a.l_part + (static_cast<size_t>(gu) * a.S + split) * NH + h;
+  const int orow0 = (a.S == 1 ? q : gu * a.S + split) * NH;
+  uint8_t* box0 = smem + OFF_ST + g * 4 * OBOX_BYTES;
+  const bool second = quarter >= 2;                            // lanes 64..127: the copies
+  const int brow = quarter * 32 + lane;                        // this lane's box row
+  for (int c = 0; c < 128 / 32; ++c) {
+    uint8_t* box = box0 + c * OBOX_BYTES;
+    float o[32];
+    if (have) {
+      tmem_ld32(lane_base + O_COL + 128 * g + c * 32, o);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0.f;
+    }
+    // the copies park their raw O in box rows 64..127
+    if (second) {
+#pragma unroll
+      for (int jb = 0; jb < 8; ++jb)
+        *reinterpret_cast<float4*>(box + brow * 128 + ((jb ^ (brow & 7)) << 4)) =
+            make_float4(o[4 * jb], o[4 * jb + 1], o[4 * jb + 2], o[4 * jb + 3]);
+    }
+    named_barrier(2 + g, 128);
+    if (!second) {
+      const int prow = brow + 64;                              // the same head's copy
+#pragma unroll
+      for (int jb = 0; jb < 8; ++jb) {
+        const float4 u = *reinterpret_cast<const float4*>(box + prow * 128 + ((jb ^ (prow & 7)) << 4));
+        const float4 w = have && lt > 0.f
+                             ? make_float4((o[4 * jb] + u.x) * inv, (o[4 * jb + 1] + u.y) * inv,
+                                           (o[4 * jb + 2] + u.z) * inv, (o[4 * jb + 3] + u.w) * inv)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(box + brow * 128 + ((jb ^ (brow & 7)) << 4)) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    named_barrier(2 + g, 128);
+    if (gt == 128 * g) {
+      tma_store_2d(&maps.o[layer], box, static_cast<int>(rank) * 256 + 128 * g + 32 * c, orow0);
+      bulk_commit_group();
+    }
+  }
+  if (gt == 128 * g) bulk_wait_all_read();
+  if (rank == 0 && g == 0 && !second)
+    *lrow = lt > 0.f ? m_use * 0.69314718055994531f + logf(lt) : -INFINITY;
+}
+
 template <int NH, bool KV8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     sparse_mla_tc_kernel(const __grid_constant__ MlaMaps maps, const __grid_constant__ MlaTcArgs a) {
@@ -278,8 +521,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_holder;
   if (tid == 0) {
     tma_prefetch_desc(&maps.q[layer]);
-    mbar_arrive_expect_tx(q_ready, NH * 128);
-    tma_load_2d(qrope, &maps.q[layer], 8 * 64, q * NH, q_ready);
+    if constexpr (NH == 64) {
+      // 64 heads: rows 64..127 repeat rows 0..63 (TMEM lanes 64..127 carry
+      // the same heads; see the softmax)
+      mbar_arrive_expect_tx(q_ready, 2 * NH * 128);
+      tma_load_2d(qrope, &maps.q[layer], 8 * 64, q * NH, q_ready);
+      tma_load_2d(qrope + NH * 128, &maps.q[layer], 8 * 64, q * NH, q_ready);
+    } else {
+      mbar_arrive_expect_tx(q_ready, NH * 128);
+      tma_load_2d(qrope, &maps.q[layer], 8 * 64, q * NH, q_ready);
+    }
   }
   // the selected indices (and the error word) come from the kernel before
   pdl_wait();
@@ -473,6 +724,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
       }
     }
+  } else if constexpr (NH == 64) {
+    softmax_dup64(a, maps, smem, tmem, layer, q, split, gu, ntiles, nrows, crd, xb, mx, s_full,
+                  p_full, slot_free, x_full, x_free, o_final, q_ready, warp, lane, tid, rank);
   } else {
     // ------------------------------------------------------------ softmax
     const int g = (warp - 2) >> 2;                 // warpgroup: tile rows [32g, 32g+32)
