@@ -266,6 +266,32 @@ def test_indexshare_tail_split_matches_oracle(B):
             check_attention(outs[l][q].cpu().numpy(), lses[l][q].cpu().numpy(), o_ref, l_ref)
 
 
+@pytest.mark.parametrize("n_layers,G", [(6, 4), (9, 8)])
+def test_index_groups_of_uneven_and_long_length_match_oracle(n_layers, G):
+    """Six layers in groups of four (a full group, then two layers) and nine
+    in groups of eight (a group longer than one grouped launch of four
+    layers, then one layer alone): every layer attends over its group
+    leader's indices."""
+    inp = make_inputs(get_workload("indexshare4_b64_ctx16k_128k", B=3, L_range=(2500, 5000),
+                                   n_layers=n_layers, index_share=G), seed=17, device=DEV)
+    outs, lses, idx = run_decode_step(inp, num_splits=1)
+    host = oracle_inputs(inp)
+    ix = idx.cpu().numpy()
+    assert ix.shape[0] == (n_layers + G - 1) // G
+    for g in range(ix.shape[0]):
+        ind = host["indexer"][g]
+        for q in range(inp.Q):
+            k0, vis = int(host["seq_offsets"][q]), int(host["q_vis"][q])
+            sc = O.indexer_scores(ind["q_idx"][q], ind["w"][q], ind["k_idx"][k0:k0 + vis])
+            check_topk_row(ix[g, q], sc, inp.topk)
+    for l in range(n_layers):
+        lay = host["layers"][l]
+        for q in range(inp.Q):
+            o_ref, l_ref = oracle_attention_for_idx(lay["pool"], host["page_table"][q], lay["q"][q],
+                                                    ix[l // G, q], inp.scale)
+            check_attention(outs[l][q].cpu().numpy(), lses[l][q].cpu().numpy(), o_ref, l_ref)
+
+
 def test_device_bounds_are_flagged_not_faulted():
     inp = make_inputs(get_workload("decode_b32_ctx128k", B=2, L=3000), seed=9, device=DEV)
     bad_pt = inp.page_table.clone()
