@@ -734,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const bool live = quarter * 32 < NH;         // this warp's lanes carry heads
+    constexpr bool live = true;                  // 128 heads: every lane carries one
     const uint32_t peer = rank ^ 1u;
     const uint32_t peer_x = map_to_rank(smem_u32(xb), peer);
     const uint32_t peer_xfull = map_to_rank(smem_u32(x_full), peer);
