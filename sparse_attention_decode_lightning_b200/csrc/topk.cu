@@ -345,11 +345,31 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   if (cnt0 <= static_cast<uint32_t>(CAND_CAP)) {
     // ---- gather: digit < t0 goes out now, digit == t0 goes to rank 0
     auto gather = [&](auto better, auto in) {
+      // One pass over the slice records which of this thread's elements are
+      // "in" and which of those are "better" as bits of two masks (bit c is
+      // the thread's c-th element in for_slice order, element j(c) below);
+      // the writes then visit only the set bits.  Slices of up to 64
+      // elements a thread; longer ones read the slice a second time.
+      const bool masked = n <= 64 * THREADS;
+      uint64_t m_in = 0, m_better = 0;
       uint32_t nb = 0, ni = 0;
-      for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
-        nb += valid && better(pos, key);
-        ni += valid && in(pos, key);
-      });
+      if (masked) {
+        int c = 0;
+        for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+          if (valid && in(pos, key)) {
+            m_in |= 1ull << c;
+            if (better(pos, key)) m_better |= 1ull << c;
+          }
+          ++c;
+        });
+        nb = static_cast<uint32_t>(__popcll(m_better));
+        ni = static_cast<uint32_t>(__popcll(m_in));
+      } else {
+        for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+          nb += valid && better(pos, key);
+          ni += valid && in(pos, key);
+        });
+      }
       // per CTA nb < topk and ni - nb <= cnt0 <= CAND_CAP: both halves stay below 2^16
       uint32_t tot;
       const uint32_t pre = block_excl_scan((nb << 16) | (ni - nb), s_warp, &tot);
@@ -366,23 +386,35 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
       uint32_t o = s_obase - (rank == 0 ? nb_cta : 0u) + (pre >> 16);
       uint32_t ci = s_cbase + (pre & 0xFFFFu);
       const uint32_t cand0 = map_to_rank(smem_u32(s_cand), 0u);
-      for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
-        if (valid && in(pos, key)) {
-          if (better(pos, key)) {
-            if (o < static_cast<uint32_t>(topk)) {
-              oi[o] = pos;
-              if (os) os[o] = key_float(key);
-            } else {
-              raise_error(a.err, DEVERR_BOUNDS);
-            }
-            ++o;
+      auto emit = [&](int pos, uint32_t key, bool is_better) {
+        if (is_better) {
+          if (o < static_cast<uint32_t>(topk)) {
+            oi[o] = pos;
+            if (os) os[o] = key_float(key);
           } else {
-            if (ci < static_cast<uint32_t>(CAND_CAP)) st_cluster_u64(cand0 + ci * 8u, make_v(pos, key));
-            else raise_error(a.err, DEVERR_BOUNDS);
-            ++ci;
+            raise_error(a.err, DEVERR_BOUNDS);
           }
+          ++o;
+        } else {
+          if (ci < static_cast<uint32_t>(CAND_CAP)) st_cluster_u64(cand0 + ci * 8u, make_v(pos, key));
+          else raise_error(a.err, DEVERR_BOUNDS);
+          ++ci;
         }
-      });
+      };
+      if (masked) {
+        // element c of this thread: j = (c / 4) * 4 * THREADS + 4 * tid + c % 4
+        // (for_slice's order); visited in increasing c, as the first pass saw them
+        for (uint64_t m = m_in; m; m &= m - 1) {
+          const int c = __ffsll(static_cast<long long>(m)) - 1;
+          const int j = (c >> 2) * (4 * THREADS) + 4 * tid + (c & 3);
+          const uint32_t key = j < a.scap ? s_key[j] : float_key(__ldg(grow + j));
+          emit(beg + j, key, (m_better >> c) & 1ull);
+        }
+      } else {
+        for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
+          if (valid && in(pos, key)) emit(pos, key, better(pos, key));
+        });
+      }
     };
     if (fast0) gather(fast_better, fast_in);
     else gather(gen_better, gen_in);
