@@ -53,6 +53,7 @@ constexpr int CAND_CAP = 4096;                // bin-t positions rank 0 gathers
 constexpr int MAX_CLUSTER = 8;                // portable cluster size
 constexpr int MAX_CLUSTER_NP = 16;            // non-portable size for a few long rows
 constexpr int MIN_SLICE = 2048;               // rows are not cut finer than this
+constexpr int RS_MIN_CLUSTER = 8;             // clusters this large merge by parts (see below)
 static_assert(BINS == 4 * THREADS, "bins are merged THREADS at a time, scanned 4 per thread");
 
 constexpr size_t smem_bytes(int scap) {
@@ -177,6 +178,8 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
   __shared__ uint32_t s_t, s_cb, s_cnt;         // threshold digit, count below it, its count
   __shared__ __align__(8) uint64_t s_ctr;      // rank 0: output slots | gathered candidates << 32
   __shared__ uint32_t s_obase, s_cbase;
+  __shared__ uint32_t s_sum[BINS / RS_MIN_CLUSTER];   // this CTA's part of the summed histogram
+  __shared__ uint32_t s_part, s_pidx, s_pbefore;   // its total; the part holding the threshold
 
   const int tid = threadIdx.x;
   const int C = static_cast<int>(gridDim.x);    // cluster = one grid row
@@ -273,6 +276,53 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
 
   // threshold digit of the cluster's summed histograms; h = this pass's buffer
   auto merged_threshold = [&](const uint32_t* h, uint32_t need) {
+    if (C >= RS_MIN_CLUSTER) {
+      // By parts: CTA r sums bins [lo_r, hi_r) over the cluster (BINS remote
+      // loads a CTA, instead of C per bin up to the threshold's chunk), the
+      // part totals locate the part that holds the threshold, and every CTA
+      // scans that part's sums.  One cluster barrier more, 1/C of the
+      // distributed shared memory traffic.
+      const int lo = static_cast<int>(rank) * BINS / C, hi = (static_cast<int>(rank) + 1) * BINS / C;
+      uint32_t m = 0;
+      if (tid < hi - lo) {
+        const uint32_t a0 = smem_u32(h + lo + tid);
+        for (int r = 0; r < C; ++r) m += ld_cluster_u32(map_to_rank(a0, static_cast<uint32_t>(r)));
+        s_sum[tid] = m;
+      }
+      uint32_t tot;
+      block_excl_scan(m, s_warp, &tot);
+      if (tid == 0) s_part = tot;
+      cluster_sync();          // every part summed
+      if (tid < 32) {
+        const uint32_t pt = tid < C ? ld_cluster_u32(map_to_rank(smem_u32(&s_part), static_cast<uint32_t>(tid))) : 0u;
+        uint32_t incl = pt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (tid >= off) incl += y;
+        }
+        const uint32_t before = incl - pt;
+        if (tid < C && before < need && incl >= need) {
+          s_pidx = static_cast<uint32_t>(tid);
+          s_pbefore = before;
+        }
+      }
+      __syncthreads();
+      const int p = static_cast<int>(s_pidx);
+      const int plo = p * BINS / C, phi = (p + 1) * BINS / C;
+      const uint32_t pb = s_pbefore;
+      const uint32_t v = tid < phi - plo
+                             ? ld_cluster_u32(map_to_rank(smem_u32(&s_sum[tid]), static_cast<uint32_t>(p)))
+                             : 0u;
+      const uint32_t ex = pb + block_excl_scan(v, s_warp, &tot);
+      if (tid < phi - plo && ex < need && ex + v >= need) {
+        s_t = static_cast<uint32_t>(plo + tid);
+        s_cb = ex;
+        s_cnt = v;
+      }
+      __syncthreads();
+      return;
+    }
     uint32_t carry = 0;
     for (int c0 = 0; c0 < BINS; c0 += THREADS) {
       const uint32_t a0 = smem_u32(h + c0 + tid);
