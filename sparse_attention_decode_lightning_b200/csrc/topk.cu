@@ -398,22 +398,34 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
       // One pass over the slice records which of this thread's elements are
       // "in" and which of those are "better" as bits of two masks (bit c is
       // the thread's c-th element in for_slice order, element j(c) below);
-      // the writes then visit only the set bits.  Slices of up to 64
-      // elements a thread; longer ones read the slice a second time.
-      const bool masked = n <= 64 * THREADS;
-      uint64_t m_in = 0, m_better = 0;
+      // the writes then visit only the set bits.  Slices of up to
+      // 64 * MASK_WORDS elements a thread; longer ones read the slice twice.
+      constexpr int MASK_WORDS = 2;               // (the adds below name both words)
+      const bool masked = n <= 64 * MASK_WORDS * THREADS;
+      uint64_t m_in[MASK_WORDS] = {}, m_better[MASK_WORDS] = {};
       uint32_t nb = 0, ni = 0;
       if (masked) {
         int c = 0;
         for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
           if (valid && in(pos, key)) {
-            m_in |= 1ull << c;
-            if (better(pos, key)) m_better |= 1ull << c;
+            // words picked by comparison, not by index, to stay in registers
+            const uint64_t bit = 1ull << (c & 63);
+            const bool bt = better(pos, key);
+            if (c < 64) {
+              m_in[0] |= bit;
+              if (bt) m_better[0] |= bit;
+            } else {
+              m_in[1] |= bit;
+              if (bt) m_better[1] |= bit;
+            }
           }
           ++c;
         });
-        nb = static_cast<uint32_t>(__popcll(m_better));
-        ni = static_cast<uint32_t>(__popcll(m_in));
+#pragma unroll
+        for (int w = 0; w < MASK_WORDS; ++w) {
+          nb += static_cast<uint32_t>(__popcll(m_better[w]));
+          ni += static_cast<uint32_t>(__popcll(m_in[w]));
+        }
       } else {
         for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
           nb += valid && better(pos, key);
@@ -454,11 +466,15 @@ __global__ void __launch_bounds__(THREADS, 1) topk_cluster_kernel(TopkArgs a) {
       if (masked) {
         // element c of this thread: j = (c / 4) * 4 * THREADS + 4 * tid + c % 4
         // (for_slice's order); visited in increasing c, as the first pass saw them
-        for (uint64_t m = m_in; m; m &= m - 1) {
-          const int c = __ffsll(static_cast<long long>(m)) - 1;
-          const int j = (c >> 2) * (4 * THREADS) + 4 * tid + (c & 3);
-          const uint32_t key = j < a.scap ? s_key[j] : float_key(__ldg(grow + j));
-          emit(beg + j, key, (m_better >> c) & 1ull);
+#pragma unroll
+        for (int w = 0; w < MASK_WORDS; ++w) {
+          for (uint64_t m = m_in[w]; m; m &= m - 1) {
+            const int b = __ffsll(static_cast<long long>(m)) - 1;
+            const int c = 64 * w + b;
+            const int j = (c >> 2) * (4 * THREADS) + 4 * tid + (c & 3);
+            const uint32_t key = j < a.scap ? s_key[j] : float_key(__ldg(grow + j));
+            emit(beg + j, key, (m_better[w] >> b) & 1ull);
+          }
         }
       } else {
         for_slice(s_key, grow, beg, n, a.scap, [&](int pos, uint32_t key, bool valid) {
