@@ -125,6 +125,18 @@ size_t dsa_workspace_bytes(int Q, int max_len, int topk, int num_splits);
 int dsa_choose_splits(int Q, int topk, int num_splits);
 
 /*
+ * How dsa_decode_step runs the grouped attention of an IndexShare group of
+ * `units` (layer, query) pairs with one split each, every unit on a pair of
+ * SMs: when the units leave a last wave that fills at most half of the GPU's
+ * 74 SM pairs, those tail units run as a second grid cut into *tail_splits
+ * parts (merged by log-sum-exp) and the first *head_units run whole.
+ * Without such a tail: *head_units = units, *tail_units = 0, *tail_splits = 1.
+ * Returns 1, or 0 (outputs untouched) for invalid sizes or null pointers.
+ * Host only; for callers that size or schedule around the step.
+ */
+int dsa_mla_group_plan(int units, int topk, int* head_units, int* tail_units, int* tail_splits);
+
+/*
  * Lightning indexer, scores only  (section 2.2: the indexer stage).
  *   q_idx  e4m3 [Q,idx_heads,128]   w [Q,idx_heads] fp32   k_idx e4m3 [total_keys,128]
  *   idx_heads  64 (DeepSeek-V3.2) or 32 (GLM-5.2)

@@ -37,6 +37,7 @@ SIGNATURES = {
     "dsa_version": (_I, []),
     "dsa_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "dsa_choose_splits": (_I, [_I, _I, _I]),
+    "dsa_mla_group_plan": (_I, [_I, _I, _P, _P, _P]),
     "dsa_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _SZ,
                                 _P]),
     "dsa_topk_select": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -140,6 +141,15 @@ def dsa_status_string(s: int) -> str:
 
 def dsa_choose_splits(Q: int, topk: int, num_splits: int = 0) -> int:
     return lib().dsa_choose_splits(Q, topk, num_splits)
+
+
+def dsa_mla_group_plan(units: int, topk: int):
+    """(head_units, tail_units, tail_splits) of an IndexShare group's grouped
+    attention, or None for invalid sizes."""
+    h, t, ts = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    if not lib().dsa_mla_group_plan(units, topk, ctypes.byref(h), ctypes.byref(t), ctypes.byref(ts)):
+        return None
+    return h.value, t.value, ts.value
 
 
 def dsa_workspace_bytes(Q: int, max_len: int, topk: int, num_splits: int = 0) -> int:

@@ -30,6 +30,22 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+// Grouped IndexShare attention: `units` (layer, query) units of one split on
+// the SM pairs.  When they leave a last wave that fills at most half of the
+// pairs, the units of that wave (tail) run cut into tail_s splits; head units
+// run whole.  Without such a tail: head = units, tail = 0, tail_s = 1.
+void plan_group(int units, int topk, int* head, int* tail, int* tail_s) {
+  const int pairs = TAIL_PARTS;
+  const int waves = units / pairs, rest = units % pairs;
+  int s = rest > 0 ? pairs / rest : 1;
+  const int max_s = topk / 64 < DSA_MAX_SPLITS ? topk / 64 : DSA_MAX_SPLITS;
+  if (s > max_s) s = max_s;
+  const bool split = waves >= 1 && rest > 0 && s >= 2;
+  *head = split ? waves * pairs : units;
+  *tail = split ? rest : 0;
+  *tail_s = split ? s : 1;
+}
+
 int choose_splits(int Q, int topk, int requested) {
   int S = requested;
   if (S <= 0) {
@@ -247,6 +263,13 @@ const char* dsa_status_string(int s) {
 
 int dsa_version(void) { return 300; }
 
+int dsa_mla_group_plan(int units, int topk, int* head_units, int* tail_units, int* tail_splits) {
+  if (units <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || !head_units || !tail_units || !tail_splits)
+    return 0;
+  plan_group(units, topk, head_units, tail_units, tail_splits);
+  return 1;
+}
+
 int dsa_choose_splits(int Q, int topk, int num_splits) {
   if (Q <= 0 || topk <= 0 || topk > DSA_MAX_TOPK || num_splits < 0 || num_splits > DSA_MAX_SPLITS)
     return 0;
@@ -459,7 +482,6 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
       // that fills at most half of the pairs, those tail units run as a
       // second grid cut into splits (merged by LSE), so the last wave takes
       // a fraction of a unit's time instead of a whole one.
-      const int pairs = TAIL_PARTS;
       for (int c0 = l0; c0 < l1; c0 += MLA_MAX_LAYERS_PER_LAUNCH) {
         const int n = l1 - c0 < MLA_MAX_LAYERS_PER_LAUNCH ? l1 - c0 : MLA_MAX_LAYERS_PER_LAUNCH;
         MlaLayerPtrs lp[MLA_MAX_LAYERS_PER_LAUNCH];
@@ -467,13 +489,9 @@ dsa_status dsa_decode_step(int n_layers, int index_share, int mtp_index_share,
           lp[i] = {static_cast<const __nv_bfloat16*>(q_layers[c0 + i]),
                    static_cast<const __nv_bfloat16*>(pool_layers[c0 + i]),
                    page_table_layers[c0 + i], out_layers[c0 + i], lse_layers[c0 + i]};
-        const int units = n * Q;
-        const int waves = units / pairs, tail = units % pairs;
-        int tail_s = tail > 0 ? pairs / tail : 1;
-        const int max_s = topk / 64 < DSA_MAX_SPLITS ? topk / 64 : DSA_MAX_SPLITS;
-        if (tail_s > max_s) tail_s = max_s;
-        const bool split_tail = waves >= 1 && tail > 0 && tail_s >= 2;
-        const int head = split_tail ? waves * pairs : units;
+        int head = 0, tail = 0, tail_s = 1;
+        plan_group(n * Q, topk, &head, &tail, &tail_s);
+        const bool split_tail = tail > 0;
         uint32_t* err = ws_ptr<uint32_t>(ws, L.err);
         if (launch_sparse_mla_layers(lp, n, num_pages, page_size, max_pages, q_offsets, q_vis,
                                      idx_g, B, Q, heads, topk, scale, 1, nullptr, nullptr, err, st,

@@ -58,6 +58,30 @@ def test_split_choice():
         assert 1 <= s <= 16 and 2048 // s >= 64
 
 
+def test_mla_group_plan():
+    plan = dsa.dsa_mla_group_plan
+    assert plan(0, 2048) is None and plan(10, 0) is None and plan(10, 4096) is None
+    # fewer units than SM pairs: one wave, nothing split
+    assert plan(64, 2048) == (64, 0, 1)
+    assert plan(74, 2048) == (74, 0, 1)
+    # IndexShare, 4 layers x 64 queries: three full waves, the last 34 units in 2 splits
+    assert plan(256, 2048) == (222, 34, 2)
+    assert plan(80, 2048) == (74, 6, 12)
+    assert plan(100, 2048) == (74, 26, 2)
+    assert plan(111, 2048) == (74, 37, 2)
+    # a last wave more than half full runs whole
+    assert plan(112, 2048) == (112, 0, 1)
+    assert plan(128, 2048) == (128, 0, 1)
+    # splits capped at DSA_MAX_SPLITS (32) and at one split per 64 selected tokens
+    assert plan(150, 2048) == (148, 2, 32)
+    assert plan(150, 256) == (148, 2, 4)
+    assert plan(75, 64) == (75, 0, 1)
+    for units in range(1, 600):
+        head, tail, ts = plan(units, 2048)
+        assert head + tail == units and head % 74 == 0 or tail == 0
+        assert tail * ts <= 74
+
+
 def test_workspace_bytes_arithmetic():
     f = dsa.dsa_workspace_bytes
     assert f(0, 10, 2048, 0) == 0
