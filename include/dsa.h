@@ -274,10 +274,15 @@ dsa_status dsa_sparse_mla_decode_window(const void* q, const void* kv_pool, int 
  *             row is the code's value times kv_scale (one scale for the
  *             whole cache, > 0)
  * Everything else as in dsa_sparse_mla_decode.  The gather widens each e4m3
- * row exactly to bf16 on chip (every e4m3 value is a bf16 value) for the
- * same bf16 tensor-core products; kv_scale multiplies the scores (with
- * `scale`) and the output, so nothing is rounded that the bf16 call would
- * not round.  A row is 576 bytes instead of 1152.
+ * row exactly on chip (every e4m3 value is an fp16 and a bf16 value): the 512
+ * latent dims to fp16, the 64 RoPE dims to bf16.  The tensor-core products of
+ * the latent dims then take the query's latent dims as fp16, which is exact
+ * for every element that is zero or of magnitude 2^-14 .. 65504; smaller ones
+ * round to fp16's subnormal spacing 2^-24.  A query element of magnitude
+ * 65536 or more (beyond fp16) is flagged as DSA_ERR_DEVICE_BOUNDS through the
+ * workspace's error word, and that call's output is not valid.  kv_scale
+ * multiplies the scores (with `scale`) and the output.  A row is 576 bytes
+ * instead of 1152.
  */
 dsa_status dsa_sparse_mla_decode_fp8(const void* q, const void* kv_pool, float kv_scale,
                                      int num_pages, int page_size, const int32_t* page_table,

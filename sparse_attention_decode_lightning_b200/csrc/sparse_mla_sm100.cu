@@ -203,6 +203,57 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
                     e4m3x2_to_bf16x2(v.y & 0xFFFFu), e4m3x2_to_bf16x2(v.y >> 16));
 }
 
+// two e4m3 codes -> two fp16, exactly (one cvt: an e4m3 value is an fp16
+// value, its smallest subnormal 2^-9 above fp16's normal minimum)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3);
+  return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint2 v) {
+  return make_uint4(e4m3x2_to_f16x2(v.x & 0xFFFFu), e4m3x2_to_f16x2(v.x >> 16),
+                    e4m3x2_to_f16x2(v.y & 0xFFFFu), e4m3x2_to_f16x2(v.y >> 16));
+}
+
+// a bf16 pair with a finite element of magnitude >= 65536, which fp16 cannot hold
+// (no bf16 value lies between fp16's maximum 65504 and 65536)
+__device__ __forceinline__ bool bf16x2_beyond_f16(uint32_t w) {
+  const uint32_t lo = w & 0x7FFFu, hi = (w >> 16) & 0x7FFFu;
+  return (lo >= 0x4780u && lo < 0x7F80u) || (hi >= 0x4780u && hi < 0x7F80u);
+}
+
+// head h's 256 latent query dims of this CTA -> its TMEM lane at columns
+// [Q_COL, Q_COL + 128): bf16 pairs as given, or (FP8 cache) fp16 pairs, since
+// both operands of the scores MMA take one type.  bf16 -> fp16 is exact for
+// magnitudes 2^-14 .. 65504; below, fp16's subnormal spacing 2^-24 rounds; an
+// element beyond fp16's range is flagged as out of range.
+template <bool F16>
+__device__ __forceinline__ void load_query_tmem(const __nv_bfloat16* qh, uint32_t lane_addr,
+                                                uint32_t* err) {
+  const uint4* src = reinterpret_cast<const uint4*>(qh);
+  bool bad = false;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float w[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint4 v = __ldg(src + c * 8 + i);
+      if constexpr (F16) {
+        bad |= bf16x2_beyond_f16(v.x) | bf16x2_beyond_f16(v.y) | bf16x2_beyond_f16(v.z) |
+               bf16x2_beyond_f16(v.w);
+        v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                       bf16x2_to_f16x2(v.w));
+      }
+      w[4 * i + 0] = __uint_as_float(v.x);
+      w[4 * i + 1] = __uint_as_float(v.y);
+      w[4 * i + 2] = __uint_as_float(v.z);
+      w[4 * i + 3] = __uint_as_float(v.w);
+    }
+    tmem_st32(lane_addr + Q_COL + c * 32, w);
+  }
+  if (F16 && bad) raise_error(err, DEVERR_BOUNDS);
+}
+
 // the per-layer tensor maps: RoPE query dims, and the output
 struct MlaMaps {
   CUtensorMap q[MAX_LAYERS];
@@ -223,6 +274,7 @@ constexpr int DUP_BLOCKS = 4;                                  // 16-row blocks 
 constexpr int DUP_CODE_BYTES = DUP_HEADS * NR * 2;            // 8 KB of codes a tile
 static_assert(DUP_CODE_BYTES + DUP_HEADS * DUP_BLOCKS * 4 <= X_BYTES, "exchange slot");
 
+template <bool KV8>
 __device__ __forceinline__ void softmax_dup64(
     const MlaTcArgs& a, const MlaMaps& maps, uint8_t* smem, uint32_t tmem, int layer, int q,
     int split, int gu, int ntiles, int nrows, const int* crd, uint8_t* xb, float* mx,
@@ -241,21 +293,8 @@ __device__ __forceinline__ void softmax_dup64(
   const uint32_t peer_xfree = map_to_rank(smem_u32(x_free), peer);
   if (g == 0) {
     // head h's 256 latent query dims of this CTA -> both of its TMEM lanes
-    const uint4* src = reinterpret_cast<const uint4*>(
-        a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float w[32];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 v = __ldg(src + c * 8 + i);
-        w[4 * i + 0] = __uint_as_float(v.x);
-        w[4 * i + 1] = __uint_as_float(v.y);
-        w[4 * i + 2] = __uint_as_float(v.z);
-        w[4 * i + 3] = __uint_as_float(v.w);
-      }
-      tmem_st32(lane_base + Q_COL + c * 32, w);
-    }
+    load_query_tmem<KV8>(a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0),
+                         lane_base, a.err);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -594,7 +633,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if constexpr (KV8) {
         // e4m3 rows of 576 bytes: a lane loads all its 8-byte pieces (8 dims
         // of each of its 5 chunks of its 4 rows) before it widens them exactly
-        // to bf16 and stores them where the bf16 path's copies land
+        // and stores them where the bf16 path's copies land: the 256 latent
+        // dims as fp16 (the type of P and of the fp16 query, so no later
+        // rewrite), the RoPE dims as bf16 (the type of the RoPE query)
         constexpr int RI = NR / (4 * PRODUCERS);
         uint2 v[RI][MAXCH];
 #pragma unroll
@@ -615,7 +656,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           uint8_t* dst = stage + r * 128 + ((pu ^ (r & 7)) * 16);
 #pragma unroll
           for (int c = 0; c < MAXCH; ++c)
-            *reinterpret_cast<uint4*>(dst + c * CHUNK_T) = e4m3x8_to_bf16x8(v[i][c]);
+            *reinterpret_cast<uint4*>(dst + c * CHUNK_T) =
+                c < 4 ? e4m3x8_to_f16x8(v[i][c]) : e4m3x8_to_bf16x8(v[i][c]);
         }
         fence_proxy_async_smem();      // generic-proxy stores, read by the tensor core
         mbar_arrive(&full[s]);
@@ -667,14 +709,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // converted before tile k waits for its stage.
     for (int k = 0; k < ntiles + 2 && ok; ++k) {
       if (k < NST && k < ntiles) ok = gather(k);
-      if (ok && k >= 2) ok = convert(k - 2);
+      if (!KV8 && ok && k >= 2) ok = convert(k - 2);
       if (ok && k >= NST && k < ntiles) ok = gather(k);
     }
     cp_async_wait<0>();                 // nothing in flight when the CTA retires
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t idesc_s = umma_idesc(1 /*BF16*/, DSA_HEADS, NR);
+      // latent dims: bf16, or fp16 over an FP8 cache; RoPE dims: bf16
+      constexpr uint32_t idesc_s = umma_idesc(KV8 ? 0 /*F16*/ : 1 /*BF16*/, DSA_HEADS, NR);
+      constexpr uint32_t idesc_r = umma_idesc(1 /*BF16*/, DSA_HEADS, NR);
       constexpr uint32_t idesc_pv = umma_idesc(0 /*F16*/, DSA_HEADS, 256, 0, 1);
       bool ok = mbar_wait(q_ready, 0, a.err);
       tc_fence_after();
@@ -700,13 +744,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 2 * rank; kk < 2 * rank + 2; ++kk)
             mma_f16(d, umma_desc_sw128(qra + kk * 32, 1024, 16),
-                    umma_desc_sw128(ta + 4 * CHUNK_T + kk * 32, 1024, 16), idesc_s, 1u);
+                    umma_desc_sw128(ta + 4 * CHUNK_T + kk * 32, 1024, 16), idesc_r, 1u);
           mma_commit(&s_full[sb]);
         }
         if (u >= 1) {
           const int t = u - 1, pbuf = t & 1, s = t % NST;
           if (!(ok = mbar_wait(&p_full[pbuf], (t >> 1) & 1, a.err))) break;
-          if (!(ok = mbar_wait(&v_ready[s], (t / NST) & 1, a.err))) break;
+          if (!KV8 && !(ok = mbar_wait(&v_ready[s], (t / NST) & 1, a.err))) break;
           fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t pa = tmem + S_COL + pbuf * NR;   // P (fp16 pairs) in cols [0,32)
@@ -725,7 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
     }
   } else if constexpr (NH == 64) {
-    softmax_dup64(a, maps, smem, tmem, layer, q, split, gu, ntiles, nrows, crd, xb, mx, s_full,
+    softmax_dup64<KV8>(a, maps, smem, tmem, layer, q, split, gu, ntiles, nrows, crd, xb, mx, s_full,
                   p_full, slot_free, x_full, x_free, o_final, q_ready, warp, lane, tid, rank);
   } else {
     // ------------------------------------------------------------ softmax
@@ -743,22 +787,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // the peer's shared memory with st.async and reads the peer's from its own
     if (g == 0) {
       if (live) {
-        // head h's 256 latent query dims of this CTA -> tensor memory (bf16 pairs)
-        const uint4* src = reinterpret_cast<const uint4*>(
-            a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0));
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float w[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 v = __ldg(src + c * 8 + i);
-            w[4 * i + 0] = __uint_as_float(v.x);
-            w[4 * i + 1] = __uint_as_float(v.y);
-            w[4 * i + 2] = __uint_as_float(v.z);
-            w[4 * i + 3] = __uint_as_float(v.w);
-          }
-          tmem_st32(lane_base + Q_COL + c * 32, w);
-        }
+        // head h's 256 latent query dims of this CTA -> tensor memory
+        load_query_tmem<KV8>(
+            a.q[layer] + (static_cast<size_t>(q) * NH + h) * DSA_DIM + (rank ? 256 : 0), lane_base,
+            a.err);
         tmem_st_wait();
         tc_fence_before();
       }

@@ -1,8 +1,11 @@
 """Sparse MLA over an FP8 (e4m3) latent cache with one per-tensor scale (the
 deploy page's fp8_e4m3 KV cache, "GLM-5.2 推理部署").  Parity with the oracle,
 which decodes the codes exactly and multiplies by the scale; and, with scale
-1, bitwise equality with the bf16 call on the exactly widened cache (the
-kernel widens on chip to the same bf16 tiles)."""
+1, bitwise equality with the bf16 call on the exactly widened cache.  Over an
+FP8 cache the kernel widens the latent dims on chip to fp16 (exact) and takes
+the query's latent dims as fp16, which is exact for every bf16 element that is
+zero or an fp16 normal; the equality case uses such queries.  A query element
+beyond fp16's range is flagged as out of range."""
 import numpy as np
 import pytest
 import torch
@@ -53,17 +56,40 @@ def test_fp8_cache_matches_oracle(name, S, kv_scale):
 def test_fp8_cache_equals_bf16_call_on_widened_cache(name):
     inp, codes, idx = _fp8_case(name, 9, None)
     widened = codes.view(torch.float8_e4m3fn).to(torch.bfloat16).contiguous()
+    q = inp.layers[0]["q"].clone()
+    q[q.abs() < 2.0 ** -14] = 0               # fp16 subnormals would be rounded
+    assert (q != 0).float().mean() > 0.99
     res = []
     for fp8 in (True, False):
         out = torch.empty(inp.Q, inp.heads, 512, device=DEV)
         lse = torch.empty(inp.Q, inp.heads, device=DEV)
         ws = dsa.workspace(inp.Q, 1, 2048, 2)
         if fp8:
-            dsa.dsa_sparse_mla_decode_fp8(inp.layers[0]["q"], codes, 1.0, inp.page_table, inp.q_offsets,
+            dsa.dsa_sparse_mla_decode_fp8(q, codes, 1.0, inp.page_table, inp.q_offsets,
                                           inp.q_vis, idx, inp.B, inp.scale, out, lse, ws, num_splits=2)
         else:
-            dsa.dsa_sparse_mla_decode(inp.layers[0]["q"], widened, inp.page_table, inp.q_offsets,
+            dsa.dsa_sparse_mla_decode(q, widened, inp.page_table, inp.q_offsets,
                                       inp.q_vis, idx, inp.B, inp.scale, out, lse, ws, num_splits=2)
         dsa.dsa_check_error(ws)
         res.append((out, lse))
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+
+
+@pytest.mark.parametrize("name", ["decode_b32_ctx128k", "glm52_decode_b32_ctx128k"])
+def test_fp8_cache_flags_query_beyond_f16_range(name):
+    inp, codes, idx = _fp8_case(name, 11, None)
+    q = inp.layers[0]["q"].clone()
+    ws = dsa.workspace(inp.Q, 1, 2048, 1)
+    out = torch.empty(inp.Q, inp.heads, 512, device=DEV)
+    lse = torch.empty(inp.Q, inp.heads, device=DEV)
+    q[1, 3, 100] = 65280.0                    # fp16 holds it: no flag
+    dsa.dsa_sparse_mla_decode_fp8(q, codes, 1.0, inp.page_table, inp.q_offsets, inp.q_vis, idx,
+                                  inp.B, inp.scale, out, lse, ws, num_splits=1)
+    dsa.dsa_check_error(ws)
+    q[1, 3, 300] = -65536.0                   # the next bf16 value: beyond fp16
+    dsa.dsa_sparse_mla_decode_fp8(q, codes, 1.0, inp.page_table, inp.q_offsets, inp.q_vis, idx,
+                                  inp.B, inp.scale, out, lse, ws, num_splits=1)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.dsa_check_error(ws)
+    assert e.value.status == 4
+    dsa.dsa_check_error(ws)                   # the flag was cleared
