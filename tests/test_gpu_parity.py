@@ -23,18 +23,17 @@ def _e4m3(x: torch.Tensor) -> torch.Tensor:
 
 
 # ------------------------------------------------------------------ indexer
-# indexer heads: 64 (DeepSeek-V3.2) and 32 (GLM-5.2)
-@pytest.mark.parametrize("T,first_only,hi", [(1, False, 64), (8, False, 64), (8, True, 64),
-                                             (1, False, 32), (8, False, 32), (8, True, 32)])
-def test_indexer_scores_match_oracle(T, first_only, hi):
-    torch.manual_seed(0)
+def _indexer_case(counts, first_only, hi, seed=0):
+    """Scores of sequences of lengths `lens` with counts[b] queries each (an MTP
+    verify sequence's position t sees all but its last counts[b]-1-t keys)."""
+    torch.manual_seed(seed)
     lens = [1000, 300, 129, 4096 + 77]
     B = len(lens)
-    Q = B * T
+    Q = int(sum(counts))
     seq_off = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int64, device=DEV)
-    q_off = torch.arange(B + 1, dtype=torch.int32, device=DEV) * T
-    vis = torch.tensor([lens[b] - (T - 1 - t) for b in range(B) for t in range(T)],
-                       dtype=torch.int32, device=DEV)
+    q_off = torch.tensor([0] + list(np.cumsum(counts)), dtype=torch.int32, device=DEV)
+    pos = [(b, t) for b in range(B) for t in range(counts[b])]
+    vis = torch.tensor([lens[b] - (counts[b] - 1 - t) for b, t in pos], dtype=torch.int32, device=DEV)
     k = _e4m3(torch.randn(int(sum(lens)), 128, device=DEV))
     qi = _e4m3(torch.randn(Q, hi, 128, device=DEV))
     w = torch.randn(Q, hi, device=DEV) / 8
@@ -49,8 +48,7 @@ def test_indexer_scores_match_oracle(T, first_only, hi):
     kb, qb, wb = np_bits(k), np_bits(qi), w.cpu().numpy()
     so = seq_off.cpu().numpy()
     vv = vis.cpu().numpy()
-    for q in range(Q):
-        b, t = divmod(q, T)
+    for q, (b, t) in enumerate(pos):
         if first_only and t > 0:
             assert np.isnan(sc[q]).all()
             continue
@@ -64,6 +62,19 @@ def test_indexer_scores_match_oracle(T, first_only, hi):
         bad = np.abs(got - ref) > tol
         assert not bad.any(), (q, np.flatnonzero(bad)[:5], got[bad][:5], ref[bad][:5])
         assert np.isnan(sc[q, vv[q]:]).all()
+
+
+# indexer heads: 64 (DeepSeek-V3.2) and 32 (GLM-5.2)
+@pytest.mark.parametrize("T,first_only,hi", [(1, False, 64), (8, False, 64), (8, True, 64),
+                                             (1, False, 32), (8, False, 32), (8, True, 32)])
+def test_indexer_scores_match_oracle(T, first_only, hi):
+    _indexer_case([T] * 4, first_only, hi)
+
+
+# several queries a sequence with odd counts: a pair's second query is absent
+@pytest.mark.parametrize("hi", [64, 32])
+def test_indexer_scores_ragged_queries_per_sequence(hi):
+    _indexer_case([3, 8, 1, 5], False, hi, seed=1)
 
 
 # ------------------------------------------------------------------ selector
