@@ -228,9 +228,14 @@ dsa_status dsa_indexer_topk_fused(const uint8_t* q_idx, const float* w, const ui
  * slot beyond max_pages are skipped and flagged (DSA_ERR_DEVICE_BOUNDS).
  * Precision: bf16 products accumulate in fp32 on the tensor cores.  Each
  * score is the sum of two partial dot products (latent dims split between a
- * pair of SMs); one partial crosses to the other SM rounded to a 24-bit
- * float (15 mantissa bits), which moves O by well under 1e-3 of its RMS.  P
- * enters the value product as a bf16 high + low pair (~16 significant bits).
+ * pair of SMs); each partial crosses between them as 16-bit integer codes
+ * with one fp32 scale per 32 values (error at most 1/65520 of the block's
+ * largest magnitude), which moves O by well under 1e-3 of its RMS.  The value
+ * product takes P as fp16 (11 significant bits, relative to a running
+ * maximum) and the 512 value dims as fp16, rewritten on chip from bf16:
+ * exact for magnitudes 2^-14 .. 65504, rounded to fp16's spacing 2^-24 below.
+ * Latent values of magnitude 65536 or more do not fit fp16 and are not
+ * flagged: the call takes latents inside fp16's range.
  * ws: at least dsa_workspace_bytes(Q, 1, topk, num_splits) bytes.
  */
 dsa_status dsa_sparse_mla_decode(const void* q, const void* kv_pool, int num_pages, int page_size,
